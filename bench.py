@@ -1,0 +1,547 @@
+#!/usr/bin/env python
+"""Benchmark of the ParisKV decode-time retrieval path on B200.
+
+One *step* = pk_search + pk_attend for every (sequence, KV head) pair of one
+decoder layer: query preparation, collision scan, candidate compaction +
+4-bit rerank + Top-k, and gather + exact attention, on a fresh query.
+
+Default workload (the metric's 128K point): 8 sequences x n = 131072 keys,
+8 KV heads, 32 query heads, head_dim 128, bf16 K/V in HBM, Top-100, ratio-table
+budgets.  The line also carries the metric's 1M point (n = 1048576, 8 KV
+heads, K/V in pinned host memory read through UVA) under "million_token".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload throughput|million|llama|tiny] [--no-million]
+                  [--no-cpu-baseline] [--no-e2e] [--no-dense]
+
+For N > 1 launch under torch.distributed.run: every rank runs its own copy of
+the workload (pairs shard with no data-path collective: weak scaling); the
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("retrieval+attend steps/sec per layer (all KV heads) at 128K and 1M; "
+          "HBM % peak; Recall@100")
+L2_BYTES = 126 * 1024 * 1024
+FLUSH_BYTES = 256 * 1024 * 1024
+
+WORKLOADS = {
+    "throughput": dict(name="throughput_8x131072", batch=8, n=131072, H=8, G=4, cand=0, kv_host=False),
+    "million": dict(name="million_1x1048576_uva", batch=1, n=1 << 20, H=8, G=4, cand=0, kv_host=True),
+    "llama": dict(name="llama_1x32768", batch=1, n=32768, H=8, G=4, cand=2048, kv_host=False),
+    "tiny": dict(name="tiny_1x4096", batch=1, n=4096, H=1, G=1, cand=512, kv_host=False),
+}
+
+
+# ----------------------------------------------------------------- helpers
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="throughput", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-million", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (of measured)"
+    return 6650.0, "fallback 6.65 TB/s (of fallback)"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "utilization.gpu")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="pk_clocks_", suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "50"]
+            if self.uuid:
+                cmd += ["--id=" + self.uuid]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower().startswith("active")})
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        loaded = [r for r in rows if (num(r[8]) or 0) > 0] or rows
+        sm = [num(r[0]) for r in loaded if num(r[0]) is not None]
+        mx = [num(r[1]) for r in rows if num(r[1]) is not None]
+        pw = [num(r[2]) for r in loaded if num(r[2]) is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows),
+                "samples_under_load": len(loaded)}
+
+
+def src_hash(*names):
+    h = hashlib.sha256()
+    for nm in names:
+        with open(os.path.join(ROOT, "kv_cache_top_b200", "csrc", nm), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary in
+    profiles/, or None when there is none or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", txt)
+    hm = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
+    files = {"collision_scan": ["k_collision_scan.cu", "pk_internal.cuh"],
+             "rerank_topk": ["k_rerank_topk.cu", "pk_internal.cuh"],
+             "query_prep": ["k_query_prep.cu", "pk_internal.cuh"],
+             "gather_attend": ["k_gather_attend.cu", "pk_internal.cuh"]}.get(kernel)
+    if not m or not hm or not files or hm.group(1) != src_hash(*files):
+        return None
+    return float(m.group(1))
+
+
+# -------------------------------------------------------- algorithmic bytes
+def alg_bytes(kernel: str, wl: dict, C: int, topk: int = 100):
+    """Bytes a launch must move at minimum (per launch, all pairs)."""
+    bh, n, G = wl["batch"] * wl["H"], wl["n"], wl["G"]
+    if kernel == "query_prep":
+        return bh * (G * 128 * 2 + 16 * 256 * 4 + 16 * 32 * 4 + 128 * 4)
+    if kernel == "collision_scan":
+        return bh * (16 * n + n)                     # codes read + S written
+    if kernel == "rerank_topk":
+        return bh * (n + 128 * C + 8 * topk)         # S read + candidate records + result
+    if kernel == "gather_attend":
+        return bh * (2 * topk * 128 * 2 + G * 128 * (2 + 4))   # K/V rows + q + o
+    raise KeyError(kernel)
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
+    import torch
+    import kv_cache_top_b200 as pk
+    import workloads
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    seed = args.seed + rank
+    batch, n, H, G = wl["batch"], wl["n"], wl["H"], wl["G"]
+    bh, topk, nq = batch * H, 100, 64
+    w = workloads.llama_layer(batch, n, H=H, G=G, seed=seed, device=dev, n_queries=nq)
+    p = pk.pk_default_params(batch=batch, n_kv_heads=H, group=G, topk=topk, cand_budget=wl["cand"],
+                             kv_dtype=pk.PK_BF16,
+                             kv_location=pk.PK_KV_HOST_PINNED if wl["kv_host"] else pk.PK_KV_DEVICE)
+    stream = torch.cuda.current_stream()
+    h = pk.pk_build_index(w["K"], w["V"], n, p)
+    torch.cuda.synchronize()
+    C, R = pk.pk_resolve(n, wl["cand"], 0.0, topk)
+    info = pk.pk_get_info(h)
+    q = w["q"]
+    idx = torch.empty(bh, topk, dtype=torch.int32, device=dev)
+    score = torch.empty(bh, topk, dtype=torch.float32, device=dev)
+    out = torch.empty(batch, H * G, 128, dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    # Recall@100 against exact Top-100 of <k_i, q_agg> (fp32 matmul, metric only)
+    recalls = []
+    for qi in range(4):
+        pk.pk_search(h, q[qi], topk, idx, score)
+        got = idx.cpu()
+        qa = q[qi].float().view(batch, H, G, 128).sum(2)                     # [batch][H][D]
+        for b in range(batch):
+            for hh in range(H):
+                s = w["K"][b, hh].float() @ qa[b, hh]
+                ex = torch.topk(s, topk).indices.cpu()
+                recalls.append(len(set(ex.tolist()) & set(got[b * H + hh].tolist())) / topk)
+    recall = sum(recalls) / len(recalls)
+    if wl["kv_host"]:
+        del w["K"], w["V"]
+        torch.cuda.empty_cache()
+
+    def step(i):
+        pk.pk_search(h, q[i % nq], topk, idx, score)
+        pk.pk_attend(h, q[i % nq], idx, topk, out)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(None)
+    if rank == 0:
+        try:
+            sampler.uuid = str(torch.cuda.get_device_properties(dev).uuid)
+            if not sampler.uuid.startswith("GPU-"):
+                sampler.uuid = "GPU-" + sampler.uuid
+        except Exception:
+            sampler.uuid = None
+        sampler.start()
+        time.sleep(0.3)
+
+    def timed_pass(trace: bool):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        if trace:
+            pk.pk_trace_enable(h, True)
+            pk.pk_trace_read(h)
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()                      # L2 flush outside the timed events
+            evs[i][0].record(stream)
+            step(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+        if world > 1:
+            torch.distributed.barrier()
+        ms = sum(a.elapsed_time(b) for a, b in evs)
+        kern = None
+        if trace:
+            kern = pk.pk_trace_read(h)
+            pk.pk_trace_enable(h, False)
+        return ms, wall, kern
+
+    ms_clean, wall_clean, _ = timed_pass(False)
+    ms_traced, _, kern = timed_pass(True)
+
+    # end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        q_host = q.cpu().pin_memory()
+        q_dev = torch.empty_like(q[0])
+        o_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        i_host = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+        ks = min(args.steps, 500)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(ks)]
+        torch.cuda.synchronize()
+        for i in range(ks):
+            flush.zero_()
+            evs[i][0].record(stream)
+            q_dev.copy_(q_host[i % nq], non_blocking=True)
+            pk.pk_search(h, q_dev, topk, idx, score)
+            pk.pk_attend(h, q_dev, idx, topk, out)
+            o_host.copy_(out, non_blocking=True)
+            i_host.copy_(idx, non_blocking=True)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in evs) / ks
+        e2e = {"value": 1000.0 / e2e_ms, "unit": "steps/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": q_dev.numel() * q_dev.element_size(),
+               "d2h_bytes_per_step": out.numel() * 4 + idx.numel() * 4}
+
+    clocks = sampler.stop() if rank == 0 else None
+
+    # max over ranks of the device time
+    if world > 1:
+        t = torch.tensor([ms_clean], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_clean = float(t.item())
+
+    res = dict(ms_total=ms_clean, wall=wall_clean, kern=kern, recall=recall, C=C, R=R, info=info,
+               e2e=e2e, clocks=clocks, ms_traced=ms_traced)
+
+    # dense-attention comparator on the same tensors (HBM workloads only)
+    if rank == 0 and not wl["kv_host"] and not args.no_dense:
+        try:
+            import torch.nn.functional as F
+            qd = q[0].view(batch, H * G, 1, 128)
+            Kd, Vd = w["K"], w["V"]
+            for _ in range(3):
+                F.scaled_dot_product_attention(qd, Kd, Vd, enable_gqa=True)
+            torch.cuda.synchronize()
+            ds = []
+            for _ in range(10):
+                flush.zero_()
+                a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a_.record(stream)
+                F.scaled_dot_product_attention(qd, Kd, Vd, enable_gqa=True)
+                b_.record(stream)
+                torch.cuda.synchronize()
+                ds.append(a_.elapsed_time(b_))
+            dms = statistics.median(ds)
+            res["dense"] = {"kind": "torch SDPA over all n keys (same K/V, same queries)",
+                            "ms_per_step": dms, "steps_s": 1000.0 / dms,
+                            "bytes_per_step": 2 * bh * n * 128 * 2,
+                            "gbs": 2 * bh * n * 128 * 2 / dms / 1e6}
+        except Exception as e:                  # comparator only; never the product
+            res["dense"] = {"error": str(e)[:200]}
+
+    # host-link reference (pinned H2D copy) for UVA workloads
+    if rank == 0 and wl["kv_host"]:
+        hb = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+        db = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        best = 1e9
+        for _ in range(5):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            db.copy_(hb, non_blocking=True)
+            b_.record(stream)
+            torch.cuda.synchronize()
+            best = min(best, a_.elapsed_time(b_))
+        res["h2d_gbs"] = (256 << 20) / best / 1e6
+        del hb, db
+
+    # CPU baseline: the oracle on a bounded sample of the same workload
+    if want_cpu:
+        res["cpu"] = cpu_baseline(wl, seed, w if not wl["kv_host"] else None, dev)
+
+    pk.pk_free(h)
+    del w, flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def cpu_baseline(wl, seed, w, dev, pairs_wanted=4, queries=32):
+    """Time the oracle (as it stands, 1 thread) on sampled pairs of the same
+    workload: index build untimed, then search + attend per query."""
+    import torch
+    import oracle
+    import workloads
+    batch, n, H, G = wl["batch"], wl["n"], wl["H"], wl["G"]
+    bh = batch * H
+    pairs = sorted({(i * bh) // pairs_wanted for i in range(pairs_wanted)})
+    if n > 200000:
+        pairs, queries = pairs[:1], 8
+    tot, cnt = 0.0, 0
+    for pidx in pairs:
+        b, hh = divmod(pidx, H)
+        K, V, qq = workloads.llama_pair(b, hh, n, H=H, G=G, seed=seed, device=dev, n_queries=queries)
+        Kn, Vn, qn = workloads.to_np_f32(K), workloads.to_np_f32(V), workloads.to_np_f32(qq)
+        del K, V, qq
+        enc = oracle.build_index(Kn)
+        for i in range(queries):
+            t0 = time.perf_counter()
+            o = oracle.search(enc, qn[i], topk_k=100, cand_budget=wl["cand"])
+            oracle.attend(qn[i], Kn, Vn, o["idx"], 1.0 / math.sqrt(128))
+            tot += time.perf_counter() - t0
+            cnt += 1
+    per_pair = tot / cnt
+    return {"value": 1.0 / (per_pair * bh), "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "sample": "%d of %d (sequence, KV head) pairs x %d queries each (%.1f s of timed "
+                      "search+attend, index build untimed); one step = %d pair-searches" %
+                      (len(pairs), bh, queries, tot, bh),
+            "ms_per_pair": per_pair * 1000.0}
+
+
+def kernel_table(kern, steps, wl, C, peak):
+    tot = sum(v[1] for v in kern.values()) or 1.0
+    out = {}
+    for k, (nl, ms) in kern.items():
+        if nl == 0:
+            continue
+        avg_ms = ms / nl
+        ab = alg_bytes(k, wl, C)
+        out[k] = {"launches": nl, "avg_us": avg_ms * 1000.0, "share": ms / tot,
+                  "alg_bytes_per_launch": ab, "gbs": ab / avg_ms / 1e6, "hbm_frac": ab / avg_ms / 1e6 / peak}
+    return out
+
+
+def main():
+    args = parse_args()
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    peak, peak_src = load_peaks()
+    wl = WORKLOADS[args.workload]
+    want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
+    res = run_ours(args, wl, rank, world, local_rank, want_cpu, peak)
+
+    mil = None
+    if args.workload == "throughput" and not args.no_million:
+        wl_m = WORKLOADS["million"]
+        margs = argparse.Namespace(**vars(args))
+        margs.steps = min(args.steps, 500)
+        margs.no_e2e = True
+        rm = run_ours(margs, wl_m, rank, world, local_rank, want_cpu, peak)
+        km = kernel_table(rm["kern"], margs.steps, wl_m, rm["C"], peak)
+        link_bytes = wl_m["batch"] * wl_m["H"] * 100 * 2 * 128 * 2
+        att = km.get("gather_attend", {})
+        mil = {"workload": wl_m["name"], "steps_s": margs.steps * world / (rm["ms_total"] / 1000.0),
+               "ms_per_step": rm["ms_total"] / margs.steps, "steps": margs.steps,
+               "search_us": sum(km[k]["avg_us"] for k in ("query_prep", "collision_scan", "rerank_topk") if k in km),
+               "attend_us": att.get("avg_us"), "recall_at_100": rm["recall"],
+               "uva_bytes_per_step": link_bytes,
+               "host_link_gbs": (link_bytes / (att["avg_us"] * 1e-6) / 1e9) if att else None,
+               "h2d_copy_gbs": rm.get("h2d_gbs"),
+               "host_link_frac_of_h2d_copy": ((link_bytes / (att["avg_us"] * 1e-6) / 1e9) / rm["h2d_gbs"])
+               if att and rm.get("h2d_gbs") else None,
+               "kernels": km, "cand_budget": rm["C"], "collision_budget": rm["R"],
+               "cpu_baseline": rm.get("cpu")}
+        if world > 1:
+            pass
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    km = kernel_table(res["kern"], args.steps, wl, res["C"], peak)
+    dom = max(km, key=lambda k: km[k]["share"])
+    step_bytes = sum(alg_bytes(k, wl, res["C"]) for k in km)
+    ms_per_step = res["ms_total"] / args.steps
+    value = args.steps * world / (res["ms_total"] / 1000.0)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl["name"], "batch": wl["batch"], "n": wl["n"], "kv_heads": wl["H"],
+                   "q_heads": wl["H"] * wl["G"], "head_dim": 128, "topk": 100,
+                   "cand_budget": res["C"], "collision_budget": res["R"],
+                   "kv_location": "pinned host (UVA)" if wl["kv_host"] else "hbm",
+                   "kv_dtype": "bf16", "index": "16 B codes + 128 B 4-bit record per key",
+                   "l2": "flushed between timed steps (256 MiB write outside the events)",
+                   "queries": "fresh query per step from a 64-query pool",
+                   "parallelism": "replicas: each rank its own %d pairs" % (wl["batch"] * wl["H"])},
+        "recall_at_100": res["recall"],
+        "hbm": {"alg_bytes_per_step": step_bytes, "gbs": step_bytes / ms_per_step / 1e6,
+                "frac": step_bytes / ms_per_step / 1e6 / peak},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": km[dom]["gbs"], "peak": peak,
+                     "unit": "GB/s", "frac": km[dom]["gbs"] / peak,
+                     "traffic": profiled_traffic(dom, wl["name"]), "peak_source": peak_src},
+        "kernels": km,
+        "gpu_launches": 4 * args.steps,
+        "clocks": res["clocks"],
+        "e2e": res["e2e"],
+        "cpu_baseline": res.get("cpu"),
+        "wall_s_timed_region": res["wall"],
+        "ms_per_step_traced": res["ms_traced"] / args.steps,
+    }
+    if "dense" in res:
+        line["dense_attention"] = res["dense"]
+    if mil is not None:
+        line["million_token"] = mil
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    """The reference arm is the CPU oracle as it stands (1 thread): each step
+    is one sampled (sequence, KV head) pair searched and attended; the value
+    extrapolates to whole steps of the same workload."""
+    if rank != 0:
+        return
+    import torch
+    import oracle
+    import workloads
+    wl = WORKLOADS[args.workload]
+    batch, n, H, G = wl["batch"], wl["n"], wl["H"], wl["G"]
+    bh = batch * H
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    npairs = 2 if n <= 200000 else 1
+    nq = 16
+    data = []
+    for i in range(npairs):
+        pidx = (i * bh) // npairs
+        b, hh = divmod(pidx, H)
+        K, V, qq = workloads.llama_pair(b, hh, n, H=H, G=G, seed=args.seed, device=dev, n_queries=nq)
+        Kn, Vn, qn = workloads.to_np_f32(K), workloads.to_np_f32(V), workloads.to_np_f32(qq)
+        data.append((oracle.build_index(Kn), Kn, Vn, qn))
+
+    def one(i):
+        enc, Kn, Vn, qn = data[i % npairs]
+        o = oracle.search(enc, qn[(i // npairs) % nq], topk_k=100, cand_budget=wl["cand"])
+        oracle.attend(qn[(i // npairs) % nq], Kn, Vn, o["idx"], 1.0 / math.sqrt(128))
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    dt = time.perf_counter() - t0
+    per_pair = dt / args.steps
+    value = 1.0 / (per_pair * bh)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_pair * bh * 1000.0,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl["name"], "batch": batch, "n": n, "kv_heads": H, "q_heads": H * G,
+                       "head_dim": 128, "topk": 100},
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                             "sample": "each timed step = one of %d sampled pairs (search + attend); "
+                                       "value = 1 / (mean pair time x %d pairs)" % (npairs, bh)},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

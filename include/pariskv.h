@@ -1,0 +1,215 @@
+/*
+ * pariskv.h -- C-ABI of the B200 (sm_100a) ParisKV decode-time KV-cache
+ * retrieval library (libpariskv.so).
+ *
+ * What the library computes (citations are to two public pages: the
+ * "ParisKV" GitHub README of amy-77/ParisKV, called [readme] below, and the
+ * slide deck "ParisKV: Fast and Drift-Robust KV-Cache Retrieval" reading of
+ * arXiv 2602.07721v3, called [slides]):
+ *
+ *   pk_build_index  prefill: normalise + SRHT-rotate every key, split it into
+ *                   B = D/m blocks, store the sign-pattern centre id of each
+ *                   block (PolarANN codes) and the 4-bit RSQ-IP summary (1 sign
+ *                   bit + 3-bit Lloyd-Max magnitude index per coordinate, one
+ *                   fp32 weight per block) on the GPU; copy K/V into
+ *                   index-owned storage in HBM or pinned host memory.
+ *                   [readme] "Prefill: build compact retrieval metadata";
+ *                   [slides] Eqs. (5)-(10).
+ *   pk_append       index newly decoded keys with the same fixed codebook
+ *                   ([slides] "new decode keys can be indexed without
+ *                   retraining centroids").
+ *   pk_search       per (sequence, KV head): GQA-aggregate and rotate the
+ *                   query, rank the sign-pattern buckets of every block, give
+ *                   buckets inside the top-rho fraction one of six tier
+ *                   bonuses 6..1, sum them into collision scores S_i
+ *                   ([slides] Sec. 4.2.2, App. B.2.1 Eq. 15), keep the top
+ *                   C = ceil(beta n) keys by S ([slides] Sec. 4.3), rerank
+ *                   them with the 4-bit estimator ([slides] Eqs. 7-10) and
+ *                   return the final Top-k indices.
+ *   pk_attend       exact softmax attention of every query head over the
+ *                   selected full-precision K/V rows, read from HBM or, for
+ *                   host-resident K/V, over the host link through UVA
+ *                   ([slides] Sec. 3 Eqs. (1)-(3); [readme] "Attention: fetch
+ *                   only selected KV pairs").
+ *
+ * Conventions for every call:
+ *   - D (head_dim) must be 128 and m (sub_dim) must be 8 (B = 16 blocks of
+ *     256 sign-pattern centres).  Other values return PK_ERR_UNSUPPORTED.
+ *   - Tensors are dense, row-major, and addressed by plain pointers that the
+ *     GPU can dereference: device memory, or pinned/mapped host memory (UVA).
+ *     Pageable host memory is rejected with PK_ERR_INVALID_ARG.
+ *   - "BH" = batch * n_kv_heads; pair bh = b * n_kv_heads + h.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work on it and returns; nothing
+ *     waits for the GPU except pk_last_device_error, pk_trace_read and the
+ *     allocation/free calls.
+ *   - Arguments are checked on the host before any launch; a bad argument
+ *     returns an error status and launches nothing.  Kernels never trap: a
+ *     device-side check that fails (e.g. an out-of-range index given to
+ *     pk_attend) skips the access and records a code read by
+ *     pk_last_device_error.
+ *   - No C++ exception crosses this boundary.  Calls on one index must not
+ *     run concurrently from several host threads or streams (they share the
+ *     index's workspace).
+ */
+#ifndef PARISKV_H
+#define PARISKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PK_OK = 0,
+    PK_ERR_INVALID_ARG = 1,   /* null / misaligned / pageable pointer, bad value */
+    PK_ERR_CAPACITY = 2,      /* n < topk, n + n_new > n_cap, n too large       */
+    PK_ERR_OOM = 3,           /* device or pinned-host allocation failed        */
+    PK_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
+    PK_ERR_TIMEOUT = 5,       /* reserved: a bounded device wait gave up        */
+    PK_ERR_DEVICE_CHECK = 6,  /* a device-side check recorded a bad value       */
+    PK_ERR_UNSUPPORTED = 7    /* head_dim != 128, sub_dim != 8, topk > 1024     */
+} pk_status;
+
+typedef enum { PK_F32 = 0, PK_BF16 = 1 } pk_dtype;
+typedef enum { PK_KV_DEVICE = 0, PK_KV_HOST_PINNED = 1 } pk_kv_location;
+
+/* Index parameters.  [readme] parameter table: final_topk, enable_offload;
+ * adaptive ratio table for beta (candidate ratio) and rho (collision ratio). */
+typedef struct {
+    int32_t batch;            /* sequences                                     */
+    int32_t n_kv_heads;       /* H                                             */
+    int32_t group;            /* G query heads per KV head (GQA); >= 1, <= 8   */
+    int32_t head_dim;         /* D, must be 128                                */
+    int32_t sub_dim;          /* m, must be 8                                  */
+    int32_t topk;             /* largest k pk_search / pk_attend accept; <=1024 */
+    int64_t n_cap;            /* keys per (sequence, KV head), appends included */
+    int64_t cand_budget;      /* C; 0 = ceil(beta(n) n) from the ratio table   */
+    float collision_ratio;    /* rho; 0 = ratio table                          */
+    float attn_scale;         /* softmax scale; 0 = 1/sqrt(D)                  */
+    uint64_t rot_seed;        /* seed of the SRHT sign diagonal                */
+    int32_t kv_dtype;         /* pk_dtype of K, V and queries                  */
+    int32_t kv_location;      /* pk_kv_location of the full K/V store          */
+} pk_params;
+
+typedef struct pk_index pk_index;
+
+/* Facts about a built index (host struct filled by pk_get_info). */
+typedef struct {
+    int64_t n;                /* keys per (sequence, KV head) now              */
+    int64_t n_cap;
+    int32_t bh;               /* batch * n_kv_heads                            */
+    int32_t nchunks;          /* key chunks per pair used by pk_search at n    */
+    int64_t chunk;            /* keys per chunk                                */
+    int64_t cand;             /* C at n                                        */
+    int64_t coll;             /* R = ceil(rho n) at n                          */
+    int64_t index_bytes;      /* codes + summaries + occupancy (device)        */
+    int64_t kv_bytes;         /* full K/V store (device or pinned host)        */
+    int32_t kv_location;
+    int32_t num_sms;
+} pk_info;
+
+/* Optional intermediate outputs of pk_search_debug (device pointers; any may
+ * be NULL).  Layouts: qt [BH][D] f32; qnorm [BH] f32; bonus [BH][16][256] u8;
+ * S [BH][n] u8; hist [BH][97] u32 (count of S = s); sstar [BH] i32 (the S
+ * threshold); cand [BH][C] i32 (candidate ids in ascending order); cand_est
+ * [BH][C] f32 (the 4-bit estimate of cand[.]). */
+typedef struct {
+    float *qt;
+    float *qnorm;
+    uint8_t *bonus;
+    uint8_t *S;
+    uint32_t *hist;
+    int32_t *sstar;
+    int32_t *cand;
+    float *cand_est;
+} pk_debug_out;
+
+/* Fill *p with defaults: batch 1, H 8, G 4, D 128, m 8, topk 100, n_cap 0,
+ * ratio-table C and rho, scale 1/sqrt(D), seed 0, bf16, K/V in HBM. */
+void pk_default_params(pk_params *p);
+
+/* Build an index over n keys per pair.
+ *   K, V   [BH][n][D] of kv_dtype (device or pinned host pointers; copied in).
+ *   n      1 <= n <= n_cap (n_cap 0 means n).
+ * On success *out owns: codes [BH][n_cap][16] u8, summary records
+ * [BH][n_cap][128 B], occupancy [BH][16][256] u32, search workspace, and the
+ * K/V store [BH][n_cap][D] (HBM, or cudaHostAlloc'd mapped host memory).
+ * Errors: PK_ERR_INVALID_ARG, PK_ERR_UNSUPPORTED, PK_ERR_CAPACITY,
+ * PK_ERR_OOM (nothing leaks), PK_ERR_CUDA. */
+pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_params *params,
+                         void *stream, pk_index **out);
+
+/* Append n_new keys/values per pair: k_new, v_new [BH][n_new][D] kv_dtype.
+ * Encodes them at positions n .. n+n_new-1 and updates the occupancy table.
+ * PK_ERR_CAPACITY when n + n_new > n_cap (nothing is written). */
+pk_status pk_append(pk_index *index, const void *k_new, const void *v_new, int64_t n_new,
+                    void *stream);
+
+/* Retrieve the Top-k keys of every pair for one decode step.
+ *   q          [batch][H*G][D] kv_dtype; query head j belongs to KV head j/G.
+ *   topk       1 <= topk <= params.topk and topk <= n.
+ *   out_idx    [BH][topk] i32 device: key ids, best first (estimate desc, id asc).
+ *   out_score  [BH][topk] f32 device or NULL: the 4-bit estimates.
+ * Ties use one rule everywhere: higher score first, then lower key id. */
+pk_status pk_search(pk_index *index, const void *q, int32_t topk, int32_t *out_idx,
+                    float *out_score, void *stream);
+
+/* pk_search that also writes the intermediates named in *dbg (may be NULL). */
+pk_status pk_search_debug(pk_index *index, const void *q, int32_t topk, int32_t *out_idx,
+                          float *out_score, const pk_debug_out *dbg, void *stream);
+
+/* Exact attention over the selected rows.
+ *   q        [batch][H*G][D] kv_dtype (the un-aggregated query heads).
+ *   sel_idx  [BH][topk] i32 device; ids outside [0, n) are skipped and recorded
+ *            as PK_ERR_DEVICE_CHECK (see pk_last_device_error).
+ *   out      [batch][H*G][D] f32 device (or mapped host):
+ *            o_g = sum_r softmax_r(scale <q_g, K[sel_r]>) V[sel_r]. */
+pk_status pk_attend(pk_index *index, const void *q, const int32_t *sel_idx, int32_t topk,
+                    float *out, void *stream);
+
+/* Free everything the index owns (synchronises the device first). NULL is ok. */
+void pk_free(pk_index *index);
+
+/* Static description of a status code. */
+const char *pk_status_str(pk_status s);
+
+/* Wait for the device, then return and clear the index's device-check word:
+ * PK_OK, or PK_ERR_DEVICE_CHECK with *detail (nullable) set to the first bad
+ * value seen (e.g. the out-of-range key id). */
+pk_status pk_last_device_error(pk_index *index, int64_t *detail);
+
+pk_status pk_get_info(const pk_index *index, pk_info *info);
+
+/* Copy the index's codes [BH][n][16] u8, records [BH][n][128] u8 and occupancy
+ * [BH][16][256] u32 into caller device buffers (any may be NULL). */
+pk_status pk_export_index(const pk_index *index, uint8_t *codes, uint8_t *records,
+                          uint32_t *occ, void *stream);
+
+/* The fp32 Lloyd-Max magnitude levels (L of them) and midpoints (L-1) of the
+ * prior y = |u_j|, (u_j)^2 ~ Beta(1/2, (m-1)/2) ([slides] Prop. 4.1 /
+ * App. B.1), computed on the host; the index uses m = 8, L = 8. */
+pk_status pk_magnitude_levels(int32_t m, int32_t L, float *levels, float *thresholds);
+
+/* Budgets for a retrieval zone of n keys ([readme] ratio table):
+ * C = cand_budget or ceil(beta n), then min(max(C, topk), n);
+ * R = ceil(rho n) clamped to [1, n], rho = collision_ratio or the table's. */
+pk_status pk_resolve(int64_t n, int64_t cand_budget, float collision_ratio, int32_t topk,
+                     int64_t *C, int64_t *R);
+
+/* Per-kernel timing.  While tracing is on, the library records a CUDA event
+ * pair on the launching stream around each of its kernels.  pk_trace_read
+ * synchronises, then returns per kernel kind (0 encode, 1 query_prep,
+ * 2 collision_scan, 3 rerank_topk, 4 gather_attend) the launch count and the
+ * summed event time in ms; it clears the record. */
+enum { PK_K_ENCODE = 0, PK_K_QUERY_PREP = 1, PK_K_COLLISION_SCAN = 2, PK_K_RERANK_TOPK = 3,
+       PK_K_GATHER_ATTEND = 4, PK_K_COUNT = 5 };
+pk_status pk_trace_enable(pk_index *index, int32_t on);
+pk_status pk_trace_read(pk_index *index, int64_t *launches, double *total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PARISKV_H */

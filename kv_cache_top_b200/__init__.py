@@ -1,0 +1,148 @@
+"""B200 (sm_100a) ParisKV decode-time KV-cache retrieval.
+
+A thin binding over ``libpariskv.so`` (C-ABI in ``include/pariskv.h``): the
+functions below have the C names and only marshal arguments (tensor data
+pointers, the current CUDA stream).  Every step of the path runs in the
+library's CUDA kernels; PyTorch supplies device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+
+from . import _lib
+from ._lib import (KERNELS, PK_BF16, PK_F32, PK_KV_DEVICE, PK_KV_HOST_PINNED, PK_OK, pk_debug_out,
+                   pk_info, pk_params)
+
+lib = _lib.load()
+
+__all__ = [
+    "PkError", "pk_default_params", "pk_build_index", "pk_append", "pk_search", "pk_search_debug",
+    "pk_attend", "pk_free", "pk_status_str", "pk_last_device_error", "pk_get_info",
+    "pk_export_index", "pk_magnitude_levels", "pk_resolve", "pk_trace_enable", "pk_trace_read",
+    "pk_params", "pk_info", "pk_debug_out", "PK_F32", "PK_BF16", "PK_KV_DEVICE",
+    "PK_KV_HOST_PINNED", "KERNELS", "lib",
+]
+
+
+class PkError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (what, pk_status_str(status), status))
+
+
+def _check(status: int, what: str):
+    if status != PK_OK:
+        raise PkError(status, what)
+
+
+def _ptr(x):
+    """Data pointer of a tensor (or an int address, or None)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def pk_status_str(status: int) -> str:
+    return lib.pk_status_str(status).decode()
+
+
+def pk_default_params(**kw) -> pk_params:
+    p = pk_params()
+    lib.pk_default_params(C.byref(p))
+    for k, v in kw.items():
+        if not hasattr(p, k):
+            raise AttributeError("pk_params has no field %r" % k)
+        setattr(p, k, v)
+    return p
+
+
+def pk_build_index(K, V, n: int, params: pk_params, stream=None) -> C.c_void_p:
+    h = C.c_void_p()
+    _check(lib.pk_build_index(_ptr(K), _ptr(V), int(n), C.byref(params), _stream(stream), C.byref(h)),
+           "pk_build_index")
+    return h
+
+
+def pk_append(index, k_new, v_new, n_new: int, stream=None):
+    _check(lib.pk_append(index, _ptr(k_new), _ptr(v_new), int(n_new), _stream(stream)), "pk_append")
+
+
+def pk_search(index, q, topk: int, out_idx, out_score=None, stream=None):
+    _check(lib.pk_search(index, _ptr(q), int(topk), _ptr(out_idx), _ptr(out_score), _stream(stream)),
+           "pk_search")
+
+
+def pk_search_debug(index, q, topk: int, out_idx, out_score=None, dbg: dict | None = None,
+                    stream=None):
+    d = pk_debug_out()
+    for k, v in (dbg or {}).items():
+        setattr(d, k, _ptr(v))
+    _check(lib.pk_search_debug(index, _ptr(q), int(topk), _ptr(out_idx), _ptr(out_score), C.byref(d),
+                               _stream(stream)), "pk_search_debug")
+
+
+def pk_attend(index, q, sel_idx, topk: int, out, stream=None):
+    _check(lib.pk_attend(index, _ptr(q), _ptr(sel_idx), int(topk), _ptr(out), _stream(stream)),
+           "pk_attend")
+
+
+def pk_free(index):
+    lib.pk_free(index)
+
+
+def pk_last_device_error(index):
+    """(status, detail): waits for the device, then reads and clears the
+    index's device-check word."""
+    det = C.c_int64(0)
+    st = lib.pk_last_device_error(index, C.byref(det))
+    return st, det.value
+
+
+def pk_get_info(index) -> pk_info:
+    info = pk_info()
+    _check(lib.pk_get_info(index, C.byref(info)), "pk_get_info")
+    return info
+
+
+def pk_export_index(index, codes=None, records=None, occ=None, stream=None):
+    _check(lib.pk_export_index(index, _ptr(codes), _ptr(records), _ptr(occ), _stream(stream)),
+           "pk_export_index")
+
+
+def pk_magnitude_levels(m: int = 8, L: int = 8):
+    lev = np.empty(L, np.float32)
+    thr = np.empty(L - 1, np.float32)
+    _check(lib.pk_magnitude_levels(m, L, lev.ctypes.data, thr.ctypes.data), "pk_magnitude_levels")
+    return lev, thr
+
+
+def pk_resolve(n: int, cand_budget: int = 0, collision_ratio: float = 0.0, topk: int = 100):
+    c = C.c_int64()
+    r = C.c_int64()
+    _check(lib.pk_resolve(n, cand_budget, collision_ratio, topk, C.byref(c), C.byref(r)), "pk_resolve")
+    return c.value, r.value
+
+
+def pk_trace_enable(index, on: bool = True):
+    _check(lib.pk_trace_enable(index, 1 if on else 0), "pk_trace_enable")
+
+
+def pk_trace_read(index):
+    """{kernel: (launches, total_ms)} since the last read (synchronises)."""
+    n = np.zeros(len(KERNELS), np.int64)
+    ms = np.zeros(len(KERNELS), np.float64)
+    _check(lib.pk_trace_read(index, n.ctypes.data, ms.ctypes.data), "pk_trace_read")
+    return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(KERNELS)}

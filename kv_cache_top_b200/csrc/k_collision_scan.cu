@@ -1,0 +1,175 @@
+// k_collision_scan.cu -- multi-tier collision counting and the integer Top-C
+// threshold.
+//
+// S_i = sum_b bonus_b[code_{i,b}]  (ParisKV slides, "Stage I uses multi-tier
+// collision votes to prune keys", App. B.2.1 Eq. 15), an integer in [0, 96].
+// "Small integer scores allow histogram and prefix-scan selection instead of a
+// full sort" (same frame): each CTA histograms the S of its chunk, and the
+// last CTA of a pair to finish (ticket counter, no spin-wait) finds the
+// threshold s* = max{s : #{S >= s} >= C}, and for every chunk the first slot of
+// its candidates and how many of its S = s* keys it keeps (lower ids first),
+// so the rerank kernel can compact candidates in ascending id order without
+// any further global synchronisation.
+//
+// Hot loop: 16 B of codes per key read with 128-bit streaming loads; the 16
+// bonus tables (4 bits x 256 centres = one 32-bit register per lane per
+// block) live in registers and are read with warp shuffles, which have no
+// bank conflicts whatever the codes are.
+#include "pk_internal.cuh"
+
+namespace pk {
+
+constexpr int kScanThreads = 256;
+constexpr int kScanUnroll = 4;
+constexpr int kHistPad = 104;
+
+__device__ __forceinline__ uint32_t lookup_bonus(const uint32_t (&tab)[kB], int b, uint32_t code)
+{
+    const uint32_t w = __shfl_sync(kFull, tab[b], (int)(code >> 3));
+    return (w >> ((code & 7u) << 2)) & 0xfu;
+}
+
+__device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], uint4 c)
+{
+    uint32_t s = 0;
+    const uint32_t wds[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+#pragma unroll
+        for (int k = 0; k < 4; k++) s += lookup_bonus(tab, 4 * q + k, (wds[q] >> (8 * k)) & 0xffu);
+    }
+    return s;
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
+{
+    const int bh = blockIdx.y, chunk = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = kScanThreads / 32;
+    __shared__ uint32_t s_hist[NW][kHistPad];
+    __shared__ uint32_t s_cum[kHistPad];
+    __shared__ uint32_t s_ws[NW + 1];
+    __shared__ int s_last;
+
+    for (int i = tid; i < NW * kHistPad; i += kScanThreads) (&s_hist[0][0])[i] = 0u;
+
+    uint32_t tab[kB];
+    const uint32_t *bp = a.bonus_packed + (size_t)bh * kB * 32;
+#pragma unroll
+    for (int b = 0; b < kB; b++) tab[b] = bp[b * 32 + lane];
+    __syncthreads();
+
+    const int64_t lo = (int64_t)chunk * a.chunk;
+    const int64_t hi = min(lo + a.chunk, a.n);
+    const int64_t cnt = hi - lo;
+    const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes + ((size_t)bh * a.n_cap + lo) * kB);
+    uint8_t *S = a.S + (size_t)bh * a.n_cap + lo;
+    uint8_t *dS = a.dbg_S ? a.dbg_S + (size_t)bh * a.n + lo : nullptr;
+
+    // every lane runs every iteration (the shuffles need the full warp);
+    // lanes past the end of the chunk compute on a zero code and store nothing
+    for (int64_t base = (int64_t)warp * 32 * kScanUnroll; base < cnt;
+         base += (int64_t)NW * 32 * kScanUnroll) {
+        uint4 c[kScanUnroll];
+#pragma unroll
+        for (int u = 0; u < kScanUnroll; u++) {
+            const int64_t i = base + u * 32 + lane;
+            c[u] = (i < cnt) ? __ldcs(codes + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kScanUnroll; u++) {
+            const int64_t i = base + u * 32 + lane;
+            const uint32_t s = collision_score(tab, c[u]);
+            if (i < cnt) {
+                S[i] = (uint8_t)s;
+                if (dS) dS[i] = (uint8_t)s;
+                atomicAdd(&s_hist[warp][s], 1u);
+            }
+        }
+    }
+    __syncthreads();
+
+    // chunk histogram -> suffix counts cum[s] = #{S >= s}, s = 0..97
+    uint32_t hv = 0;
+    if (tid < kBins) {
+#pragma unroll
+        for (int w = 0; w < NW; w++) hv += s_hist[w][tid];
+    }
+    if (tid < kHistPad) s_cum[tid] = (tid < kBins) ? hv : 0u;
+    __syncthreads();
+    // suffix sum by a reversed exclusive scan over 256 threads
+    {
+        const int s = kScanThreads - 1 - tid;   // thread tid handles bin s (descending)
+        const uint32_t v = (s < kBins) ? s_cum[s] : 0u;
+        uint32_t tot;
+        const uint32_t ex = block_excl_scan<kScanThreads>(v, s_ws, &tot);
+        if (s < kCum) a.chunk_cum[((size_t)bh * a.max_chunks + chunk) * kCum + s] = ex + v;
+    }
+    if (tid < kBins && hv) atomicAdd(&a.head_hist[(size_t)bh * kBins + tid], hv);
+
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(&a.tickets[(size_t)bh * 2 + 0], 1u) == (unsigned)(a.nchunks - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // ---- last CTA of this pair: threshold and per-chunk candidate slots
+    uint32_t H = 0;
+    if (tid < kBins) H = __ldcg(&a.head_hist[(size_t)bh * kBins + tid]);
+    if (a.dbg_hist && tid < kBins) a.dbg_hist[(size_t)bh * kBins + tid] = H;
+    int64_t cumH;
+    {
+        const int s = kScanThreads - 1 - tid;
+        const uint32_t v = (s < kBins) ? __ldcg(&a.head_hist[(size_t)bh * kBins + s]) : 0u;
+        uint32_t tot;
+        const uint32_t ex = block_excl_scan<kScanThreads>(v, s_ws, &tot);
+        cumH = (int64_t)(ex + v);           // #{S >= s} for s = 255 - tid
+        // s* = largest s with #{S >= s} >= C  (cum is non-increasing in s)
+        const int pred = (s < kCum) && (cumH >= a.C);
+        const int nsat = __syncthreads_count(pred);
+        if (tid == 0) s_last = nsat - 1;    // reuse as s*
+    }
+    __syncthreads();
+    const int sstar = s_last;
+    if (tid == 0) {
+        a.sstar[bh] = sstar;
+        if (a.dbg_sstar) a.dbg_sstar[bh] = sstar;
+        a.tickets[(size_t)bh * 2 + 0] = 0u;
+    }
+    // gt_total = #{S > s*}, ties to take t = C - gt_total (1 <= t <= #{S = s*})
+    __shared__ uint32_t s_gt_total;
+    if (kScanThreads - 1 - tid == sstar + 1) s_gt_total = (uint32_t)cumH;   // s* + 1 <= 97
+    __syncthreads();
+    const int64_t ties = a.C - (int64_t)s_gt_total;
+    uint32_t carry_eq = 0, carry_slot = 0;
+    for (int j0 = 0; j0 < a.nchunks; j0 += kScanThreads) {
+        const int j = j0 + tid;
+        uint32_t gt = 0, eq = 0;
+        if (j < a.nchunks) {
+            const uint32_t *cj = a.chunk_cum + ((size_t)bh * a.max_chunks + j) * kCum;
+            const uint32_t c0 = __ldcg(cj + sstar), c1 = __ldcg(cj + sstar + 1);
+            gt = c1;
+            eq = c0 - c1;
+        }
+        uint32_t tot_eq;
+        const uint32_t ex_eq = carry_eq + block_excl_scan<kScanThreads>(eq, s_ws, &tot_eq);
+        const int64_t room = ties - (int64_t)ex_eq;
+        const uint32_t quota = room <= 0 ? 0u : (room >= (int64_t)eq ? eq : (uint32_t)room);
+        uint32_t tot_slot;
+        const uint32_t ex_slot = carry_slot + block_excl_scan<kScanThreads>(gt + quota, s_ws, &tot_slot);
+        if (j < a.nchunks) a.chunk_info[(size_t)bh * a.max_chunks + j] = make_uint2(ex_slot, quota);
+        carry_eq += tot_eq;
+        carry_slot += tot_slot;
+    }
+}
+
+}  // namespace pk
+
+namespace pk {
+cudaError_t launch_collision_scan(const ScanArgs &a, int bh, cudaStream_t s)
+{
+    k_collision_scan<<<dim3(a.nchunks, bh), kScanThreads, 0, s>>>(a);
+    return cudaGetLastError();
+}
+}  // namespace pk

@@ -1,0 +1,626 @@
+// pk_api.cu -- host side of the C-ABI declared in include/pariskv.h:
+// argument checks, index storage, launch configuration and tracing.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "pk_internal.cuh"
+
+using namespace pk;
+
+struct TraceRec {
+    int kind;
+    cudaEvent_t a, b;
+};
+
+struct pk_index {
+    pk_params p;
+    int32_t bh = 0;
+    int64_t n = 0;
+    int device = 0;
+    int num_sms = 148;
+    int32_t max_chunks = 1;
+    int32_t topk_cap = 100;
+    int es = 2;
+    float scale = 0.0f;
+    RotConst rot{};
+    Levels lv{};
+    // index storage (device)
+    uint8_t *codes = nullptr;
+    uint8_t *rec = nullptr;
+    uint32_t *occ = nullptr;
+    // K/V store (device, or mapped pinned host)
+    void *K = nullptr, *V = nullptr;
+    bool kv_host = false;
+    // search workspace (device)
+    float *qt = nullptr, *qnorm = nullptr;
+    uint32_t *bonus_packed = nullptr;
+    uint8_t *S = nullptr;
+    uint32_t *chunk_cum = nullptr, *head_hist = nullptr, *tickets = nullptr;
+    uint2 *chunk_info = nullptr;
+    int32_t *sstar = nullptr;
+    unsigned long long *partial = nullptr;
+    int32_t *dev_err = nullptr;
+    long long *dev_err_detail = nullptr;
+    // tracing
+    bool trace = false;
+    std::vector<TraceRec> tr;
+    std::vector<cudaEvent_t> ev_pool;
+    size_t ev_used = 0;
+};
+
+namespace {
+
+constexpr int64_t kMinChunk = 1024;
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+pk_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return PK_OK;
+    if (e == cudaErrorMemoryAllocation) return PK_ERR_OOM;
+    return PK_ERR_CUDA;
+}
+
+// A pointer the GPU can read: device memory or page-locked host memory.
+bool device_accessible(const void *ptr)
+{
+    if (!ptr) return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeHost ||
+           at.type == cudaMemoryTypeManaged;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+void ratio_table(int64_t n, double *beta, double *rho)
+{
+    // README adaptive ratio table; K = 1000, half-open ranges.
+    if (n < 5000) { *beta = 0.50; *rho = 0.50; }
+    else if (n < 10000) { *beta = 0.25; *rho = 0.30; }
+    else if (n < 30000) { *beta = 0.20; *rho = 0.25; }
+    else { *beta = 0.10; *rho = 0.20; }
+}
+
+void resolve(int64_t n, int64_t cand_budget, float collision_ratio, int32_t topk, int64_t *C,
+             int64_t *R)
+{
+    double beta, rho;
+    ratio_table(n, &beta, &rho);
+    int64_t c = cand_budget > 0 ? cand_budget : (int64_t)std::ceil(beta * (double)n);
+    if (c < topk) c = topk;
+    if (c > n) c = n;
+    const double r = collision_ratio > 0.0f ? (double)collision_ratio : rho;
+    int64_t rr = (int64_t)std::ceil(r * (double)n);
+    if (rr < 1) rr = 1;
+    if (rr > n) rr = n;
+    *C = c;
+    *R = rr;
+}
+
+uint64_t splitmix64(uint64_t x)
+{
+    uint64_t z = x + 0x9e3779b97f4a7c15ULL;
+    z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ULL;
+    z = (z ^ (z >> 27)) * 0x94d049bb133111ebULL;
+    return z ^ (z >> 31);
+}
+
+void chunking(const pk_index *ix, int64_t n, int32_t *nchunks, int64_t *chunk)
+{
+    int64_t nch = ceil_div(4 * (int64_t)ix->num_sms, ix->bh);
+    nch = std::max<int64_t>(1, std::min<int64_t>(nch, ceil_div(n, kMinChunk)));
+    nch = std::min<int64_t>(nch, ix->max_chunks);
+    int64_t ch = ceil_div(ceil_div(n, nch), 16) * 16;
+    *chunk = ch;
+    *nchunks = (int32_t)ceil_div(n, ch);
+}
+
+void free_all(pk_index *ix)
+{
+    if (!ix) return;
+    cudaFree(ix->codes);
+    cudaFree(ix->rec);
+    cudaFree(ix->occ);
+    if (ix->kv_host) {
+        cudaFreeHost(ix->K);
+        cudaFreeHost(ix->V);
+    } else {
+        cudaFree(ix->K);
+        cudaFree(ix->V);
+    }
+    cudaFree(ix->qt);
+    cudaFree(ix->qnorm);
+    cudaFree(ix->bonus_packed);
+    cudaFree(ix->S);
+    cudaFree(ix->chunk_cum);
+    cudaFree(ix->head_hist);
+    cudaFree(ix->tickets);
+    cudaFree(ix->chunk_info);
+    cudaFree(ix->sstar);
+    cudaFree(ix->partial);
+    cudaFree(ix->dev_err);
+    cudaFree(ix->dev_err_detail);
+    for (cudaEvent_t e : ix->ev_pool) cudaEventDestroy(e);
+}
+
+template <class T>
+cudaError_t dalloc(T **p, size_t count)
+{
+    return cudaMalloc((void **)p, count * sizeof(T) + 16);
+}
+
+// ---- tracing
+void trace_begin(pk_index *ix, int kind, cudaStream_t s)
+{
+    if (!ix->trace) return;
+    if (ix->ev_used + 2 > ix->ev_pool.size()) {
+        for (int i = 0; i < 256; i++) {
+            cudaEvent_t e;
+            if (cudaEventCreate(&e) != cudaSuccess) return;
+            ix->ev_pool.push_back(e);
+        }
+    }
+    TraceRec r{kind, ix->ev_pool[ix->ev_used], ix->ev_pool[ix->ev_used + 1]};
+    ix->ev_used += 2;
+    cudaEventRecord(r.a, s);
+    ix->tr.push_back(r);
+}
+
+void trace_end(pk_index *ix, cudaStream_t s)
+{
+    if (!ix->trace || ix->tr.empty()) return;
+    cudaEventRecord(ix->tr.back().b, s);
+}
+
+pk_status check_params(const pk_params *p)
+{
+    if (!p) return PK_ERR_INVALID_ARG;
+    if (p->head_dim != kD || p->sub_dim != kM) return PK_ERR_UNSUPPORTED;
+    if (p->batch < 1 || p->n_kv_heads < 1 || p->group < 1 || p->group > kMaxGroup)
+        return PK_ERR_INVALID_ARG;
+    if (p->topk < 1) return PK_ERR_INVALID_ARG;
+    if (p->topk > kMaxTopk) return PK_ERR_UNSUPPORTED;
+    if (p->kv_dtype != PK_F32 && p->kv_dtype != PK_BF16) return PK_ERR_INVALID_ARG;
+    if (p->kv_location != PK_KV_DEVICE && p->kv_location != PK_KV_HOST_PINNED)
+        return PK_ERR_INVALID_ARG;
+    if (p->cand_budget < 0 || !(p->collision_ratio >= 0.0f) || p->collision_ratio > 1.0f ||
+        !(p->attn_scale >= 0.0f))
+        return PK_ERR_INVALID_ARG;
+    return PK_OK;
+}
+
+pk_status encode_range(pk_index *ix, const void *Kin, int64_t n_new, int64_t pos0, cudaStream_t s)
+{
+    EncodeArgs a{};
+    a.K = Kin;
+    a.n_new = n_new;
+    a.pos0 = pos0;
+    a.n_cap = ix->p.n_cap;
+    a.bh = ix->bh;
+    a.is_bf16 = ix->p.kv_dtype == PK_BF16;
+    a.codes = ix->codes;
+    a.rec = ix->rec;
+    a.occ = ix->occ;
+    a.rot = ix->rot;
+    a.lv = ix->lv;
+    trace_begin(ix, PK_K_ENCODE, s);
+    cudaError_t e = launch_encode(a, s);
+    trace_end(ix, s);
+    return cuda_status(e);
+}
+
+// copy [BH][n_new][D] rows into the store at positions pos0.. of each pair
+pk_status copy_rows(pk_index *ix, void *store, const void *src, int64_t n_new, int64_t pos0,
+                    cudaStream_t s)
+{
+    const size_t row = (size_t)kD * ix->es;
+    cudaError_t e = cudaMemcpy2DAsync((char *)store + (size_t)pos0 * row, (size_t)ix->p.n_cap * row,
+                                      src, (size_t)n_new * row, (size_t)n_new * row, (size_t)ix->bh,
+                                      cudaMemcpyDefault, s);
+    return cuda_status(e);
+}
+
+pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_idx, float *out_score,
+                      const pk_debug_out *dbg, cudaStream_t s)
+{
+    if (!ix || !q || !out_idx) return PK_ERR_INVALID_ARG;
+    if (topk < 1 || topk > ix->topk_cap) return PK_ERR_INVALID_ARG;
+    if (ix->n < topk) return PK_ERR_CAPACITY;
+    if (!device_accessible(q) || !device_accessible(out_idx) ||
+        (out_score && !device_accessible(out_score)))
+        return PK_ERR_INVALID_ARG;
+    if (!aligned(q, ix->es) || !aligned(out_idx, 4) || (out_score && !aligned(out_score, 4)))
+        return PK_ERR_INVALID_ARG;
+    int64_t C, R;
+    resolve(ix->n, ix->p.cand_budget, ix->p.collision_ratio, topk, &C, &R);
+    int32_t nchunks;
+    int64_t chunk;
+    chunking(ix, ix->n, &nchunks, &chunk);
+
+    PrepArgs pa{};
+    pa.q = q;
+    pa.H = ix->p.n_kv_heads;
+    pa.G = ix->p.group;
+    pa.is_bf16 = ix->p.kv_dtype == PK_BF16;
+    pa.bh = ix->bh;
+    pa.R = R;
+    pa.occ = ix->occ;
+    pa.rot = ix->rot;
+    pa.qt = ix->qt;
+    pa.qnorm = ix->qnorm;
+    pa.bonus_packed = ix->bonus_packed;
+    pa.head_hist = ix->head_hist;
+    pa.tickets = ix->tickets;
+    if (dbg) {
+        pa.dbg_bonus = dbg->bonus;
+        pa.dbg_qt = dbg->qt;
+        pa.dbg_qnorm = dbg->qnorm;
+    }
+    trace_begin(ix, PK_K_QUERY_PREP, s);
+    cudaError_t e = launch_query_prep(pa, s);
+    trace_end(ix, s);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    ScanArgs sa{};
+    sa.codes = ix->codes;
+    sa.bonus_packed = ix->bonus_packed;
+    sa.n = ix->n;
+    sa.n_cap = ix->p.n_cap;
+    sa.chunk = chunk;
+    sa.C = C;
+    sa.nchunks = nchunks;
+    sa.S = ix->S;
+    sa.chunk_cum = ix->chunk_cum;
+    sa.head_hist = ix->head_hist;
+    sa.tickets = ix->tickets;
+    sa.chunk_info = ix->chunk_info;
+    sa.sstar = ix->sstar;
+    sa.max_chunks = ix->max_chunks;
+    if (dbg) {
+        sa.dbg_S = dbg->S;
+        sa.dbg_hist = dbg->hist;
+        sa.dbg_sstar = dbg->sstar;
+    }
+    trace_begin(ix, PK_K_COLLISION_SCAN, s);
+    e = launch_collision_scan(sa, ix->bh, s);
+    trace_end(ix, s);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    RerankArgs ra{};
+    ra.S = ix->S;
+    ra.rec = ix->rec;
+    ra.qt = ix->qt;
+    ra.qnorm = ix->qnorm;
+    ra.chunk_info = ix->chunk_info;
+    ra.sstar = ix->sstar;
+    ra.n = ix->n;
+    ra.n_cap = ix->p.n_cap;
+    ra.chunk = chunk;
+    ra.C = C;
+    ra.nchunks = nchunks;
+    ra.max_chunks = ix->max_chunks;
+    ra.topk = topk;
+    ra.tickets = ix->tickets;
+    ra.partial = ix->partial;
+    ra.topk_cap = ix->topk_cap;
+    ra.lv = ix->lv;
+    ra.out_idx = out_idx;
+    ra.out_score = out_score;
+    if (dbg) {
+        ra.dbg_cand = dbg->cand;
+        ra.dbg_est = dbg->cand_est;
+    }
+    ra.dev_err = ix->dev_err;
+    trace_begin(ix, PK_K_RERANK_TOPK, s);
+    e = launch_rerank_topk(ra, ix->bh, s);
+    trace_end(ix, s);
+    return cuda_status(e);
+}
+
+}  // namespace
+
+// ======================================================================
+extern "C" {
+
+void pk_default_params(pk_params *p)
+{
+    if (!p) return;
+    std::memset(p, 0, sizeof(*p));
+    p->batch = 1;
+    p->n_kv_heads = 8;
+    p->group = 4;
+    p->head_dim = kD;
+    p->sub_dim = kM;
+    p->topk = 100;
+    p->n_cap = 0;
+    p->cand_budget = 0;
+    p->collision_ratio = 0.0f;
+    p->attn_scale = 0.0f;
+    p->rot_seed = 0;
+    p->kv_dtype = PK_BF16;
+    p->kv_location = PK_KV_DEVICE;
+}
+
+const char *pk_status_str(pk_status s)
+{
+    switch (s) {
+    case PK_OK: return "ok";
+    case PK_ERR_INVALID_ARG: return "invalid argument";
+    case PK_ERR_CAPACITY: return "capacity exceeded";
+    case PK_ERR_OOM: return "out of memory";
+    case PK_ERR_CUDA: return "CUDA error";
+    case PK_ERR_TIMEOUT: return "device wait timed out";
+    case PK_ERR_DEVICE_CHECK: return "device-side check failed";
+    case PK_ERR_UNSUPPORTED: return "unsupported configuration";
+    }
+    return "unknown status";
+}
+
+pk_status pk_resolve(int64_t n, int64_t cand_budget, float collision_ratio, int32_t topk,
+                     int64_t *C, int64_t *R)
+{
+    if (n < 1 || !C || !R || topk < 1 || cand_budget < 0 || !(collision_ratio >= 0.0f))
+        return PK_ERR_INVALID_ARG;
+    resolve(n, cand_budget, collision_ratio, topk, C, R);
+    return PK_OK;
+}
+
+pk_status pk_magnitude_levels(int32_t m, int32_t L, float *levels, float *thresholds)
+{
+    if (m < 3 || L < 2 || L > 4096 || !levels || !thresholds) return PK_ERR_INVALID_ARG;
+    std::vector<double> lev(L), thr(L - 1);
+    if (lloyd_max_levels(m, L, lev.data(), thr.data()) < 0) return PK_ERR_CUDA;
+    for (int t = 0; t < L; t++) levels[t] = (float)lev[t];
+    for (int t = 0; t < L - 1; t++) thresholds[t] = (float)thr[t];
+    return PK_OK;
+}
+
+pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_params *params,
+                         void *stream, pk_index **out)
+{
+    if (!out) return PK_ERR_INVALID_ARG;
+    *out = nullptr;
+    pk_status st = check_params(params);
+    if (st != PK_OK) return st;
+    if (!K || !V || n < 1) return PK_ERR_INVALID_ARG;
+    const int64_t n_cap = params->n_cap > 0 ? params->n_cap : n;
+    if (n > n_cap || n_cap > (int64_t)0x7fffffff - 16) return PK_ERR_CAPACITY;
+    if (!device_accessible(K) || !device_accessible(V)) return PK_ERR_INVALID_ARG;
+    const int es = params->kv_dtype == PK_BF16 ? 2 : 4;
+    if (!aligned(K, es) || !aligned(V, es)) return PK_ERR_INVALID_ARG;
+
+    pk_index *ix = new (std::nothrow) pk_index();
+    if (!ix) return PK_ERR_OOM;
+    ix->p = *params;
+    ix->p.n_cap = ceil_div(n_cap, 16) * 16;   // keeps every per-pair row 16-byte aligned
+    ix->bh = params->batch * params->n_kv_heads;
+    ix->es = es;
+    ix->topk_cap = params->topk;
+    ix->scale = params->attn_scale > 0.0f ? params->attn_scale : (float)(1.0 / std::sqrt((double)kD));
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaGetDevice(&ix->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ix->num_sms, cudaDevAttrMultiProcessorCount, ix->device);
+    if (e != cudaSuccess) {
+        delete ix;
+        return cuda_status(e);
+    }
+    ix->max_chunks = (int32_t)std::max<int64_t>(1, ceil_div(4 * (int64_t)ix->num_sms, ix->bh));
+
+    // SRHT sign diagonal and scale; Lloyd-Max levels
+    for (int r = 0; r < 4; r++) ix->rot.sign_mask[r] = 0;
+    for (int j = 0; j < kD; j++)
+        if (splitmix64(params->rot_seed * (uint64_t)kD + (uint64_t)j) >> 63)
+            ix->rot.sign_mask[j / 32] |= 1u << (j % 32);
+    ix->rot.c = (float)(1.0 / std::sqrt((double)kD));
+    {
+        double lev[kL], thr[kL - 1];
+        if (lloyd_max_levels(kM, kL, lev, thr) < 0) {
+            delete ix;
+            return PK_ERR_CUDA;
+        }
+        for (int t = 0; t < kL; t++) ix->lv.lev[t] = (float)lev[t];
+        for (int t = 0; t < kL - 1; t++) ix->lv.thr[t] = (float)thr[t];
+    }
+
+    const size_t BH = ix->bh, NC = ix->p.n_cap, MC = ix->max_chunks;
+    e = cudaSuccess;
+    auto chk = [&](cudaError_t x) { if (e == cudaSuccess) e = x; };
+    chk(dalloc(&ix->codes, BH * NC * kB));
+    chk(dalloc(&ix->rec, BH * NC * kRecBytes));
+    chk(dalloc(&ix->occ, BH * kB * kNC));
+    chk(dalloc(&ix->qt, BH * kD));
+    chk(dalloc(&ix->qnorm, BH));
+    chk(dalloc(&ix->bonus_packed, BH * kB * 32));
+    chk(dalloc(&ix->S, BH * NC));
+    chk(dalloc(&ix->chunk_cum, BH * MC * kCum));
+    chk(dalloc(&ix->head_hist, BH * kBins));
+    chk(dalloc(&ix->tickets, BH * 2));
+    chk(dalloc(&ix->chunk_info, BH * MC));
+    chk(dalloc(&ix->sstar, BH));
+    chk(dalloc(&ix->partial, BH * MC * (size_t)ix->topk_cap));
+    chk(dalloc(&ix->dev_err, 1));
+    chk(dalloc(&ix->dev_err_detail, 1));
+    const size_t kv_bytes = BH * NC * kD * (size_t)es;
+    if (params->kv_location == PK_KV_HOST_PINNED) {
+        ix->kv_host = true;
+        chk(cudaHostAlloc(&ix->K, kv_bytes, cudaHostAllocMapped | cudaHostAllocPortable));
+        chk(cudaHostAlloc(&ix->V, kv_bytes, cudaHostAllocMapped | cudaHostAllocPortable));
+    } else {
+        chk(cudaMalloc(&ix->K, kv_bytes));
+        chk(cudaMalloc(&ix->V, kv_bytes));
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        free_all(ix);
+        delete ix;
+        return PK_ERR_OOM;
+    }
+    chk(cudaMemsetAsync(ix->occ, 0, BH * kB * kNC * sizeof(uint32_t), s));
+    chk(cudaMemsetAsync(ix->head_hist, 0, BH * kBins * sizeof(uint32_t), s));
+    chk(cudaMemsetAsync(ix->tickets, 0, BH * 2 * sizeof(uint32_t), s));
+    chk(cudaMemsetAsync(ix->dev_err, 0, sizeof(int32_t), s));
+    chk(cudaMemsetAsync(ix->dev_err_detail, 0, sizeof(long long), s));
+    if (e == cudaSuccess) st = copy_rows(ix, ix->K, K, n, 0, s);
+    if (e == cudaSuccess && st == PK_OK) st = copy_rows(ix, ix->V, V, n, 0, s);
+    if (e == cudaSuccess && st == PK_OK) st = encode_range(ix, K, n, 0, s);
+    if (e != cudaSuccess || st != PK_OK) {
+        cudaStreamSynchronize(s);
+        free_all(ix);
+        delete ix;
+        return e != cudaSuccess ? cuda_status(e) : st;
+    }
+    ix->n = n;
+    *out = ix;
+    return PK_OK;
+}
+
+pk_status pk_append(pk_index *ix, const void *k_new, const void *v_new, int64_t n_new, void *stream)
+{
+    if (!ix || !k_new || !v_new || n_new < 1) return PK_ERR_INVALID_ARG;
+    if (ix->n + n_new > ix->p.n_cap) return PK_ERR_CAPACITY;
+    if (!device_accessible(k_new) || !device_accessible(v_new)) return PK_ERR_INVALID_ARG;
+    if (!aligned(k_new, ix->es) || !aligned(v_new, ix->es)) return PK_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    pk_status st = copy_rows(ix, ix->K, k_new, n_new, ix->n, s);
+    if (st == PK_OK) st = copy_rows(ix, ix->V, v_new, n_new, ix->n, s);
+    if (st == PK_OK) st = encode_range(ix, k_new, n_new, ix->n, s);
+    if (st == PK_OK) ix->n += n_new;
+    return st;
+}
+
+pk_status pk_search(pk_index *ix, const void *q, int32_t topk, int32_t *out_idx, float *out_score,
+                    void *stream)
+{
+    return search_impl(ix, q, topk, out_idx, out_score, nullptr, (cudaStream_t)stream);
+}
+
+pk_status pk_search_debug(pk_index *ix, const void *q, int32_t topk, int32_t *out_idx,
+                          float *out_score, const pk_debug_out *dbg, void *stream)
+{
+    return search_impl(ix, q, topk, out_idx, out_score, dbg, (cudaStream_t)stream);
+}
+
+pk_status pk_attend(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t topk, float *out,
+                    void *stream)
+{
+    if (!ix || !q || !sel_idx || !out) return PK_ERR_INVALID_ARG;
+    if (topk < 1 || topk > ix->topk_cap) return PK_ERR_INVALID_ARG;
+    if (!device_accessible(q) || !device_accessible(sel_idx) || !device_accessible(out))
+        return PK_ERR_INVALID_ARG;
+    if (!aligned(q, ix->es) || !aligned(sel_idx, 4) || !aligned(out, 4)) return PK_ERR_INVALID_ARG;
+    AttendArgs a{};
+    a.q = q;
+    a.idx = sel_idx;
+    a.K = ix->K;
+    a.V = ix->V;
+    a.out = out;
+    a.n = ix->n;
+    a.n_cap = ix->p.n_cap;
+    a.H = ix->p.n_kv_heads;
+    a.G = ix->p.group;
+    a.topk = topk;
+    a.is_bf16 = ix->p.kv_dtype == PK_BF16;
+    a.scale = ix->scale;
+    a.dev_err = ix->dev_err;
+    a.dev_err_detail = ix->dev_err_detail;
+    cudaStream_t s = (cudaStream_t)stream;
+    trace_begin(ix, PK_K_GATHER_ATTEND, s);
+    cudaError_t e = launch_gather_attend(a, ix->bh, s);
+    trace_end(ix, s);
+    return cuda_status(e);
+}
+
+void pk_free(pk_index *ix)
+{
+    if (!ix) return;
+    cudaDeviceSynchronize();
+    free_all(ix);
+    delete ix;
+}
+
+pk_status pk_last_device_error(pk_index *ix, int64_t *detail)
+{
+    if (!ix) return PK_ERR_INVALID_ARG;
+    int32_t code = 0;
+    long long det = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpy(&code, ix->dev_err, sizeof(code), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemcpy(&det, ix->dev_err_detail, sizeof(det), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(ix->dev_err, 0, sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemset(ix->dev_err_detail, 0, sizeof(long long));
+    if (e != cudaSuccess) return cuda_status(e);
+    if (detail) *detail = det;
+    return code == 0 ? PK_OK : PK_ERR_DEVICE_CHECK;
+}
+
+pk_status pk_get_info(const pk_index *ix, pk_info *info)
+{
+    if (!ix || !info) return PK_ERR_INVALID_ARG;
+    std::memset(info, 0, sizeof(*info));
+    info->n = ix->n;
+    info->n_cap = ix->p.n_cap;
+    info->bh = ix->bh;
+    chunking(ix, ix->n, &info->nchunks, &info->chunk);
+    resolve(ix->n, ix->p.cand_budget, ix->p.collision_ratio, ix->p.topk, &info->cand, &info->coll);
+    info->index_bytes = (int64_t)ix->bh * ix->p.n_cap * (kB + kRecBytes) + (int64_t)ix->bh * kB * kNC * 4;
+    info->kv_bytes = 2 * (int64_t)ix->bh * ix->p.n_cap * kD * ix->es;
+    info->kv_location = ix->p.kv_location;
+    info->num_sms = ix->num_sms;
+    return PK_OK;
+}
+
+pk_status pk_export_index(const pk_index *ix, uint8_t *codes, uint8_t *records, uint32_t *occ,
+                          void *stream)
+{
+    if (!ix) return PK_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (codes)
+        e = cudaMemcpy2DAsync(codes, (size_t)ix->n * kB, ix->codes, (size_t)ix->p.n_cap * kB,
+                              (size_t)ix->n * kB, ix->bh, cudaMemcpyDefault, s);
+    if (e == cudaSuccess && records)
+        e = cudaMemcpy2DAsync(records, (size_t)ix->n * kRecBytes, ix->rec, (size_t)ix->p.n_cap * kRecBytes,
+                              (size_t)ix->n * kRecBytes, ix->bh, cudaMemcpyDefault, s);
+    if (e == cudaSuccess && occ)
+        e = cudaMemcpyAsync(occ, ix->occ, (size_t)ix->bh * kB * kNC * sizeof(uint32_t), cudaMemcpyDefault, s);
+    return cuda_status(e);
+}
+
+pk_status pk_trace_enable(pk_index *ix, int32_t on)
+{
+    if (!ix) return PK_ERR_INVALID_ARG;
+    ix->trace = on != 0;
+    return PK_OK;
+}
+
+pk_status pk_trace_read(pk_index *ix, int64_t *launches, double *total_ms)
+{
+    if (!ix || !launches || !total_ms) return PK_ERR_INVALID_ARG;
+    for (int k = 0; k < PK_K_COUNT; k++) {
+        launches[k] = 0;
+        total_ms[k] = 0.0;
+    }
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e);
+    for (const TraceRec &r : ix->tr) {
+        float ms = 0.0f;
+        if (cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+            launches[r.kind] += 1;
+            total_ms[r.kind] += ms;
+        } else {
+            cudaGetLastError();
+        }
+    }
+    ix->tr.clear();
+    ix->ev_used = 0;
+    return PK_OK;
+}
+
+}  // extern "C"

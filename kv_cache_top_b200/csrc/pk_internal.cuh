@@ -1,0 +1,243 @@
+// pk_internal.cuh -- shared device helpers and kernel argument blocks of the
+// ParisKV retrieval library (sm_100a).  Not part of the public C-ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pariskv.h"
+
+namespace pk {
+
+constexpr int kD = 128;          // head_dim
+constexpr int kM = 8;            // sub-space dimension m
+constexpr int kB = kD / kM;      // blocks per key (16)
+constexpr int kNC = 1 << kM;     // sign-pattern centres per block (256)
+constexpr int kL = 8;            // magnitude levels (3 bits)
+constexpr int kSMax = 6 * kB;    // largest collision score (96)
+constexpr int kBins = kSMax + 1; // score histogram bins (97)
+constexpr int kCum = kBins + 1;  // suffix-count entries per chunk (98, last = 0)
+constexpr int kRecBytes = 128;   // 4-bit summary record per key
+constexpr int kMaxTopk = 1024;
+constexpr int kMaxGroup = 8;
+constexpr unsigned kFull = 0xffffffffu;
+
+// Device-check codes written to the index's error word (first one wins).
+enum : int32_t { DEVCHK_NONE = 0, DEVCHK_BAD_INDEX = 1, DEVCHK_CAND_COUNT = 2 };
+
+struct RotConst {
+    uint32_t sign_mask[4];   // bit l of word r: coordinate l + 32 r has s = -1
+    float c;                 // fp32(1/sqrt(D))
+};
+
+struct Levels {
+    float lev[kL];
+    float thr[kL - 1];
+};
+
+struct EncodeArgs {
+    const void *K;           // [BH][n_new][D] kv dtype
+    int64_t n_new;
+    int64_t pos0;            // first position written
+    int64_t n_cap;
+    int32_t bh;
+    int32_t is_bf16;
+    uint8_t *codes;          // [BH][n_cap][16]
+    uint8_t *rec;            // [BH][n_cap][128]
+    uint32_t *occ;           // [BH][16][256]
+    RotConst rot;
+    Levels lv;
+};
+
+struct PrepArgs {
+    const void *q;           // [batch][H*G][D]
+    int32_t H, G, is_bf16, bh;
+    int64_t R;               // collision budget ceil(rho n)
+    const uint32_t *occ;
+    RotConst rot;
+    float *qt;               // [BH][D]
+    float *qnorm;            // [BH]
+    uint32_t *bonus_packed;  // [BH][16][32]  (4-bit bonus per centre)
+    uint32_t *head_hist;     // [BH][kBins]   zeroed here
+    uint32_t *tickets;       // [BH][2]       zeroed here
+    uint8_t *dbg_bonus;      // [BH][16][256] or null
+    float *dbg_qt;
+    float *dbg_qnorm;
+};
+
+struct ScanArgs {
+    const uint8_t *codes;
+    const uint32_t *bonus_packed;
+    int64_t n, n_cap, chunk, C;
+    int32_t nchunks;
+    uint8_t *S;              // [BH][n_cap]
+    uint32_t *chunk_cum;     // [BH][max_chunks][kCum]
+    uint32_t *head_hist;     // [BH][kBins]
+    uint32_t *tickets;       // [BH][2]
+    uint2 *chunk_info;       // [BH][max_chunks]  (first candidate slot, tie quota)
+    int32_t *sstar;          // [BH]
+    int32_t max_chunks;
+    uint8_t *dbg_S;
+    uint32_t *dbg_hist;
+    int32_t *dbg_sstar;
+};
+
+struct RerankArgs {
+    const uint8_t *S;
+    const uint8_t *rec;
+    const float *qt;
+    const float *qnorm;
+    const uint2 *chunk_info;
+    const int32_t *sstar;
+    int64_t n, n_cap, chunk, C;
+    int32_t nchunks, max_chunks, topk;
+    uint32_t *tickets;
+    unsigned long long *partial;   // [BH][max_chunks][topk_cap]
+    int32_t topk_cap;
+    Levels lv;
+    int32_t *out_idx;        // [BH][topk]
+    float *out_score;        // [BH][topk] or null
+    int32_t *dbg_cand;       // [BH][C] or null
+    float *dbg_est;          // [BH][C] or null
+    int32_t *dev_err;
+};
+
+struct AttendArgs {
+    const void *q;           // [batch][H*G][D]
+    const int32_t *idx;      // [BH][topk]
+    const void *K;           // [BH][n_cap][D]  (device or mapped host)
+    const void *V;
+    float *out;              // [batch][H*G][D]
+    int64_t n, n_cap;
+    int32_t H, G, topk, is_bf16;
+    float scale;
+    int32_t *dev_err;
+    long long *dev_err_detail;
+};
+
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ float ld_as_f32(const void *p, int64_t i, int is_bf16)
+{
+    if (is_bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+    return reinterpret_cast<const float *>(p)[i];
+}
+
+// Map an fp32 value to an unsigned key whose integer order is the float order.
+// -0.0 must already be folded into +0.0 by the caller (x + 0.0f).
+__device__ __forceinline__ uint32_t ord_f32(float x)
+{
+    uint32_t u = __float_as_uint(x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float unord_f32(uint32_t k)
+{
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+// Record a device-check failure (first writer wins) without trapping.
+__device__ __forceinline__ void devchk(int32_t *err, long long *detail, int32_t code, long long v)
+{
+    if (err && atomicCAS(err, 0, code) == 0 && detail) *detail = v;
+}
+
+// Canonical fp32 normalise + SRHT rotate of one 128-vector held by a warp:
+// lane l holds x[r] = coordinate l + 32 r.  Every operation is one IEEE
+// round-to-nearest step in the fixed order (i) sum of squares by the halving
+// tree, sqrt; (ii) divide by the norm; (iii) sign diagonal; (iv) Walsh-Hadamard
+// butterflies h = 1, 2, .., 64; (v) scale by c.  Returns the norm; a zero
+// vector stays zero.
+__device__ __forceinline__ float warp_rotate128(float x[4], const RotConst &rc, int lane)
+{
+    float s0 = __fmul_rn(x[0], x[0]), s1 = __fmul_rn(x[1], x[1]);
+    float s2 = __fmul_rn(x[2], x[2]), s3 = __fmul_rn(x[3], x[3]);
+    s0 = __fadd_rn(s0, s2);          // h = 64: s[j] += s[j+64]
+    s1 = __fadd_rn(s1, s3);
+    s0 = __fadd_rn(s0, s1);          // h = 32: s[j] += s[j+32]
+#pragma unroll
+    for (int h = 16; h >= 1; h >>= 1) s0 = __fadd_rn(s0, __shfl_xor_sync(kFull, s0, h));
+    const float nrm = __fsqrt_rn(s0);
+    if (nrm == 0.0f) {
+#pragma unroll
+        for (int r = 0; r < 4; r++) x[r] = 0.0f;
+        return 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+        float y = __fdiv_rn(x[r], nrm);
+        x[r] = ((rc.sign_mask[r] >> lane) & 1u) ? -y : y;
+    }
+#pragma unroll
+    for (int h = 1; h <= 16; h <<= 1) {
+        const bool hi = (lane & h) != 0;
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+            float p = __shfl_xor_sync(kFull, x[r], h);
+            x[r] = hi ? __fsub_rn(p, x[r]) : __fadd_rn(x[r], p);
+        }
+    }
+    {   // h = 32: registers (0,1), (2,3)
+        float a = x[0], b = x[1];
+        x[0] = __fadd_rn(a, b); x[1] = __fsub_rn(a, b);
+        a = x[2]; b = x[3];
+        x[2] = __fadd_rn(a, b); x[3] = __fsub_rn(a, b);
+    }
+    {   // h = 64: registers (0,2), (1,3)
+        float a = x[0], b = x[2];
+        x[0] = __fadd_rn(a, b); x[2] = __fsub_rn(a, b);
+        a = x[1]; b = x[3];
+        x[1] = __fadd_rn(a, b); x[3] = __fsub_rn(a, b);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; r++) x[r] = __fmul_rn(x[r], rc.c);
+    return nrm;
+}
+
+// Block-wide exclusive scan of one u32 per thread (blockDim.x == NT, NT a
+// multiple of 32, NT <= 1024).  `ws` needs NT/32 + 1 words of shared memory.
+// Returns the exclusive prefix; *total receives the block sum.
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *ws, uint32_t *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) ws[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = (lane < NT / 32) ? ws[lane] : 0u;
+        uint32_t t = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t y = __shfl_up_sync(kFull, t, o);
+            if (lane >= o) t += y;
+        }
+        if (lane < NT / 32) ws[lane] = t - w;
+        if (lane == 31) ws[NT / 32] = t;
+    }
+    __syncthreads();
+    uint32_t r = ws[warp] + x - v;
+    *total = ws[NT / 32];
+    __syncthreads();
+    return r;
+}
+
+}  // namespace pk
+
+namespace pk {
+// kernel launchers (one per kernel translation unit)
+cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
+cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s);
+cudaError_t launch_collision_scan(const ScanArgs &a, int bh, cudaStream_t s);
+cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s);
+cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s);
+size_t gather_attend_smem(int is_bf16);
+// host-side Lloyd-Max levels of the magnitude prior (closed-form integrals)
+int lloyd_max_levels(int m, int L, double *lev, double *thr);
+}  // namespace pk

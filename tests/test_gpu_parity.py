@@ -1,0 +1,249 @@
+"""GPU parity: the CUDA path through the C-ABI against the CPU oracle.
+
+Every case compares the library's outputs with the oracle element by element
+on the same seeded inputs (see tests/parity.py for the acceptance rules).
+Sizes span several chunks and compaction windows with ragged tails; the full
+8 x 128K and 1M workloads run in the launch configuration the benchmark
+times and are checked on sampled (sequence, KV head) pairs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pk():
+    from kv_cache_top_b200 import build
+    build.build()
+    import kv_cache_top_b200 as pk
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return pk
+
+
+def _dt(dtype):
+    return 1 if dtype == torch.bfloat16 else 0
+
+
+def build(pk, K, V, n, batch, H, G, topk=100, cand_budget=0, collision_ratio=0.0, n_cap=0,
+          kv_location=0, rot_seed=0):
+    p = pk.pk_default_params(batch=batch, n_kv_heads=H, group=G, topk=topk, n_cap=n_cap,
+                             cand_budget=cand_budget, collision_ratio=collision_ratio,
+                             kv_dtype=_dt(K.dtype), kv_location=kv_location, rot_seed=rot_seed)
+    return pk.pk_build_index(K, V, n, p)
+
+
+def search_debug(pk, h, q, BH, n, C, topk):
+    idx = torch.empty(BH, topk, dtype=torch.int32, device="cuda")
+    score = torch.empty(BH, topk, dtype=torch.float32, device="cuda")
+    dbg = parity.alloc_debug(BH, n, C)
+    pk.pk_search_debug(h, q, topk, idx, score, dbg)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), score.cpu().numpy(), parity.to_np(dbg)
+
+
+def export(pk, h, BH, n):
+    codes = torch.empty(BH, n, 16, dtype=torch.uint8, device="cuda")
+    rec = torch.empty(BH, n, 128, dtype=torch.uint8, device="cuda")
+    occ = torch.empty(BH, 16, 256, dtype=torch.int32, device="cuda")
+    pk.pk_export_index(h, codes, rec, occ)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), rec.cpu().numpy(), occ.cpu().numpy().view(np.uint32)
+
+
+def check_pairs(pk, h, K, V, q, pairs, batch, H, G, n, topk, cand_budget=0, collision_ratio=0.0,
+                attn_tol=parity.ATTN_ABS, check_encode=True):
+    BH = batch * H
+    C, R = pk.pk_resolve(n, cand_budget, collision_ratio, topk)
+    idx, score, dbg = search_debug(pk, h, q, BH, n, C, topk)
+    out = torch.empty(batch, H * G, 128, dtype=torch.float32, device="cuda")
+    pk.pk_attend(h, q, torch.from_numpy(idx).cuda(), topk, out)
+    st, det = pk.pk_last_device_error(h)
+    assert st == 0, (st, det)
+    out = out.cpu().numpy()
+    codes = rec = occ = None
+    if check_encode:
+        codes, rec, occ = export(pk, h, BH, n)
+    assert (idx >= 0).all() and (idx < n).all()
+    for p in pairs:
+        b, hh = divmod(p, H)
+        K_np = workloads.to_np_f32(K[b, hh, :n])
+        V_np = workloads.to_np_f32(V[b, hh, :n])
+        qg = workloads.to_np_f32(q[b, hh * G:(hh + 1) * G])
+        enc, orc = parity.oracle_pair(K_np, qg, topk, cand_budget, collision_ratio=collision_ratio)
+        assert orc["C"] == C and orc["R"] == R
+        if check_encode:
+            parity.check_encoding(enc, codes[p], rec[p], occ[p])
+        parity.check_search_pair(dbg, p, orc, enc, n)
+        parity.check_topk(idx[p], score[p], orc, enc)
+        o_ref = parity.oracle.attend(qg, K_np, V_np, idx[p], 1.0 / math.sqrt(128))
+        err = np.abs(out[b, hh * G:(hh + 1) * G] - o_ref).max()
+        assert err <= attn_tol, "attention max-abs %.3g" % err
+    return idx
+
+
+# ------------------------------------------------------------- configs
+def test_tiny_single_head_config(pk):
+    """1 KV head, n = 4096 fp32 keys with 4 outlier channels x8, 16 queries
+    q = K[j] + N(0, 0.5^2), subspace dim 8, C = 512, Top-100."""
+    w = workloads.tiny(seed=0, device="cuda")
+    h = build(pk, w["K"], w["V"], 4096, 1, 1, 1, cand_budget=512)
+    try:
+        for qi in range(16):
+            check_pairs(pk, h, w["K"], w["V"], w["q"][qi], [0], 1, 1, 1, 4096, 100,
+                        cand_budget=512, attn_tol=1e-4, check_encode=(qi == 0))
+    finally:
+        pk.pk_free(h)
+
+
+def test_llama_shaped_layer_config(pk):
+    """batch 1, 32 query heads, 8 KV heads (G = 4), n = 32768 bf16 keys with
+    LogNormal channel scales and RoPE; C = 2048; every pair checked."""
+    w = workloads.llama_layer(1, 32768, H=8, G=4, seed=0, device="cuda", n_queries=2)
+    h = build(pk, w["K"], w["V"], 32768, 1, 8, 4, cand_budget=2048)
+    try:
+        for qi in range(2):
+            check_pairs(pk, h, w["K"], w["V"], w["q"][qi], list(range(8)), 1, 8, 4, 32768, 100,
+                        cand_budget=2048, check_encode=(qi == 0))
+    finally:
+        pk.pk_free(h)
+
+
+@pytest.mark.parametrize("n,cand,topk,batch,H,G", [
+    (5000, 0, 100, 2, 2, 2),      # ratio table, ragged chunk tail, batch > 1
+    (100, 0, 100, 1, 1, 1),       # n == topk: every key is a candidate and returned
+    (1500, 1500, 37, 1, 2, 1),    # full budget C = n
+    (16, 0, 16, 1, 1, 1),         # smallest index
+    (3001, 0, 1, 1, 1, 3),        # topk = 1
+    (70001, 0, 100, 1, 1, 4),     # many compaction windows, odd n
+    (9000, 200, 200, 3, 1, 8),    # C == topk, G = 8
+])
+def test_edge_and_ragged_sizes(pk, n, cand, topk, batch, H, G):
+    w = workloads.llama_layer(batch, n, H=H, G=G, seed=n, device="cuda")
+    h = build(pk, w["K"], w["V"], n, batch, H, G, topk=topk, cand_budget=cand)
+    try:
+        check_pairs(pk, h, w["K"], w["V"], w["q"][0], list(range(batch * H)), batch, H, G, n, topk,
+                    cand_budget=cand)
+    finally:
+        pk.pk_free(h)
+
+
+def test_duplicate_keys_tie_rule(pk):
+    """Many identical keys: equal scores everywhere, so the lower-id rule
+    decides the candidate set and the Top-k, bit-exactly."""
+    base = workloads.llama_layer(1, 64, H=1, G=1, seed=5, device="cuda")
+    K = base["K"][:, :, :8].repeat(1, 1, 600, 1).contiguous()   # n = 4800, 8 distinct keys
+    V = base["V"][:, :, :8].repeat(1, 1, 600, 1).contiguous()
+    h = build(pk, K, V, 4800, 1, 1, 1, cand_budget=700)
+    try:
+        idx = check_pairs(pk, h, K, V, base["q"][0], [0], 1, 1, 1, 4800, 100, cand_budget=700)
+        assert len(set(idx[0].tolist())) == 100
+    finally:
+        pk.pk_free(h)
+
+
+def test_append_matches_oracle(pk):
+    """pk_append encodes new decode keys with the fixed codebook: the index
+    after appends equals an index built over all keys at once."""
+    w = workloads.llama_layer(1, 4200, H=2, G=2, seed=9, device="cuda")
+    K, V = w["K"], w["V"]
+    h = build(pk, K[:, :, :3000].contiguous(), V[:, :, :3000].contiguous(), 3000, 1, 2, 2,
+              n_cap=4200)
+    try:
+        for i in range(3000, 3005):
+            pk.pk_append(h, K[:, :, i:i + 1].contiguous(), V[:, :, i:i + 1].contiguous(), 1)
+        pk.pk_append(h, K[:, :, 3005:4200].contiguous(), V[:, :, 3005:4200].contiguous(), 1195)
+        assert pk.pk_get_info(h).n == 4200
+        with pytest.raises(pk.PkError) as e:
+            pk.pk_append(h, K[:, :, :1].contiguous(), V[:, :, :1].contiguous(), 1)
+        assert e.value.status == 2
+        check_pairs(pk, h, K, V, w["q"][0], [0, 1], 1, 2, 2, 4200, 100)
+    finally:
+        pk.pk_free(h)
+
+
+def test_host_pinned_kv_store(pk):
+    """K/V kept in pinned host memory and read through UVA by the attention."""
+    w = workloads.llama_layer(1, 20000, H=2, G=4, seed=3, device="cuda")
+    h = build(pk, w["K"], w["V"], 20000, 1, 2, 4, kv_location=1)
+    try:
+        assert pk.pk_get_info(h).kv_location == 1
+        check_pairs(pk, h, w["K"], w["V"], w["q"][0], [0, 1], 1, 2, 4, 20000, 100)
+    finally:
+        pk.pk_free(h)
+
+
+def test_attend_out_of_range_ids_are_skipped_and_recorded(pk):
+    w = workloads.llama_layer(1, 500, H=1, G=1, seed=4, device="cuda")
+    h = build(pk, w["K"], w["V"], 500, 1, 1, 1)
+    try:
+        sel = torch.arange(100, dtype=torch.int32, device="cuda").view(1, 100)
+        sel[0, 7] = 505
+        out = torch.empty(1, 1, 128, dtype=torch.float32, device="cuda")
+        pk.pk_attend(h, w["q"][0], sel, 100, out)
+        st, det = pk.pk_last_device_error(h)
+        assert st == 6 and det == 505
+        assert torch.isfinite(out).all()
+        keep = [i for i in range(100) if i != 7]
+        ref = parity.oracle.attend(workloads.to_np_f32(w["q"][0, 0]), workloads.to_np_f32(w["K"][0, 0]),
+                                   workloads.to_np_f32(w["V"][0, 0]), np.array(keep, np.int32),
+                                   1.0 / math.sqrt(128))
+        assert np.abs(out[0].cpu().numpy() - ref).max() <= parity.ATTN_ABS
+        assert pk.pk_last_device_error(h)[0] == 0
+    finally:
+        pk.pk_free(h)
+
+
+def test_search_rejects_bad_arguments(pk):
+    w = workloads.llama_layer(1, 300, H=1, G=1, seed=6, device="cuda")
+    h = build(pk, w["K"], w["V"], 300, 1, 1, 1)
+    try:
+        idx = torch.empty(1, 100, dtype=torch.int32, device="cuda")
+        with pytest.raises(pk.PkError) as e:
+            pk.pk_search(h, w["q"][0], 101, idx)
+        assert e.value.status == 1
+        host = np.zeros((1, 1, 128), np.float32)        # pageable host memory
+        with pytest.raises(pk.PkError) as e:
+            pk.pk_search(h, host.ctypes.data, 100, idx)
+        assert e.value.status == 1
+    finally:
+        pk.pk_free(h)
+
+
+# ------------------------------------------------- full-size workloads
+def test_throughput_batch_full_size_sampled(pk):
+    """8 sequences x n = 131072, 8 KV heads, 32 query heads, bf16, ratio-table
+    budgets (C = 13108, R = 26215), K/V in HBM: the benchmark's workload and
+    launch configuration; two sampled pairs checked against the oracle."""
+    batch, n, H, G = 8, 131072, 8, 4
+    w = workloads.llama_layer(batch, n, H=H, G=G, seed=0, device="cuda")
+    h = build(pk, w["K"], w["V"], n, batch, H, G)
+    try:
+        idx = check_pairs(pk, h, w["K"], w["V"], w["q"][0], [0, 45], batch, H, G, n, 100,
+                          check_encode=True)
+        for p in range(batch * H):
+            assert len(set(idx[p].tolist())) == 100
+    finally:
+        pk.pk_free(h)
+        del w
+        torch.cuda.empty_cache()
+
+
+def test_million_token_offload_sampled(pk):
+    """batch 1, n = 1048576, 8 KV heads, bf16, full K/V (4 GiB) in pinned host
+    memory, codes + summaries on the GPU, Top-100 fetched through UVA."""
+    n, H, G = 1 << 20, 8, 4
+    w = workloads.llama_layer(1, n, H=H, G=G, seed=1, device="cuda")
+    h = build(pk, w["K"], w["V"], n, 1, H, G, kv_location=1)
+    try:
+        check_pairs(pk, h, w["K"], w["V"], w["q"][0], [5], 1, H, G, n, 100, check_encode=False)
+    finally:
+        pk.pk_free(h)
+        del w
+        torch.cuda.empty_cache()

@@ -66,6 +66,27 @@ def tiny(seed: int = 0, device="cpu", n: int = 4096, D: int = 128, n_queries: in
                 q=q.view(n_queries, 1, 1, D).contiguous(), qsrc=j)
 
 
+def llama_pair(b: int, h: int, n: int, H: int = 8, G: int = 4, D: int = 128, seed: int = 0,
+               device="cpu", n_queries: int = 1, dtype=torch.bfloat16, noise: float = 0.5,
+               rope: bool = True):
+    """One (sequence b, KV head h) pair of the Llama-shaped layer: K, V [n][D]
+    and its G query heads q [n_queries][G][D].  Drawn from the pair's own
+    generator, so any pair can be regenerated alone."""
+    g = _gen(device, seed, b * H + h)
+    sig = torch.exp(0.5 * torch.randn(D, generator=g, device=device))
+    sigv = torch.exp(0.5 * torch.randn(D, generator=g, device=device))
+    k = torch.randn(n, D, generator=g, device=device) * sig
+    if rope:
+        k = rope_rotate_half(k)
+    K = k.to(dtype)
+    del k
+    V = (torch.randn(n, D, generator=g, device=device) * sigv).to(dtype)
+    j = torch.randint(0, n, (n_queries, G), generator=g, device=device)
+    kq = K.float()[j.reshape(-1)].reshape(n_queries, G, D)
+    q = (kq + noise * sig * torch.randn(n_queries, G, D, generator=g, device=device)).to(dtype)
+    return K, V, q
+
+
 def llama_layer(batch: int, n: int, H: int = 8, G: int = 4, D: int = 128, seed: int = 0,
                 device="cpu", n_queries: int = 1, dtype=torch.bfloat16, noise: float = 0.5,
                 rope: bool = True):
@@ -78,19 +99,12 @@ def llama_layer(batch: int, n: int, H: int = 8, G: int = 4, D: int = 128, seed: 
     q = torch.empty(n_queries, batch, H * G, D, dtype=dtype, device=device)
     for b in range(batch):
         for h in range(H):
-            g = _gen(device, seed, b * H + h)
-            sig = torch.exp(0.5 * torch.randn(D, generator=g, device=device))
-            sigv = torch.exp(0.5 * torch.randn(D, generator=g, device=device))
-            k = torch.randn(n, D, generator=g, device=device) * sig
-            if rope:
-                k = rope_rotate_half(k)
-            K[b, h] = k.to(dtype)
-            V[b, h] = (torch.randn(n, D, generator=g, device=device) * sigv).to(dtype)
-            j = torch.randint(0, n, (n_queries, G), generator=g, device=device)
-            kq = K[b, h].float()[j.reshape(-1)].reshape(n_queries, G, D)
-            qq = kq + noise * sig * torch.randn(n_queries, G, D, generator=g, device=device)
-            q[:, b, h * G:(h + 1) * G] = qq.to(dtype)
-            del k
+            k_, v_, q_ = llama_pair(b, h, n, H=H, G=G, D=D, seed=seed, device=device,
+                                    n_queries=n_queries, dtype=dtype, noise=noise, rope=rope)
+            K[b, h] = k_
+            V[b, h] = v_
+            q[:, b, h * G:(h + 1) * G] = q_
+            del k_, v_, q_
     return dict(K=K, V=V, q=q)
 
 
