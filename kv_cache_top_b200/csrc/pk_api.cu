@@ -19,6 +19,7 @@ struct pk_index {
     pk_params p;
     int32_t bh = 0;
     int64_t n = 0;
+    int64_t stride = 0;          // rows per pair in every per-key array (n_cap rounded up to 16)
     int device = 0;
     int num_sms = 148;
     int32_t max_chunks = 1;
@@ -202,7 +203,7 @@ pk_status encode_range(pk_index *ix, const void *Kin, int64_t n_new, int64_t pos
     a.K = Kin;
     a.n_new = n_new;
     a.pos0 = pos0;
-    a.n_cap = ix->p.n_cap;
+    a.n_cap = ix->stride;
     a.bh = ix->bh;
     a.is_bf16 = ix->p.kv_dtype == PK_BF16;
     a.codes = ix->codes;
@@ -221,7 +222,7 @@ pk_status copy_rows(pk_index *ix, void *store, const void *src, int64_t n_new, i
                     cudaStream_t s)
 {
     const size_t row = (size_t)kD * ix->es;
-    cudaError_t e = cudaMemcpy2DAsync((char *)store + (size_t)pos0 * row, (size_t)ix->p.n_cap * row,
+    cudaError_t e = cudaMemcpy2DAsync((char *)store + (size_t)pos0 * row, (size_t)ix->stride * row,
                                       src, (size_t)n_new * row, (size_t)n_new * row, (size_t)ix->bh,
                                       cudaMemcpyDefault, s);
     return cuda_status(e);
@@ -272,7 +273,7 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     sa.codes = ix->codes;
     sa.bonus_packed = ix->bonus_packed;
     sa.n = ix->n;
-    sa.n_cap = ix->p.n_cap;
+    sa.n_cap = ix->stride;
     sa.chunk = chunk;
     sa.C = C;
     sa.nchunks = nchunks;
@@ -301,7 +302,7 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     ra.chunk_info = ix->chunk_info;
     ra.sstar = ix->sstar;
     ra.n = ix->n;
-    ra.n_cap = ix->p.n_cap;
+    ra.n_cap = ix->stride;
     ra.chunk = chunk;
     ra.C = C;
     ra.nchunks = nchunks;
@@ -399,7 +400,8 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     pk_index *ix = new (std::nothrow) pk_index();
     if (!ix) return PK_ERR_OOM;
     ix->p = *params;
-    ix->p.n_cap = ceil_div(n_cap, 16) * 16;   // keeps every per-pair row 16-byte aligned
+    ix->p.n_cap = n_cap;
+    ix->stride = ceil_div(n_cap, 16) * 16;    // keeps every per-pair row 16-byte aligned
     ix->bh = params->batch * params->n_kv_heads;
     ix->es = es;
     ix->topk_cap = params->topk;
@@ -429,7 +431,7 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
         for (int t = 0; t < kL - 1; t++) ix->lv.thr[t] = (float)thr[t];
     }
 
-    const size_t BH = ix->bh, NC = ix->p.n_cap, MC = ix->max_chunks;
+    const size_t BH = ix->bh, NC = ix->stride, MC = ix->max_chunks;
     e = cudaSuccess;
     auto chk = [&](cudaError_t x) { if (e == cudaSuccess) e = x; };
     chk(dalloc(&ix->codes, BH * NC * kB));
@@ -522,7 +524,7 @@ pk_status pk_attend(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t
     a.V = ix->V;
     a.out = out;
     a.n = ix->n;
-    a.n_cap = ix->p.n_cap;
+    a.n_cap = ix->stride;
     a.H = ix->p.n_kv_heads;
     a.G = ix->p.group;
     a.topk = topk;
@@ -569,8 +571,8 @@ pk_status pk_get_info(const pk_index *ix, pk_info *info)
     info->bh = ix->bh;
     chunking(ix, ix->n, &info->nchunks, &info->chunk);
     resolve(ix->n, ix->p.cand_budget, ix->p.collision_ratio, ix->p.topk, &info->cand, &info->coll);
-    info->index_bytes = (int64_t)ix->bh * ix->p.n_cap * (kB + kRecBytes) + (int64_t)ix->bh * kB * kNC * 4;
-    info->kv_bytes = 2 * (int64_t)ix->bh * ix->p.n_cap * kD * ix->es;
+    info->index_bytes = (int64_t)ix->bh * ix->stride * (kB + kRecBytes) + (int64_t)ix->bh * kB * kNC * 4;
+    info->kv_bytes = 2 * (int64_t)ix->bh * ix->stride * kD * ix->es;
     info->kv_location = ix->p.kv_location;
     info->num_sms = ix->num_sms;
     return PK_OK;
@@ -583,10 +585,10 @@ pk_status pk_export_index(const pk_index *ix, uint8_t *codes, uint8_t *records, 
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaSuccess;
     if (codes)
-        e = cudaMemcpy2DAsync(codes, (size_t)ix->n * kB, ix->codes, (size_t)ix->p.n_cap * kB,
+        e = cudaMemcpy2DAsync(codes, (size_t)ix->n * kB, ix->codes, (size_t)ix->stride * kB,
                               (size_t)ix->n * kB, ix->bh, cudaMemcpyDefault, s);
     if (e == cudaSuccess && records)
-        e = cudaMemcpy2DAsync(records, (size_t)ix->n * kRecBytes, ix->rec, (size_t)ix->p.n_cap * kRecBytes,
+        e = cudaMemcpy2DAsync(records, (size_t)ix->n * kRecBytes, ix->rec, (size_t)ix->stride * kRecBytes,
                               (size_t)ix->n * kRecBytes, ix->bh, cudaMemcpyDefault, s);
     if (e == cudaSuccess && occ)
         e = cudaMemcpyAsync(occ, ix->occ, (size_t)ix->bh * kB * kNC * sizeof(uint32_t), cudaMemcpyDefault, s);
