@@ -154,6 +154,7 @@ def profiled_traffic(kernel: str, workload: str):
     hm = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
     files = {"collision_scan": ["k_collision_scan.cu", "pk_internal.cuh"],
              "rerank_topk": ["k_rerank_topk.cu", "pk_internal.cuh"],
+             "compact": ["k_compact.cu", "pk_internal.cuh"],
              "query_prep": ["k_query_prep.cu", "pk_internal.cuh"],
              "gather_attend": ["k_gather_attend.cu", "pk_internal.cuh"]}.get(kernel)
     if not m or not hm or not files or hm.group(1) != src_hash(*files):
@@ -169,8 +170,10 @@ def alg_bytes(kernel: str, wl: dict, C: int, topk: int = 100):
         return bh * (G * 128 * 2 + 16 * 256 * 4 + 16 * 32 * 4 + 128 * 4)
     if kernel == "collision_scan":
         return bh * (16 * n + n)                     # codes read + S written
+    if kernel == "compact":
+        return bh * (n + 4 * C)                      # S read + candidate ids written
     if kernel == "rerank_topk":
-        return bh * (n + 128 * C + 8 * topk)         # S read + candidate records + result
+        return bh * (132 * C + 8 * topk)             # ids + candidate records + result
     if kernel == "gather_attend":
         return bh * (2 * topk * 128 * 2 + G * 128 * (2 + 4))   # K/V rows + q + o
     raise KeyError(kernel)
@@ -425,7 +428,8 @@ def main():
         att = km.get("gather_attend", {})
         mil = {"workload": wl_m["name"], "steps_s": margs.steps * world / (rm["ms_total"] / 1000.0),
                "ms_per_step": rm["ms_total"] / margs.steps, "steps": margs.steps,
-               "search_us": sum(km[k]["avg_us"] for k in ("query_prep", "collision_scan", "rerank_topk") if k in km),
+               "search_us": sum(km[k]["avg_us"] for k in ("query_prep", "collision_scan", "compact", "rerank_topk")
+                                if k in km),
                "attend_us": att.get("avg_us"), "recall_at_100": rm["recall"],
                "uva_bytes_per_step": link_bytes,
                "host_link_gbs": (link_bytes / (att["avg_us"] * 1e-6) / 1e9) if att else None,
@@ -477,7 +481,7 @@ def main():
                      "unit": "GB/s", "frac": km[dom]["gbs"] / peak,
                      "traffic": profiled_traffic(dom, wl["name"]), "peak_source": peak_src},
         "kernels": km,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 5 * args.steps,
         "clocks": res["clocks"],
         "e2e": res["e2e"],
         "cpu_baseline": res.get("cpu"),

@@ -14,7 +14,13 @@
 // Hot loop: 16 B of codes per key read with 128-bit streaming loads; the 16
 // bonus tables (4 bits x 256 centres = one 32-bit register per lane per
 // block) live in registers and are read with warp shuffles, which have no
-// bank conflicts whatever the codes are.
+// bank conflicts whatever the codes are.  Lane l's word of block b holds in
+// nibble t the bonus of centre 32 t + l, so a code byte c is used as it is:
+// its low 5 bits pick the lane (the shuffle ignores higher bits), and
+// 4 (c >> 5) -- all four computed at once per 32-bit code word -- is the
+// shift of a wrap-mode funnel shift (which ignores bits above 4).  Two
+// extracted bonuses (each <= 6) are added before one mask, since their sum
+// still fits in the low nibble.
 #include "pk_internal.cuh"
 
 namespace pk {
@@ -23,20 +29,23 @@ constexpr int kScanThreads = 256;
 constexpr int kScanUnroll = 4;
 constexpr int kHistPad = 104;
 
-__device__ __forceinline__ uint32_t lookup_bonus(const uint32_t (&tab)[kB], int b, uint32_t code)
-{
-    const uint32_t w = __shfl_sync(kFull, tab[b], (int)(code >> 3));
-    return (w >> ((code & 7u) << 2)) & 0xfu;
-}
-
 __device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], uint4 c)
 {
     uint32_t s = 0;
     const uint32_t wds[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int q = 0; q < 4; q++) {
-#pragma unroll
-        for (int k = 0; k < 4; k++) s += lookup_bonus(tab, 4 * q + k, (wds[q] >> (8 * k)) & 0xffu);
+        const uint32_t w = wds[q];
+        const uint32_t A = (w >> 3) & 0x1c1c1c1cu;      // byte k: 4 * (c_k >> 5)
+        const uint32_t v0 = __shfl_sync(kFull, tab[4 * q + 0], (int)w);
+        const uint32_t v1 = __shfl_sync(kFull, tab[4 * q + 1], (int)(w >> 8));
+        const uint32_t v2 = __shfl_sync(kFull, tab[4 * q + 2], (int)(w >> 16));
+        const uint32_t v3 = __shfl_sync(kFull, tab[4 * q + 3], (int)(w >> 24));
+        const uint32_t x0 = __funnelshift_r(v0, 0u, A);
+        const uint32_t x1 = __funnelshift_r(v1, 0u, A >> 8);
+        const uint32_t x2 = __funnelshift_r(v2, 0u, A >> 16);
+        const uint32_t x3 = __funnelshift_r(v3, 0u, A >> 24);
+        s += ((x0 + x1) & 0xfu) + ((x2 + x3) & 0xfu);
     }
     return s;
 }

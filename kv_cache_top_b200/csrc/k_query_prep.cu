@@ -11,27 +11,31 @@
 //     better-ranked buckets (from the occupancy table), and a bucket inside
 //     the top-rho fraction (P(c) < R = ceil(rho n)) gets bonus 6 - floor(6P/R).
 //
-// One CTA of 16 warps per pair; warp 0 rotates, then warp b ranks block b with
-// a register bitonic sort of 256 keys (8 per lane).  Output: the 16 bonus
-// tables packed 4 bits per centre (32 words per block), the form the
-// collision scan keeps in registers.
+// Grid (16 blocks, pairs): CTA (b, pair) ranks the 256 centres of block b, one
+// thread per centre, by counting the centres that precede it (broadcast
+// shared-memory reads, no sort).  Output: the bonus table packed 4 bits per
+// centre in the layout the collision scan keeps in registers -- lane l's word
+// holds, in nibble t, the bonus of centre 32 t + l.
 #include "pk_internal.cuh"
 
 namespace pk {
 
-__global__ void __launch_bounds__(512) k_query_prep(PrepArgs a)
+__global__ void __launch_bounds__(256) k_query_prep(PrepArgs a)
 {
-    const int bh = blockIdx.x;
+    const int b = blockIdx.x, bh = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b_seq = bh / a.H, h = bh - b_seq * a.H;
     __shared__ float s_q[kD];
     __shared__ float s_qt[kD];
-    __shared__ uint8_t s_bonus[kB][kNC];
+    __shared__ float s_L[kNC];
+    __shared__ uint32_t s_occ_ranked[kNC];
+    __shared__ uint8_t s_bonus[kNC];
+    __shared__ uint32_t s_ws[9];
 
-    // reset the per-call counters of the collision scan and the rerank
-    if (tid < kBins) a.head_hist[(size_t)bh * kBins + tid] = 0u;
-    if (tid < 2) a.tickets[(size_t)bh * 2 + tid] = 0u;
-
+    if (b == 0) {   // reset the per-call counters of the collision scan and the rerank
+        if (tid < kBins) a.head_hist[(size_t)bh * kBins + tid] = 0u;
+        if (tid < 2) a.tickets[(size_t)bh * 2 + tid] = 0u;
+    }
     if (tid < kD) {
         const int64_t base = ((int64_t)b_seq * a.H * a.G + (int64_t)h * a.G) * kD + tid;
         float acc = ld_as_f32(a.q, base, a.is_bf16);
@@ -45,97 +49,58 @@ __global__ void __launch_bounds__(512) k_query_prep(PrepArgs a)
         for (int r = 0; r < 4; r++) x[r] = s_q[lane + 32 * r];
         const float nrm = warp_rotate128(x, a.rot, lane);
 #pragma unroll
-        for (int r = 0; r < 4; r++) {
-            s_qt[lane + 32 * r] = x[r];
-            a.qt[(size_t)bh * kD + lane + 32 * r] = x[r];
-            if (a.dbg_qt) a.dbg_qt[(size_t)bh * kD + lane + 32 * r] = x[r];
-        }
-        if (lane == 0) {
-            a.qnorm[bh] = nrm;
-            if (a.dbg_qnorm) a.dbg_qnorm[bh] = nrm;
+        for (int r = 0; r < 4; r++) s_qt[lane + 32 * r] = x[r];
+        if (b == 0) {
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                a.qt[(size_t)bh * kD + lane + 32 * r] = x[r];
+                if (a.dbg_qt) a.dbg_qt[(size_t)bh * kD + lane + 32 * r] = x[r];
+            }
+            if (lane == 0) {
+                a.qnorm[bh] = nrm;
+                if (a.dbg_qnorm) a.dbg_qnorm[bh] = nrm;
+            }
         }
     }
     __syncthreads();
 
-    // ---- warp b: rank the 256 centres of block b
-    const int b = warp;
-    float xq[kM];
+    // centre c = tid: score L_b(c), summed over j = 0..7 in order
+    const int c = tid;
+    float L = 0.0f;
 #pragma unroll
-    for (int j = 0; j < kM; j++) xq[j] = s_qt[b * kM + j];
-    // element e = 8 lane + i is centre c = e; sort key (ascending order =
-    // rank order): high 32 bits = ~ord(L) (L desc), low 8 bits = c (c asc)
-    unsigned long long key[8];
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const int c = lane * 8 + i;
-        float L = 0.0f;
-#pragma unroll
-        for (int j = 0; j < kM; j++) L = __fadd_rn(L, ((c >> j) & 1) ? -xq[j] : xq[j]);
-        L = __fadd_rn(L, 0.0f);   // fold -0 into +0 so equal scores tie
-        key[i] = ((unsigned long long)(~ord_f32(L)) << 8) | (unsigned)c;
+    for (int j = 0; j < kM; j++) {
+        const float x = s_qt[b * kM + j];
+        L = __fadd_rn(L, ((c >> j) & 1) ? -x : x);
     }
-    // bitonic sort, ascending, 256 elements over the warp
-#pragma unroll
-    for (int k = 2; k <= 256; k <<= 1) {
-#pragma unroll
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
-            if (jj >= 8) {
-                const int lx = jj >> 3;
-#pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const int e = lane * 8 + i;
-                    const unsigned long long o = __shfl_xor_sync(kFull, key[i], lx);
-                    const bool lower = (e & jj) == 0, up = (e & k) == 0;
-                    const bool take_min = (lower == up);
-                    key[i] = take_min ? (o < key[i] ? o : key[i]) : (o > key[i] ? o : key[i]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    if ((i & jj) == 0) {
-                        const int e = lane * 8 + i;
-                        const bool up = (e & k) == 0;
-                        const unsigned long long x0 = key[i], x1 = key[i ^ jj];
-                        const unsigned long long lo = x0 < x1 ? x0 : x1, hi = x0 < x1 ? x1 : x0;
-                        key[i] = up ? lo : hi;
-                        key[i ^ jj] = up ? hi : lo;
-                    }
-                }
-            }
-        }
+    L = __fadd_rn(L, 0.0f);   // fold -0 into +0 so equal scores tie
+    s_L[c] = L;
+    __syncthreads();
+    // rank = #{c' : L(c') > L(c) or (L(c') == L(c) and c' < c)}
+    int rank = 0;
+#pragma unroll 8
+    for (int c2 = 0; c2 < kNC; c2++) {
+        const float L2 = s_L[c2];
+        rank += (L2 > L || (L2 == L && c2 < c)) ? 1 : 0;
     }
-    // exclusive prefix of bucket sizes in rank order -> tier bonus
-    const uint32_t *occ = a.occ + ((size_t)bh * kB + b) * kNC;
-    uint32_t cnt[8], run = 0;
+    const uint32_t cnt = a.occ[((size_t)bh * kB + b) * kNC + c];
+    s_occ_ranked[rank] = cnt;
+    __syncthreads();
+    uint32_t tot;
+    const uint32_t excl = block_excl_scan<256>(s_occ_ranked[tid], s_ws, &tot);   // prefix in rank order
+    __syncthreads();
+    s_occ_ranked[tid] = excl;          // now: P of the bucket at rank tid
+    __syncthreads();
+    const uint32_t P = s_occ_ranked[rank];
+    uint32_t bon = 0;
+    if ((int64_t)P < a.R) bon = 6u - (uint32_t)((6ull * P) / (unsigned long long)a.R);
+    s_bonus[c] = (uint8_t)bon;
+    if (a.dbg_bonus) a.dbg_bonus[((size_t)bh * kB + b) * kNC + c] = (uint8_t)bon;
+    __syncthreads();
+    if (tid < 32) {
+        uint32_t word = 0;
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        cnt[i] = occ[key[i] & 0xffu];
-        run += cnt[i];
-    }
-    uint32_t incl = run;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += y;
-    }
-    uint32_t P = incl - run;
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const int c = (int)(key[i] & 0xffu);
-        uint32_t bon = 0;
-        if ((int64_t)P < a.R) bon = 6u - (uint32_t)((6ull * P) / (unsigned long long)a.R);
-        s_bonus[b][c] = (uint8_t)bon;
-        P += cnt[i];
-    }
-    __syncwarp();
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < 8; i++) word |= (uint32_t)s_bonus[b][lane * 8 + i] << (4 * i);
-    a.bonus_packed[((size_t)bh * kB + b) * 32 + lane] = word;
-    if (a.dbg_bonus) {
-#pragma unroll
-        for (int i = 0; i < 8; i++)
-            a.dbg_bonus[((size_t)bh * kB + b) * kNC + lane * 8 + i] = s_bonus[b][lane * 8 + i];
+        for (int t = 0; t < 8; t++) word |= (uint32_t)s_bonus[32 * t + tid] << (4 * t);
+        a.bonus_packed[((size_t)bh * kB + b) * 32 + tid] = word;
     }
 }
 
@@ -144,7 +109,7 @@ __global__ void __launch_bounds__(512) k_query_prep(PrepArgs a)
 namespace pk {
 cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s)
 {
-    k_query_prep<<<a.bh, 512, 0, s>>>(a);
+    k_query_prep<<<dim3(kB, a.bh), 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 }  // namespace pk

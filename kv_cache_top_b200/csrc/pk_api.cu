@@ -42,7 +42,12 @@ struct pk_index {
     uint32_t *chunk_cum = nullptr, *head_hist = nullptr, *tickets = nullptr;
     uint2 *chunk_info = nullptr;
     int32_t *sstar = nullptr;
+    int32_t *cand = nullptr;
     unsigned long long *partial = nullptr;
+    int32_t max_slices = 1;
+    float *att_part = nullptr;
+    uint32_t *att_tickets = nullptr;
+    int32_t max_splits = 1;
     int32_t *dev_err = nullptr;
     long long *dev_err_detail = nullptr;
     // tracing
@@ -123,6 +128,28 @@ void chunking(const pk_index *ix, int64_t n, int32_t *nchunks, int64_t *chunk)
     *nchunks = (int32_t)ceil_div(n, ch);
 }
 
+// rerank work split: slices of the candidate list, ~3 CTAs per SM in total
+int32_t slice_lo(const pk_index *ix) { return std::max<int32_t>(256, 2 * ix->topk_cap); }
+
+void slicing(const pk_index *ix, int64_t C, int32_t *slice, int32_t *nslices)
+{
+    const int64_t target = 3 * (int64_t)ix->num_sms;
+    int64_t sl = ceil_div(ceil_div(C * ix->bh, target), 64) * 64;
+    sl = std::max<int64_t>(sl, slice_lo(ix));
+    sl = std::min<int64_t>(sl, kMaxSlice);
+    *slice = (int32_t)sl;
+    *nslices = (int32_t)ceil_div(C, sl);
+}
+
+// attention work split: up to kAtRows selected rows per CTA
+void splitting(const pk_index *ix, int32_t topk, int32_t *rows_per, int32_t *nsplit)
+{
+    int64_t rp = ceil_div((int64_t)topk * ix->bh, 2 * (int64_t)ix->num_sms);
+    rp = std::max<int64_t>(8, std::min<int64_t>(rp, kAtRows));
+    *nsplit = (int32_t)ceil_div(topk, rp);
+    *rows_per = (int32_t)ceil_div(topk, *nsplit);
+}
+
 void free_all(pk_index *ix)
 {
     if (!ix) return;
@@ -145,7 +172,10 @@ void free_all(pk_index *ix)
     cudaFree(ix->tickets);
     cudaFree(ix->chunk_info);
     cudaFree(ix->sstar);
+    cudaFree(ix->cand);
     cudaFree(ix->partial);
+    cudaFree(ix->att_part);
+    cudaFree(ix->att_tickets);
     cudaFree(ix->dev_err);
     cudaFree(ix->dev_err_detail);
     for (cudaEvent_t e : ix->ev_pool) cudaEventDestroy(e);
@@ -294,30 +324,41 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     trace_end(ix, s);
     if (e != cudaSuccess) return cuda_status(e);
 
+    CompactArgs ca{};
+    ca.S = ix->S;
+    ca.chunk_info = ix->chunk_info;
+    ca.sstar = ix->sstar;
+    ca.n = ix->n;
+    ca.stride = ix->stride;
+    ca.chunk = chunk;
+    ca.C = C;
+    ca.max_chunks = ix->max_chunks;
+    ca.cand = ix->cand;
+    ca.dbg_cand = dbg ? dbg->cand : nullptr;
+    ca.dev_err = ix->dev_err;
+    trace_begin(ix, PK_K_COMPACT, s);
+    e = launch_compact(ca, nchunks, ix->bh, s);
+    trace_end(ix, s);
+    if (e != cudaSuccess) return cuda_status(e);
+
     RerankArgs ra{};
-    ra.S = ix->S;
+    ra.cand = ix->cand;
     ra.rec = ix->rec;
     ra.qt = ix->qt;
     ra.qnorm = ix->qnorm;
-    ra.chunk_info = ix->chunk_info;
-    ra.sstar = ix->sstar;
-    ra.n = ix->n;
-    ra.n_cap = ix->stride;
-    ra.chunk = chunk;
+    ra.stride = ix->stride;
     ra.C = C;
-    ra.nchunks = nchunks;
-    ra.max_chunks = ix->max_chunks;
+    slicing(ix, C, &ra.slice, &ra.nslices);
+    if (ra.nslices > ix->max_slices) return PK_ERR_CAPACITY;
+    ra.max_slices = ix->max_slices;
     ra.topk = topk;
+    ra.topk_cap = ix->topk_cap;
     ra.tickets = ix->tickets;
     ra.partial = ix->partial;
-    ra.topk_cap = ix->topk_cap;
     ra.lv = ix->lv;
     ra.out_idx = out_idx;
     ra.out_score = out_score;
-    if (dbg) {
-        ra.dbg_cand = dbg->cand;
-        ra.dbg_est = dbg->cand_est;
-    }
+    ra.dbg_est = dbg ? dbg->cand_est : nullptr;
     ra.dev_err = ix->dev_err;
     trace_begin(ix, PK_K_RERANK_TOPK, s);
     e = launch_rerank_topk(ra, ix->bh, s);
@@ -446,7 +487,18 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(dalloc(&ix->tickets, BH * 2));
     chk(dalloc(&ix->chunk_info, BH * MC));
     chk(dalloc(&ix->sstar, BH));
-    chk(dalloc(&ix->partial, BH * MC * (size_t)ix->topk_cap));
+    {   // largest slice count any C <= n_cap can need
+        const int64_t lo = slice_lo(ix);
+        const int64_t by_target = ceil_div(3 * (int64_t)ix->num_sms, ix->bh) + 1;
+        ix->max_slices = (int32_t)std::max<int64_t>(std::min<int64_t>(ceil_div(n_cap, lo), by_target),
+                                                    ceil_div(n_cap, kMaxSlice)) + 1;
+        ix->max_splits = (int32_t)ceil_div(ix->topk_cap, 8);
+    }
+    const size_t MS = ix->max_slices;
+    chk(dalloc(&ix->cand, BH * NC));
+    chk(dalloc(&ix->partial, BH * MS * (size_t)ix->topk_cap));
+    chk(dalloc(&ix->att_part, BH * (size_t)ix->max_splits * kMaxGroup * (kD + 2)));
+    chk(dalloc(&ix->att_tickets, BH));
     chk(dalloc(&ix->dev_err, 1));
     chk(dalloc(&ix->dev_err_detail, 1));
     const size_t kv_bytes = BH * NC * kD * (size_t)es;
@@ -467,6 +519,7 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(cudaMemsetAsync(ix->occ, 0, BH * kB * kNC * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->head_hist, 0, BH * kBins * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->tickets, 0, BH * 2 * sizeof(uint32_t), s));
+    chk(cudaMemsetAsync(ix->att_tickets, 0, BH * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->dev_err, 0, sizeof(int32_t), s));
     chk(cudaMemsetAsync(ix->dev_err_detail, 0, sizeof(long long), s));
     if (e == cudaSuccess) st = copy_rows(ix, ix->K, K, n, 0, s);
@@ -524,12 +577,16 @@ pk_status pk_attend(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t
     a.V = ix->V;
     a.out = out;
     a.n = ix->n;
-    a.n_cap = ix->stride;
+    a.stride = ix->stride;
     a.H = ix->p.n_kv_heads;
     a.G = ix->p.group;
     a.topk = topk;
     a.is_bf16 = ix->p.kv_dtype == PK_BF16;
     a.scale = ix->scale;
+    splitting(ix, topk, &a.rows_per, &a.nsplit);
+    a.max_splits = ix->max_splits;
+    a.part = ix->att_part;
+    a.tickets = ix->att_tickets;
     a.dev_err = ix->dev_err;
     a.dev_err_detail = ix->dev_err_detail;
     cudaStream_t s = (cudaStream_t)stream;

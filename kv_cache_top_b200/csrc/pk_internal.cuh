@@ -21,6 +21,8 @@ constexpr int kCum = kBins + 1;  // suffix-count entries per chunk (98, last = 0
 constexpr int kRecBytes = 128;   // 4-bit summary record per key
 constexpr int kMaxTopk = 1024;
 constexpr int kMaxGroup = 8;
+constexpr int kMaxSlice = 4096;  // candidates per rerank CTA (upper bound)
+constexpr int kAtRows = 32;      // selected rows per attention CTA (upper bound)
 constexpr unsigned kFull = 0xffffffffu;
 
 // Device-check codes written to the index's error word (first one wins).
@@ -69,7 +71,7 @@ struct PrepArgs {
 struct ScanArgs {
     const uint8_t *codes;
     const uint32_t *bonus_packed;
-    int64_t n, n_cap, chunk, C;
+    int64_t n, n_cap, chunk, C;   // n_cap: row stride of the per-key arrays
     int32_t nchunks;
     uint8_t *S;              // [BH][n_cap]
     uint32_t *chunk_cum;     // [BH][max_chunks][kCum]
@@ -83,22 +85,29 @@ struct ScanArgs {
     int32_t *dbg_sstar;
 };
 
-struct RerankArgs {
+struct CompactArgs {
     const uint8_t *S;
+    const uint2 *chunk_info;
+    const int32_t *sstar;
+    int64_t n, stride, chunk, C;
+    int32_t max_chunks;
+    int32_t *cand;           // [BH][stride]  candidate ids, ascending
+    int32_t *dbg_cand;       // [BH][C] or null
+    int32_t *dev_err;
+};
+
+struct RerankArgs {
+    const int32_t *cand;     // [BH][stride]
     const uint8_t *rec;
     const float *qt;
     const float *qnorm;
-    const uint2 *chunk_info;
-    const int32_t *sstar;
-    int64_t n, n_cap, chunk, C;
-    int32_t nchunks, max_chunks, topk;
+    int64_t stride, C;
+    int32_t slice, nslices, max_slices, topk, topk_cap;
     uint32_t *tickets;
-    unsigned long long *partial;   // [BH][max_chunks][topk_cap]
-    int32_t topk_cap;
+    unsigned long long *partial;   // [BH][max_slices][topk_cap]
     Levels lv;
     int32_t *out_idx;        // [BH][topk]
     float *out_score;        // [BH][topk] or null
-    int32_t *dbg_cand;       // [BH][C] or null
     float *dbg_est;          // [BH][C] or null
     int32_t *dev_err;
 };
@@ -106,11 +115,14 @@ struct RerankArgs {
 struct AttendArgs {
     const void *q;           // [batch][H*G][D]
     const int32_t *idx;      // [BH][topk]
-    const void *K;           // [BH][n_cap][D]  (device or mapped host)
+    const void *K;           // [BH][stride][D]  (device or mapped host)
     const void *V;
     float *out;              // [batch][H*G][D]
-    int64_t n, n_cap;
+    int64_t n, stride;
     int32_t H, G, topk, is_bf16;
+    int32_t rows_per, nsplit, max_splits;
+    float *part;             // [BH][max_splits][kMaxGroup][D + 2]
+    uint32_t *tickets;       // [BH]
     float scale;
     int32_t *dev_err;
     long long *dev_err_detail;
@@ -235,9 +247,10 @@ namespace pk {
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s);
 cudaError_t launch_collision_scan(const ScanArgs &a, int bh, cudaStream_t s);
+cudaError_t launch_compact(const CompactArgs &a, int nchunks, int bh, cudaStream_t s);
 cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s);
-size_t gather_attend_smem(int is_bf16);
+size_t rerank_smem(int slice);
 // host-side Lloyd-Max levels of the magnitude prior (closed-form integrals)
 int lloyd_max_levels(int m, int L, double *lev, double *thr);
 }  // namespace pk
