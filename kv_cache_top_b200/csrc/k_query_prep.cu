@@ -11,11 +11,10 @@
 //     better-ranked buckets (from the occupancy table), and a bucket inside
 //     the top-rho fraction (P(c) < R = ceil(rho n)) gets bonus 6 - floor(6P/R).
 //
-// Grid (16 blocks, pairs): CTA (b, pair) ranks the 256 centres of block b, one
-// thread per centre, by counting the centres that precede it (broadcast
-// shared-memory reads, no sort).  Output: the bonus table packed 4 bits per
-// centre in the layout the collision scan keeps in registers -- lane l's word
-// holds, in nibble t, the bonus of centre 32 t + l.
+// Grid (16 blocks, pairs): CTA (b, pair) ranks the 256 centres of block b with
+// a shared-memory bitonic sort, one thread per centre.  Output: the bonus
+// table packed 4 bits per centre in the layout the collision scan keeps in
+// registers -- lane l's word holds, in nibble t, the bonus of centre 32 t + l.
 #include "pk_internal.cuh"
 
 namespace pk {
@@ -27,8 +26,7 @@ __global__ void __launch_bounds__(256) k_query_prep(PrepArgs a)
     const int b_seq = bh / a.H, h = bh - b_seq * a.H;
     __shared__ float s_q[kD];
     __shared__ float s_qt[kD];
-    __shared__ float s_L[kNC];
-    __shared__ uint32_t s_occ_ranked[kNC];
+    __shared__ unsigned long long s_key[kNC];
     __shared__ uint8_t s_bonus[kNC];
     __shared__ uint32_t s_ws[9];
 
@@ -73,28 +71,33 @@ __global__ void __launch_bounds__(256) k_query_prep(PrepArgs a)
         L = __fadd_rn(L, ((c >> j) & 1) ? -x : x);
     }
     L = __fadd_rn(L, 0.0f);   // fold -0 into +0 so equal scores tie
-    s_L[c] = L;
+    // sort key, ascending = rank order: (L desc, c asc)
+    s_key[c] = ((unsigned long long)(~ord_f32(L)) << 8) | (unsigned)c;
     __syncthreads();
-    // rank = #{c' : L(c') > L(c) or (L(c') == L(c) and c' < c)}
-    int rank = 0;
-#pragma unroll 8
-    for (int c2 = 0; c2 < kNC; c2++) {
-        const float L2 = s_L[c2];
-        rank += (L2 > L || (L2 == L && c2 < c)) ? 1 : 0;
+    // bitonic sort of the 256 keys, one per thread
+    for (int k = 2; k <= kNC; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const int p = tid ^ j;
+            if (p > tid) {
+                const unsigned long long x = s_key[tid], y = s_key[p];
+                const bool up = (tid & k) == 0;
+                if (up ? (x > y) : (x < y)) {
+                    s_key[tid] = y;
+                    s_key[p] = x;
+                }
+            }
+            __syncthreads();
+        }
     }
-    const uint32_t cnt = a.occ[((size_t)bh * kB + b) * kNC + c];
-    s_occ_ranked[rank] = cnt;
-    __syncthreads();
+    // thread r now owns the centre of rank r; P = keys in better-ranked buckets
+    const int cr = (int)(s_key[tid] & 0xffu);
+    const uint32_t cnt = a.occ[((size_t)bh * kB + b) * kNC + cr];
     uint32_t tot;
-    const uint32_t excl = block_excl_scan<256>(s_occ_ranked[tid], s_ws, &tot);   // prefix in rank order
-    __syncthreads();
-    s_occ_ranked[tid] = excl;          // now: P of the bucket at rank tid
-    __syncthreads();
-    const uint32_t P = s_occ_ranked[rank];
+    const uint32_t P = block_excl_scan<256>(cnt, s_ws, &tot);
     uint32_t bon = 0;
     if ((int64_t)P < a.R) bon = 6u - (uint32_t)((6ull * P) / (unsigned long long)a.R);
-    s_bonus[c] = (uint8_t)bon;
-    if (a.dbg_bonus) a.dbg_bonus[((size_t)bh * kB + b) * kNC + c] = (uint8_t)bon;
+    s_bonus[cr] = (uint8_t)bon;
+    if (a.dbg_bonus) a.dbg_bonus[((size_t)bh * kB + b) * kNC + cr] = (uint8_t)bon;
     __syncthreads();
     if (tid < 32) {
         uint32_t word = 0;

@@ -161,7 +161,7 @@ __device__ __forceinline__ float block_dot(const float *slev, uint32_t nib, cons
     return d;
 }
 
-__global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
+__global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
 {
     extern __shared__ __align__(16) unsigned char s_dyn[];
     __shared__ RrShared sm;
@@ -186,14 +186,32 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
     __syncthreads();
 
     const bool odd = (q8 & 1) != 0;
-    for (int r0 = warp * 16; r0 < count; r0 += kRrWarps * 16) {
+    // software pipeline: the next 16 records of the warp are in flight while
+    // the current 16 are decoded
+    const int step = kRrWarps * 16;
+    uint4 vn[4];
+    int32_t idn[4];
+#pragma unroll
+    for (int u = 0; u < 4; u++) {
+        const int r = warp * 16 + 4 * u + sub;
+        idn[u] = ids[r < count ? r : 0];
+        vn[u] = __ldg(reinterpret_cast<const uint4 *>(rec + (size_t)idn[u] * kRecBytes) + q8);
+    }
+    for (int r0 = warp * 16; r0 < count; r0 += step) {
         uint4 v[4];
         int32_t id[4];
 #pragma unroll
         for (int u = 0; u < 4; u++) {
-            const int r = r0 + 4 * u + sub;
-            id[u] = ids[r < count ? r : 0];
-            v[u] = __ldg(reinterpret_cast<const uint4 *>(rec + (size_t)id[u] * kRecBytes) + q8);
+            v[u] = vn[u];
+            id[u] = idn[u];
+        }
+        if (r0 + step < count) {
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int r = r0 + step + 4 * u + sub;
+                idn[u] = ids[r < count ? r : 0];
+                vn[u] = __ldg(reinterpret_cast<const uint4 *>(rec + (size_t)idn[u] * kRecBytes) + q8);
+            }
         }
 #pragma unroll
         for (int u = 0; u < 4; u++) {

@@ -45,9 +45,7 @@ struct pk_index {
     int32_t *cand = nullptr;
     unsigned long long *partial = nullptr;
     int32_t max_slices = 1;
-    float *att_part = nullptr;
-    uint32_t *att_tickets = nullptr;
-    int32_t max_splits = 1;
+
     int32_t *dev_err = nullptr;
     long long *dev_err_detail = nullptr;
     // tracing
@@ -60,6 +58,7 @@ struct pk_index {
 namespace {
 
 constexpr int64_t kMinChunk = 1024;
+constexpr int64_t kMaxChunk = 32768;   // keys per chunk: the compaction kernel holds a chunk in registers
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -122,6 +121,7 @@ void chunking(const pk_index *ix, int64_t n, int32_t *nchunks, int64_t *chunk)
 {
     int64_t nch = ceil_div(4 * (int64_t)ix->num_sms, ix->bh);
     nch = std::max<int64_t>(1, std::min<int64_t>(nch, ceil_div(n, kMinChunk)));
+    nch = std::max<int64_t>(nch, ceil_div(n, kMaxChunk));
     nch = std::min<int64_t>(nch, ix->max_chunks);
     int64_t ch = ceil_div(ceil_div(n, nch), 16) * 16;
     *chunk = ch;
@@ -133,7 +133,7 @@ int32_t slice_lo(const pk_index *ix) { return std::max<int32_t>(256, 2 * ix->top
 
 void slicing(const pk_index *ix, int64_t C, int32_t *slice, int32_t *nslices)
 {
-    const int64_t target = 3 * (int64_t)ix->num_sms;
+    const int64_t target = 2 * (int64_t)ix->num_sms;
     int64_t sl = ceil_div(ceil_div(C * ix->bh, target), 64) * 64;
     sl = std::max<int64_t>(sl, slice_lo(ix));
     sl = std::min<int64_t>(sl, kMaxSlice);
@@ -141,13 +141,13 @@ void slicing(const pk_index *ix, int64_t C, int32_t *slice, int32_t *nslices)
     *nslices = (int32_t)ceil_div(C, sl);
 }
 
-// attention work split: up to kAtRows selected rows per CTA
-void splitting(const pk_index *ix, int32_t topk, int32_t *rows_per, int32_t *nsplit)
+// attention work split: one cluster of up to 8 CTAs per pair, ~2 CTAs per SM
+int32_t splitting(const pk_index *ix, int32_t topk)
 {
-    int64_t rp = ceil_div((int64_t)topk * ix->bh, 2 * (int64_t)ix->num_sms);
-    rp = std::max<int64_t>(8, std::min<int64_t>(rp, kAtRows));
-    *nsplit = (int32_t)ceil_div(topk, rp);
-    *rows_per = (int32_t)ceil_div(topk, *nsplit);
+    int64_t ns = ceil_div(2 * (int64_t)ix->num_sms, ix->bh);
+    ns = std::max<int64_t>(1, std::min<int64_t>(ns, 8));
+    ns = std::min<int64_t>(ns, topk);
+    return (int32_t)ns;
 }
 
 void free_all(pk_index *ix)
@@ -174,8 +174,7 @@ void free_all(pk_index *ix)
     cudaFree(ix->sstar);
     cudaFree(ix->cand);
     cudaFree(ix->partial);
-    cudaFree(ix->att_part);
-    cudaFree(ix->att_tickets);
+
     cudaFree(ix->dev_err);
     cudaFree(ix->dev_err_detail);
     for (cudaEvent_t e : ix->ev_pool) cudaEventDestroy(e);
@@ -314,6 +313,11 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     sa.chunk_info = ix->chunk_info;
     sa.sstar = ix->sstar;
     sa.max_chunks = ix->max_chunks;
+    sa.one = 1u;
+    sa.m8 = 1u << 8;
+    sa.m16 = 1u << 16;
+    sa.m24 = 1u << 24;
+    sa.m29 = 1u << 29;
     if (dbg) {
         sa.dbg_S = dbg->S;
         sa.dbg_hist = dbg->hist;
@@ -333,6 +337,7 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     ca.chunk = chunk;
     ca.C = C;
     ca.max_chunks = ix->max_chunks;
+    ca.groups = (int32_t)ceil_div(chunk, 16 * 256);
     ca.cand = ix->cand;
     ca.dbg_cand = dbg ? dbg->cand : nullptr;
     ca.dev_err = ix->dev_err;
@@ -454,7 +459,8 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
         delete ix;
         return cuda_status(e);
     }
-    ix->max_chunks = (int32_t)std::max<int64_t>(1, ceil_div(4 * (int64_t)ix->num_sms, ix->bh));
+    ix->max_chunks = (int32_t)std::max<int64_t>(ceil_div(4 * (int64_t)ix->num_sms, ix->bh),
+                                                ceil_div(n_cap, kMaxChunk) + 1);
 
     // SRHT sign diagonal and scale; Lloyd-Max levels
     for (int r = 0; r < 4; r++) ix->rot.sign_mask[r] = 0;
@@ -489,16 +495,14 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(dalloc(&ix->sstar, BH));
     {   // largest slice count any C <= n_cap can need
         const int64_t lo = slice_lo(ix);
-        const int64_t by_target = ceil_div(3 * (int64_t)ix->num_sms, ix->bh) + 1;
+        const int64_t by_target = ceil_div(2 * (int64_t)ix->num_sms, ix->bh) + 1;
         ix->max_slices = (int32_t)std::max<int64_t>(std::min<int64_t>(ceil_div(n_cap, lo), by_target),
                                                     ceil_div(n_cap, kMaxSlice)) + 1;
-        ix->max_splits = (int32_t)ceil_div(ix->topk_cap, 8);
     }
     const size_t MS = ix->max_slices;
     chk(dalloc(&ix->cand, BH * NC));
     chk(dalloc(&ix->partial, BH * MS * (size_t)ix->topk_cap));
-    chk(dalloc(&ix->att_part, BH * (size_t)ix->max_splits * kMaxGroup * (kD + 2)));
-    chk(dalloc(&ix->att_tickets, BH));
+
     chk(dalloc(&ix->dev_err, 1));
     chk(dalloc(&ix->dev_err_detail, 1));
     const size_t kv_bytes = BH * NC * kD * (size_t)es;
@@ -519,7 +523,6 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(cudaMemsetAsync(ix->occ, 0, BH * kB * kNC * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->head_hist, 0, BH * kBins * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->tickets, 0, BH * 2 * sizeof(uint32_t), s));
-    chk(cudaMemsetAsync(ix->att_tickets, 0, BH * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->dev_err, 0, sizeof(int32_t), s));
     chk(cudaMemsetAsync(ix->dev_err_detail, 0, sizeof(long long), s));
     if (e == cudaSuccess) st = copy_rows(ix, ix->K, K, n, 0, s);
@@ -583,10 +586,7 @@ pk_status pk_attend(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t
     a.topk = topk;
     a.is_bf16 = ix->p.kv_dtype == PK_BF16;
     a.scale = ix->scale;
-    splitting(ix, topk, &a.rows_per, &a.nsplit);
-    a.max_splits = ix->max_splits;
-    a.part = ix->att_part;
-    a.tickets = ix->att_tickets;
+    a.nsplit = splitting(ix, topk);
     a.dev_err = ix->dev_err;
     a.dev_err_detail = ix->dev_err_detail;
     cudaStream_t s = (cudaStream_t)stream;

@@ -80,6 +80,9 @@ struct ScanArgs {
     uint2 *chunk_info;       // [BH][max_chunks]  (first candidate slot, tie quota)
     int32_t *sstar;          // [BH]
     int32_t max_chunks;
+    // 1, 2^8, 2^16, 2^24, 2^29 passed at run time, so the compiler keeps the
+    // integer multiplies (fma pipe) that stand in for shifts and adds
+    uint32_t one, m8, m16, m24, m29;
     uint8_t *dbg_S;
     uint32_t *dbg_hist;
     int32_t *dbg_sstar;
@@ -91,6 +94,7 @@ struct CompactArgs {
     const int32_t *sstar;
     int64_t n, stride, chunk, C;
     int32_t max_chunks;
+    int32_t groups;          // 16-key groups per thread: ceil(chunk / 4096) <= 8
     int32_t *cand;           // [BH][stride]  candidate ids, ascending
     int32_t *dbg_cand;       // [BH][C] or null
     int32_t *dev_err;
@@ -120,9 +124,7 @@ struct AttendArgs {
     float *out;              // [batch][H*G][D]
     int64_t n, stride;
     int32_t H, G, topk, is_bf16;
-    int32_t rows_per, nsplit, max_splits;
-    float *part;             // [BH][max_splits][kMaxGroup][D + 2]
-    uint32_t *tickets;       // [BH]
+    int32_t nsplit;          // CTAs (one cluster) per pair, 1..8
     float scale;
     int32_t *dev_err;
     long long *dev_err_detail;
