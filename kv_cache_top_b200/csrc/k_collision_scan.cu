@@ -20,10 +20,7 @@
 // 4 (c >> 5) -- all four computed at once per 32-bit code word -- is the
 // shift of a wrap-mode funnel shift (which ignores bits above 4).  Two
 // extracted bonuses (each <= 6) are added before one mask, since their sum
-// still fits in the low nibble.  The kernel is bound by integer issue, so the
-// byte shifts (x >> 8k = high word of x * 2^(32-8k)) and the pair additions
-// run as integer multiply-adds on the fma pipe, next to the logic and funnel
-// shifts on the alu pipe.
+// still fits in the low nibble.
 #include "pk_internal.cuh"
 
 namespace pk {
@@ -32,29 +29,23 @@ constexpr int kScanThreads = 256;
 constexpr int kScanUnroll = 4;
 constexpr int kHistPad = 104;
 
-struct Muls {
-    uint32_t one, m8, m16, m24, m29;
-};
-
-__device__ __forceinline__ uint32_t mad(uint32_t a, uint32_t b, uint32_t c) { return a * b + c; }
-
-__device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], uint4 c, const Muls &mu)
+__device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], uint4 c)
 {
     uint32_t s = 0;
     const uint32_t wds[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int q = 0; q < 4; q++) {
         const uint32_t w = wds[q];
-        const uint32_t A = __umulhi(w, mu.m29) & 0x1c1c1c1cu;      // byte k: 4 * (c_k >> 5)
+        const uint32_t A = (w >> 3) & 0x1c1c1c1cu;      // byte k: 4 * (c_k >> 5)
         const uint32_t v0 = __shfl_sync(kFull, tab[4 * q + 0], (int)w);
-        const uint32_t v1 = __shfl_sync(kFull, tab[4 * q + 1], (int)__umulhi(w, mu.m24));
-        const uint32_t v2 = __shfl_sync(kFull, tab[4 * q + 2], (int)__umulhi(w, mu.m16));
-        const uint32_t v3 = __shfl_sync(kFull, tab[4 * q + 3], (int)__umulhi(w, mu.m8));
+        const uint32_t v1 = __shfl_sync(kFull, tab[4 * q + 1], (int)(w >> 8));
+        const uint32_t v2 = __shfl_sync(kFull, tab[4 * q + 2], (int)(w >> 16));
+        const uint32_t v3 = __shfl_sync(kFull, tab[4 * q + 3], (int)(w >> 24));
         const uint32_t x0 = __funnelshift_r(v0, 0u, A);
-        const uint32_t x1 = __funnelshift_r(v1, 0u, __umulhi(A, mu.m24));
-        const uint32_t x2 = __funnelshift_r(v2, 0u, __umulhi(A, mu.m16));
-        const uint32_t x3 = __funnelshift_r(v3, 0u, __umulhi(A, mu.m8));
-        s = mad(mad(x0, mu.one, x1) & 0xfu, mu.one, s) + (mad(x2, mu.one, x3) & 0xfu);
+        const uint32_t x1 = __funnelshift_r(v1, 0u, A >> 8);
+        const uint32_t x2 = __funnelshift_r(v2, 0u, A >> 16);
+        const uint32_t x3 = __funnelshift_r(v3, 0u, A >> 24);
+        s += ((x0 + x1) & 0xfu) + ((x2 + x3) & 0xfu);
     }
     return s;
 }
@@ -71,7 +62,6 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
 
     for (int i = tid; i < NW * kHistPad; i += kScanThreads) (&s_hist[0][0])[i] = 0u;
 
-    const Muls mu{a.one, a.m8, a.m16, a.m24, a.m29};
     uint32_t tab[kB];
     const uint32_t *bp = a.bonus_packed + (size_t)bh * kB * 32;
 #pragma unroll
@@ -98,7 +88,7 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
 #pragma unroll
         for (int u = 0; u < kScanUnroll; u++) {
             const int64_t i = base + u * 32 + lane;
-            const uint32_t s = collision_score(tab, c[u], mu);
+            const uint32_t s = collision_score(tab, c[u]);
             if (i < cnt) {
                 S[i] = (uint8_t)s;
                 if (dS) dS[i] = (uint8_t)s;

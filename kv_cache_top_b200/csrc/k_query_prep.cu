@@ -11,108 +11,135 @@
 //     better-ranked buckets (from the occupancy table), and a bucket inside
 //     the top-rho fraction (P(c) < R = ceil(rho n)) gets bonus 6 - floor(6P/R).
 //
-// Grid (16 blocks, pairs): CTA (b, pair) ranks the 256 centres of block b with
-// a shared-memory bitonic sort, one thread per centre.  Output: the bonus
-// table packed 4 bits per centre in the layout the collision scan keeps in
-// registers -- lane l's word holds, in nibble t, the bonus of centre 32 t + l.
+// Grid (16 blocks, pairs), one warp per CTA: the warp rotates the query, ranks
+// the 256 centres of its block with a register bitonic sort (8 keys per lane,
+// shuffles only, no block barriers), scans the bucket sizes in rank order and
+// packs the bonus table 4 bits per centre in the layout the collision scan
+// keeps in registers -- lane l's word holds, in nibble t, the bonus of centre
+// 32 t + l.
 #include "pk_internal.cuh"
 
 namespace pk {
 
-__global__ void __launch_bounds__(256) k_query_prep(PrepArgs a)
+__global__ void __launch_bounds__(32) k_query_prep(PrepArgs a)
 {
     const int b = blockIdx.x, bh = blockIdx.y;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lane = threadIdx.x;
     const int b_seq = bh / a.H, h = bh - b_seq * a.H;
-    __shared__ float s_q[kD];
-    __shared__ float s_qt[kD];
-    __shared__ unsigned long long s_key[kNC];
     __shared__ uint8_t s_bonus[kNC];
-    __shared__ uint32_t s_ws[9];
 
     if (b == 0) {   // reset the per-call counters of the collision scan and the rerank
-        if (tid < kBins) a.head_hist[(size_t)bh * kBins + tid] = 0u;
-        if (tid < 2) a.tickets[(size_t)bh * 2 + tid] = 0u;
+        for (int i = lane; i < kBins; i += 32) a.head_hist[(size_t)bh * kBins + i] = 0u;
+        if (lane < 2) a.tickets[(size_t)bh * 2 + lane] = 0u;
     }
-    if (tid < kD) {
-        const int64_t base = ((int64_t)b_seq * a.H * a.G + (int64_t)h * a.G) * kD + tid;
-        float acc = ld_as_f32(a.q, base, a.is_bf16);
-        for (int g = 1; g < a.G; g++) acc = __fadd_rn(acc, ld_as_f32(a.q, base + (int64_t)g * kD, a.is_bf16));
-        s_q[tid] = acc;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        float x[4];
+    float x[4];
+    {
+        const int64_t base = ((int64_t)b_seq * a.H * a.G + (int64_t)h * a.G) * kD;
 #pragma unroll
-        for (int r = 0; r < 4; r++) x[r] = s_q[lane + 32 * r];
-        const float nrm = warp_rotate128(x, a.rot, lane);
-#pragma unroll
-        for (int r = 0; r < 4; r++) s_qt[lane + 32 * r] = x[r];
-        if (b == 0) {
-#pragma unroll
-            for (int r = 0; r < 4; r++) {
-                a.qt[(size_t)bh * kD + lane + 32 * r] = x[r];
-                if (a.dbg_qt) a.dbg_qt[(size_t)bh * kD + lane + 32 * r] = x[r];
-            }
-            if (lane == 0) {
-                a.qnorm[bh] = nrm;
-                if (a.dbg_qnorm) a.dbg_qnorm[bh] = nrm;
-            }
+        for (int r = 0; r < 4; r++) {
+            const int64_t j = base + lane + 32 * r;
+            float acc = ld_as_f32(a.q, j, a.is_bf16);
+            for (int g = 1; g < a.G; g++) acc = __fadd_rn(acc, ld_as_f32(a.q, j + (int64_t)g * kD, a.is_bf16));
+            x[r] = acc;
         }
     }
-    __syncthreads();
-
-    // centre c = tid: score L_b(c), summed over j = 0..7 in order
-    const int c = tid;
-    float L = 0.0f;
+    const float nrm = warp_rotate128(x, a.rot, lane);
+    if (b == 0) {
 #pragma unroll
-    for (int j = 0; j < kM; j++) {
-        const float x = s_qt[b * kM + j];
-        L = __fadd_rn(L, ((c >> j) & 1) ? -x : x);
+        for (int r = 0; r < 4; r++) {
+            a.qt[(size_t)bh * kD + lane + 32 * r] = x[r];
+            if (a.dbg_qt) a.dbg_qt[(size_t)bh * kD + lane + 32 * r] = x[r];
+        }
+        if (lane == 0) {
+            a.qnorm[bh] = nrm;
+            if (a.dbg_qnorm) a.dbg_qnorm[bh] = nrm;
+        }
     }
-    L = __fadd_rn(L, 0.0f);   // fold -0 into +0 so equal scores tie
-    // sort key, ascending = rank order: (L desc, c asc)
-    s_key[c] = ((unsigned long long)(~ord_f32(L)) << 8) | (unsigned)c;
-    __syncthreads();
-    // bitonic sort of the 256 keys, one per thread
-    for (int k = 2; k <= kNC; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            const int p = tid ^ j;
-            if (p > tid) {
-                const unsigned long long x = s_key[tid], y = s_key[p];
-                const bool up = (tid & k) == 0;
-                if (up ? (x > y) : (x < y)) {
-                    s_key[tid] = y;
-                    s_key[p] = x;
+    // coordinates 8b..8b+7 live in register b/4 of lanes 8(b%4)..8(b%4)+7
+    float xq[kM];
+    {
+        float src = x[0];
+#pragma unroll
+        for (int r = 1; r < 4; r++) src = (b / 4 == r) ? x[r] : src;
+#pragma unroll
+        for (int j = 0; j < kM; j++) xq[j] = __shfl_sync(kFull, src, 8 * (b % 4) + j);
+    }
+    // element e = 8 lane + i starts as centre c = e; sort key (ascending order =
+    // rank order): high 32 bits = ~ord(L) (L desc), low 8 bits = c (c asc)
+    unsigned long long key[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const int c = lane * 8 + i;
+        float L = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kM; j++) L = __fadd_rn(L, ((c >> j) & 1) ? -xq[j] : xq[j]);
+        L = __fadd_rn(L, 0.0f);   // fold -0 into +0 so equal scores tie
+        key[i] = ((unsigned long long)(~ord_f32(L)) << 8) | (unsigned)c;
+    }
+    // bitonic sort, ascending, 256 elements over the warp
+#pragma unroll
+    for (int k = 2; k <= 256; k <<= 1) {
+#pragma unroll
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+            if (jj >= 8) {
+                const int lx = jj >> 3;
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int e = lane * 8 + i;
+                    const unsigned long long o = __shfl_xor_sync(kFull, key[i], lx);
+                    const bool take_min = ((e & jj) == 0) == ((e & k) == 0);
+                    key[i] = take_min ? (o < key[i] ? o : key[i]) : (o > key[i] ? o : key[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    if ((i & jj) == 0) {
+                        const int e = lane * 8 + i;
+                        const bool up = (e & k) == 0;
+                        const unsigned long long x0 = key[i], x1 = key[i ^ jj];
+                        const unsigned long long lo = x0 < x1 ? x0 : x1, hi = x0 < x1 ? x1 : x0;
+                        key[i] = up ? lo : hi;
+                        key[i ^ jj] = up ? hi : lo;
+                    }
                 }
             }
-            __syncthreads();
         }
     }
-    // thread r now owns the centre of rank r; P = keys in better-ranked buckets
-    const int cr = (int)(s_key[tid] & 0xffu);
-    const uint32_t cnt = a.occ[((size_t)bh * kB + b) * kNC + cr];
-    uint32_t tot;
-    const uint32_t P = block_excl_scan<256>(cnt, s_ws, &tot);
-    uint32_t bon = 0;
-    if ((int64_t)P < a.R) bon = 6u - (uint32_t)((6ull * P) / (unsigned long long)a.R);
-    s_bonus[cr] = (uint8_t)bon;
-    if (a.dbg_bonus) a.dbg_bonus[((size_t)bh * kB + b) * kNC + cr] = (uint8_t)bon;
-    __syncthreads();
-    if (tid < 32) {
-        uint32_t word = 0;
+    // exclusive prefix of bucket sizes in rank order -> tier bonus
+    const uint32_t *occ = a.occ + ((size_t)bh * kB + b) * kNC;
+    uint32_t cnt[8], run = 0;
 #pragma unroll
-        for (int t = 0; t < 8; t++) word |= (uint32_t)s_bonus[32 * t + tid] << (4 * t);
-        a.bonus_packed[((size_t)bh * kB + b) * 32 + tid] = word;
+    for (int i = 0; i < 8; i++) {
+        cnt[i] = occ[key[i] & 0xffu];
+        run += cnt[i];
     }
+    uint32_t incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+    }
+    uint32_t P = incl - run;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const int c = (int)(key[i] & 0xffu);
+        uint32_t bon = 0;
+        if ((int64_t)P < a.R) bon = 6u - (uint32_t)((6ull * P) / (unsigned long long)a.R);
+        s_bonus[c] = (uint8_t)bon;
+        if (a.dbg_bonus) a.dbg_bonus[((size_t)bh * kB + b) * kNC + c] = (uint8_t)bon;
+        P += cnt[i];
+    }
+    __syncwarp();
+    uint32_t word = 0;
+#pragma unroll
+    for (int t = 0; t < 8; t++) word |= (uint32_t)s_bonus[32 * t + lane] << (4 * t);
+    a.bonus_packed[((size_t)bh * kB + b) * 32 + lane] = word;
 }
 
-}  // namespace pk
-
-namespace pk {
 cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s)
 {
-    k_query_prep<<<dim3(kB, a.bh), 256, 0, s>>>(a);
+    k_query_prep<<<dim3(kB, a.bh), 32, 0, s>>>(a);
     return cudaGetLastError();
 }
+
 }  // namespace pk

@@ -8,19 +8,19 @@
 //
 // Work is split by candidate slices (not key ranges), so every CTA reranks
 // the same number of records wherever the candidates sit.  A CTA stages its
-// candidate ids in shared memory, then each warp keeps 16 record loads in
-// flight (8 lanes x 16 B per record, fully coalesced); after one
-// pair-exchange each lane owns two blocks (16 coordinates) with their
-// weights.  The signed level of a nibble comes from a 16-entry shared table
-// (at most 16 distinct words per request: no bank conflicts), q~ stays in
-// registers.
+// candidate ids in shared memory; four lanes share a record, each loading one
+// 32-byte group (the nibbles of 4 blocks and their 4 weights) with two 16-byte
+// loads, so a warp moves 8 whole records per load pair and every lane decodes
+// 32 coordinates with no exchange.  The signed level of a nibble comes from a
+// 16-entry shared table (at most 16 distinct words per request: no bank
+// conflicts); q~ stays in registers.
 //
 // Scores never leave the chip: the CTA turns (score, id) into 64-bit keys
-// ordered by score desc then id asc, radix-selects its Top-k, sorts it and
-// writes it; the last CTA of the pair (ticket counter, no spin-wait) merges the
-// per-slice lists into the final sorted Top-k (README: "reranks those
-// candidates with a fused 4-bit approximate inner-product kernel and selects
-// the final Top-k KV indices").
+// ordered by score desc then id asc and radix-selects its Top-k set; the last
+// CTA of the pair (ticket counter, no spin-wait) merges the per-slice sets and
+// sorts the final Top-k with one warp (README: "reranks those candidates with
+// a fused 4-bit approximate inner-product kernel and selects the final Top-k
+// KV indices").  Block barriers are few: each radix pass costs two.
 #include "pk_internal.cuh"
 
 namespace pk {
@@ -32,36 +32,74 @@ typedef unsigned long long u64;
 
 struct RrShared {
     u64 tmp[kMaxTopk];
-    uint32_t hist[256];
-    uint32_t ws[kRrWarps + 1];
-    u64 red[kRrWarps];
+    uint32_t hist[2][256];
+    u64 red[2][kRrWarps];
     uint32_t sh[4];
     uint32_t cnt;
-    u64 tau;
     float slev[16];
     int last;
 };
 
-// Keep the k largest of keys[0..count) (count > k) in keys[0..k), any order;
-// return the smallest kept key.  All threads of the block must call it.
-__device__ u64 block_topk_shrink(RrShared &sm, u64 *keys, int count, int k)
+// Keep the k largest of keys[0..count) (count > k; keys distinct) in
+// sm.tmp[0..k), any order; returns the smallest kept key.  Radix select, most
+// significant digit first, starting at the highest bit where the keys differ
+// (scores of one query share sign and exponent, so leading digits would put
+// every key in one bin); histogram increments are aggregated per warp over
+// lanes that hit the same bin.  All threads of the block must call it.
+__device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    u64 prefix = 0, mask = 0;
+    u64 lo = ~0ull, hi = 0ull;
+    for (int i = tid; i < count; i += kRrThreads) {
+        const u64 x = keys[i];
+        lo = x < lo ? x : lo;
+        hi = x > hi ? x : hi;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const u64 a = __shfl_xor_sync(kFull, lo, o), b = __shfl_xor_sync(kFull, hi, o);
+        lo = a < lo ? a : lo;
+        hi = b > hi ? b : hi;
+    }
+    if (lane == 0) {
+        sm.red[0][warp] = lo;
+        sm.red[1][warp] = hi;
+    }
+    for (int i = tid; i < 2 * 256; i += kRrThreads) (&sm.hist[0][0])[i] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kRrWarps; w++) {
+        lo = sm.red[0][w] < lo ? sm.red[0][w] : lo;
+        hi = sm.red[1][w] > hi ? sm.red[1][w] : hi;
+    }
+    const int hb = 63 - __clzll((long long)(lo ^ hi));      // highest differing bit
+    u64 mask = (hb >= 63) ? 0ull : ~((2ull << hb) - 1ull);   // bits above hb: common to all keys
+    u64 prefix = hi & mask;
     int need = k;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += kRrThreads) sm.hist[i] = 0u;
-        __syncthreads();
-        for (int i = tid; i < count; i += kRrThreads) {
-            const u64 x = keys[i];
-            if ((x & mask) == prefix) atomicAdd(&sm.hist[(x >> shift) & 0xffu], 1u);
+    int pass = 0;
+    for (int top = hb; top >= 0; top -= 8, pass ^= 1) {
+        const int width = top + 1 < 8 ? top + 1 : 8;
+        const int shift = top + 1 - width;
+        const uint32_t dmask = (1u << width) - 1u;
+        uint32_t *H = sm.hist[pass];
+        for (int base = 0; base < count; base += kRrThreads) {
+            const int i = base + tid;
+            bool act = false;
+            uint32_t bin = 0xffffffffu;
+            if (i < count) {
+                const u64 x = keys[i];
+                act = (x & mask) == prefix;
+                if (act) bin = (uint32_t)(x >> shift) & dmask;
+            }
+            const uint32_t grp = __match_any_sync(kFull, bin);
+            if (act && lane == __ffs(grp) - 1) atomicAdd(&H[bin], (uint32_t)__popc(grp));
         }
         __syncthreads();
         if (warp == 0) {
             uint32_t hc[8], sum = 0;
 #pragma unroll
             for (int i = 0; i < 8; i++) {
-                hc[i] = sm.hist[255 - 8 * lane - i];
+                hc[i] = H[255 - 8 * lane - i];
                 sum += hc[i];
             }
             uint32_t incl = sum;
@@ -79,70 +117,58 @@ __device__ u64 block_topk_shrink(RrShared &sm, u64 *keys, int count, int k)
                     sm.sh[2] = hc[i];
                 }
                 run += hc[i];
+                H[255 - 8 * lane - i] = 0u;     // ready for the pass after next
             }
         }
         __syncthreads();
         const uint32_t d = sm.sh[0], above = sm.sh[1], inbin = sm.sh[2];
         need -= (int)above;
         prefix |= (u64)d << shift;
-        mask |= (u64)0xffu << shift;
-        __syncthreads();
+        mask |= (u64)dmask << shift;
         if ((int)inbin == need) break;
     }
+    // everything at or above the selected prefix: exactly k keys
     if (tid == 0) sm.sh[3] = 0;
     __syncthreads();
+    u64 mn = ~0ull;
     for (int i = tid; i < count; i += kRrThreads) {
         const u64 x = keys[i];
         if ((x & mask) >= prefix) {
             const uint32_t pos = atomicAdd(&sm.sh[3], 1u);
-            if (pos < (uint32_t)kMaxTopk) sm.tmp[pos] = x;   // exactly k reach here
+            if (pos < (uint32_t)kMaxTopk) sm.tmp[pos] = x;
+            mn = x < mn ? x : mn;
         }
-    }
-    __syncthreads();
-    u64 mn = ~0ull;
-    for (int i = tid; i < k; i += kRrThreads) {
-        const u64 x = sm.tmp[i];
-        keys[i] = x;
-        mn = x < mn ? x : mn;
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
         const u64 y = __shfl_xor_sync(kFull, mn, o);
         mn = y < mn ? y : mn;
     }
-    if (lane == 0) sm.red[warp] = mn;
+    if (lane == 0) sm.red[0][warp] = mn;
     __syncthreads();
-    if (tid == 0) {
-        u64 m = sm.red[0];
-        for (int w = 1; w < kRrWarps; w++) m = sm.red[w] < m ? sm.red[w] : m;
-        sm.tau = m;
-    }
-    __syncthreads();
-    return sm.tau;
+#pragma unroll
+    for (int w = 0; w < kRrWarps; w++) mn = sm.red[0][w] < mn ? sm.red[0][w] : mn;
+    return mn;
 }
 
-// Sort keys[0..k) descending into sm.tmp[0..p2) (zero-padded).
-__device__ void block_sort_desc(RrShared &sm, const u64 *keys, int k)
+// One warp sorts sm.tmp[0..p2) descending in place (p2 a power of two <= 1024).
+__device__ void warp_sort_desc(u64 *v, int p2)
 {
-    const int tid = threadIdx.x;
-    int p2 = 1;
-    while (p2 < k) p2 <<= 1;
-    for (int i = tid; i < p2; i += kRrThreads) sm.tmp[i] = (i < k) ? keys[i] : 0ull;
-    __syncthreads();
+    const int lane = threadIdx.x & 31;
     for (int kk = 2; kk <= p2; kk <<= 1) {
         for (int j = kk >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < p2; i += kRrThreads) {
+            for (int i = lane; i < p2; i += 32) {
                 const int ixj = i ^ j;
                 if (ixj > i) {
-                    const u64 x = sm.tmp[i], y = sm.tmp[ixj];
+                    const u64 x = v[i], y = v[ixj];
                     const bool desc = (i & kk) == 0;
                     if (desc ? (x < y) : (x > y)) {
-                        sm.tmp[i] = y;
-                        sm.tmp[ixj] = x;
+                        v[i] = y;
+                        v[ixj] = x;
                     }
                 }
             }
-            __syncthreads();
+            __syncwarp();
         }
     }
 }
@@ -161,7 +187,7 @@ __device__ __forceinline__ float block_dot(const float *slev, uint32_t nib, cons
     return d;
 }
 
-__global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
+__global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
 {
     extern __shared__ __align__(16) unsigned char s_dyn[];
     __shared__ RrShared sm;
@@ -176,60 +202,37 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
     if (tid < 16) sm.slev[tid] = (tid & 8) ? -a.lv.lev[tid & 7] : a.lv.lev[tid & 7];
     const int32_t *cand = a.cand + (size_t)bh * a.stride + m0;
     for (int i = tid; i < count; i += kRrThreads) ids[i] = cand[i];
-    const int q8 = lane & 7, sub = lane >> 3;
-    float qr[16];
+    const int q4 = lane & 3, sub = lane >> 2;          // group of the record, record of the warp step
+    float qr[32];
 #pragma unroll
-    for (int i = 0; i < 16; i++) qr[i] = a.qt[(size_t)bh * kD + 16 * q8 + i];
+    for (int i = 0; i < 32; i++) qr[i] = a.qt[(size_t)bh * kD + 32 * q4 + i];
     const float qnorm = a.qnorm[bh];
-    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes;
+    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes + 32 * q4;
     float *dest = a.dbg_est ? a.dbg_est + (size_t)bh * a.C + m0 : nullptr;
     __syncthreads();
 
-    const bool odd = (q8 & 1) != 0;
-    // software pipeline: the next 16 records of the warp are in flight while
-    // the current 16 are decoded
-    const int step = kRrWarps * 16;
-    uint4 vn[4];
-    int32_t idn[4];
+    // each warp step: 16 records, two 16-byte loads per lane per record group
+    for (int r0 = warp * 16; r0 < count; r0 += kRrWarps * 16) {
+        uint4 nv[2], wv[2];
+        int32_t id[2];
 #pragma unroll
-    for (int u = 0; u < 4; u++) {
-        const int r = warp * 16 + 4 * u + sub;
-        idn[u] = ids[r < count ? r : 0];
-        vn[u] = __ldg(reinterpret_cast<const uint4 *>(rec + (size_t)idn[u] * kRecBytes) + q8);
-    }
-    for (int r0 = warp * 16; r0 < count; r0 += step) {
-        uint4 v[4];
-        int32_t id[4];
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            v[u] = vn[u];
-            id[u] = idn[u];
-        }
-        if (r0 + step < count) {
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int r = r0 + step + 4 * u + sub;
-                idn[u] = ids[r < count ? r : 0];
-                vn[u] = __ldg(reinterpret_cast<const uint4 *>(rec + (size_t)idn[u] * kRecBytes) + q8);
-            }
+        for (int u = 0; u < 2; u++) {
+            const int r = r0 + 8 * u + sub;
+            id[u] = ids[r < count ? r : 0];
+            const uint4 *p = reinterpret_cast<const uint4 *>(rec + (size_t)id[u] * kRecBytes);
+            nv[u] = __ldg(p);
+            wv[u] = __ldg(p + 1);
         }
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            // even lane of a pair: nibble words of blocks 4g..4g+3; odd lane: their
-            // weights.  Swap halves so lane q8 owns blocks 2 q8, 2 q8 + 1.
-            const uint32_t r0v = __shfl_xor_sync(kFull, odd ? v[u].x : v[u].z, 1);
-            const uint32_t r1v = __shfl_xor_sync(kFull, odd ? v[u].y : v[u].w, 1);
-            const uint32_t nib0 = odd ? r0v : v[u].x, nib1 = odd ? r1v : v[u].y;
-            const float w0 = __uint_as_float(odd ? v[u].z : r0v);
-            const float w1 = __uint_as_float(odd ? v[u].w : r1v);
-            const float d0 = block_dot(sm.slev, nib0, qr);
-            const float d1 = block_dot(sm.slev, nib1, qr + 8);
-            float part = fmaf(w0, d0, w1 * d1);
+        for (int u = 0; u < 2; u++) {
+            float part = __uint_as_float(wv[u].x) * block_dot(sm.slev, nv[u].x, qr);
+            part = fmaf(__uint_as_float(wv[u].y), block_dot(sm.slev, nv[u].y, qr + 8), part);
+            part = fmaf(__uint_as_float(wv[u].z), block_dot(sm.slev, nv[u].z, qr + 16), part);
+            part = fmaf(__uint_as_float(wv[u].w), block_dot(sm.slev, nv[u].w, qr + 24), part);
             part += __shfl_xor_sync(kFull, part, 1);
             part += __shfl_xor_sync(kFull, part, 2);
-            part += __shfl_xor_sync(kFull, part, 4);
-            const int r = r0 + 4 * u + sub;
-            if (q8 == 0 && r < count) {
+            const int r = r0 + 8 * u + sub;
+            if (q4 == 0 && r < count) {
                 const float est = qnorm * part;
                 keys[r] = make_key(est, id[u]);
                 if (dest) dest[r] = est;
@@ -238,10 +241,14 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
     }
     __syncthreads();
 
-    // ---- Top-k of the slice
+    // ---- Top-k set of the slice (unordered)
     const int have = min(count, k);
-    if (count > k) block_topk_shrink(sm, keys, count, k);
-    block_sort_desc(sm, keys, have);
+    if (count > k) {
+        block_topk_select(sm, keys, count, k);
+    } else {
+        for (int i = tid; i < count; i += kRrThreads) sm.tmp[i] = keys[i];
+        __syncthreads();
+    }
     u64 *part = a.partial + ((size_t)bh * a.max_slices + sl) * a.topk_cap;
     for (int i = tid; i < k; i += kRrThreads) part[i] = (i < have) ? sm.tmp[i] : 0ull;
     __threadfence();
@@ -251,7 +258,7 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
     if (!sm.last) return;
     __threadfence();
 
-    // ---- last CTA of the pair: merge the per-slice lists (keys[] is reused)
+    // ---- last CTA of the pair: merge the per-slice sets (keys[] is reused)
     const int cap = a.slice;                   // room in keys[] (>= 2k by construction)
     int cnt = 0;
     u64 tau = 0ull;
@@ -268,13 +275,21 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
         __syncthreads();
         cnt = (int)sm.cnt;
         if (cnt > k) {
-            tau = block_topk_shrink(sm, keys, cnt, k);
+            tau = block_topk_select(sm, keys, cnt, k);
+            for (int i = tid; i < k; i += kRrThreads) keys[i] = sm.tmp[i];
             cnt = k;
+            __syncthreads();
         }
     }
     const int got = min(cnt, k);
     if (got != k && tid == 0) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
-    block_sort_desc(sm, keys, got);
+    // final order (score desc, id asc) by one warp
+    int p2 = 1;
+    while (p2 < k) p2 <<= 1;
+    for (int i = tid; i < p2; i += kRrThreads) sm.tmp[i] = (i < got) ? keys[i] : 0ull;
+    __syncthreads();
+    if (warp == 0) warp_sort_desc(sm.tmp, p2);
+    __syncthreads();
     for (int i = tid; i < k; i += kRrThreads) {
         const u64 x = sm.tmp[i];
         const bool live = i < got;

@@ -313,11 +313,6 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     sa.chunk_info = ix->chunk_info;
     sa.sstar = ix->sstar;
     sa.max_chunks = ix->max_chunks;
-    sa.one = 1u;
-    sa.m8 = 1u << 8;
-    sa.m16 = 1u << 16;
-    sa.m24 = 1u << 24;
-    sa.m29 = 1u << 29;
     if (dbg) {
         sa.dbg_S = dbg->S;
         sa.dbg_hist = dbg->hist;

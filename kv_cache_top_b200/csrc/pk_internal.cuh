@@ -80,9 +80,6 @@ struct ScanArgs {
     uint2 *chunk_info;       // [BH][max_chunks]  (first candidate slot, tie quota)
     int32_t *sstar;          // [BH]
     int32_t max_chunks;
-    // 1, 2^8, 2^16, 2^24, 2^29 passed at run time, so the compiler keeps the
-    // integer multiplies (fma pipe) that stand in for shifts and adds
-    uint32_t one, m8, m16, m24, m29;
     uint8_t *dbg_S;
     uint32_t *dbg_hist;
     int32_t *dbg_sstar;
