@@ -8,19 +8,19 @@
 //
 // Work is split by candidate slices (not key ranges), so every CTA reranks
 // the same number of records wherever the candidates sit.  A CTA stages its
-// candidate ids in shared memory; four lanes share a record, each loading one
-// 32-byte group (the nibbles of 4 blocks and their 4 weights) with two 16-byte
-// loads, so a warp moves 8 whole records per load pair and every lane decodes
-// 32 coordinates with no exchange.  The signed level of a nibble comes from a
-// 16-entry shared table (at most 16 distinct words per request: no bank
-// conflicts); q~ stays in registers.
+// candidate ids in shared memory; eight lanes share a record (one coalesced
+// 128-byte load, 16 bytes per lane) and after one pair exchange each lane
+// owns two blocks (16 coordinates) with their weights.  The signed level of a
+// nibble comes from a 16-entry shared table (at most 16 distinct words per
+// request: no bank conflicts); q~ stays in registers.
 //
 // Scores never leave the chip: the CTA turns (score, id) into 64-bit keys
 // ordered by score desc then id asc and radix-selects its Top-k set; the last
 // CTA of the pair (ticket counter, no spin-wait) merges the per-slice sets and
 // sorts the final Top-k with one warp (README: "reranks those candidates with
 // a fused 4-bit approximate inner-product kernel and selects the final Top-k
-// KV indices").  Block barriers are few: each radix pass costs two.
+// KV indices").  Block barriers are few: each radix pass costs two, and
+// appends to shared lists take one atomic per warp.
 #include "pk_internal.cuh"
 
 namespace pk {
@@ -36,16 +36,51 @@ struct RrShared {
     u64 red[2][kRrWarps];
     uint32_t sh[4];
     uint32_t cnt;
+    uint32_t bcnt;
     float slev[16];
     int last;
 };
+
+// Warp-aggregated append: every lane with `want` gets a distinct slot of
+// *ctr (one shared-memory atomic per warp instead of one per lane).
+__device__ __forceinline__ uint32_t warp_append(uint32_t *ctr, bool want)
+{
+    const int lane = threadIdx.x & 31;
+    const uint32_t bal = __ballot_sync(kFull, want);
+    if (!bal) return 0u;
+    const int leader = __ffs(bal) - 1;
+    uint32_t base = 0;
+    if (lane == leader) base = atomicAdd(ctr, (uint32_t)__popc(bal));
+    base = __shfl_sync(kFull, base, leader);
+    return base + (uint32_t)__popc(bal & ((1u << lane) - 1u));
+}
+
+// One warp sorts up to 32 keys (one per lane, missing ones = 0) descending;
+// returns the lane's key at its rank (rank = lane).
+__device__ __forceinline__ u64 warp_sort32_desc(u64 x)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const u64 y = __shfl_xor_sync(kFull, x, j);
+            const bool lower = (lane & j) == 0, desc = (lane & k) == 0;
+            const bool keep_max = (lower == desc);
+            x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
+        }
+    }
+    return x;
+}
 
 // Keep the k largest of keys[0..count) (count > k; keys distinct) in
 // sm.tmp[0..k), any order; returns the smallest kept key.  Radix select, most
 // significant digit first, starting at the highest bit where the keys differ
 // (scores of one query share sign and exponent, so leading digits would put
 // every key in one bin); histogram increments are aggregated per warp over
-// lanes that hit the same bin.  All threads of the block must call it.
+// lanes that hit the same bin.  Once the bin holding the k-th key has at most
+// 32 keys, one warp sorts that bin and finishes.  All threads of the block
+// must call it.
 __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -66,6 +101,10 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
         sm.red[1][warp] = hi;
     }
     for (int i = tid; i < 2 * 256; i += kRrThreads) (&sm.hist[0][0])[i] = 0u;
+    if (tid == 0) {
+        sm.sh[3] = 0;
+        sm.bcnt = 0;
+    }
     __syncthreads();
 #pragma unroll
     for (int w = 0; w < kRrWarps; w++) {
@@ -77,6 +116,8 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
     u64 prefix = hi & mask;
     int need = k;
     int pass = 0;
+    uint32_t inbin = 0;
+    u64 bmask = 0, bprefix = 0;         // the boundary bin (valid when it is small)
     for (int top = hb; top >= 0; top -= 8, pass ^= 1) {
         const int width = top + 1 < 8 ? top + 1 : 8;
         const int shift = top + 1 - width;
@@ -121,29 +162,56 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
             }
         }
         __syncthreads();
-        const uint32_t d = sm.sh[0], above = sm.sh[1], inbin = sm.sh[2];
+        const uint32_t d = sm.sh[0], above = sm.sh[1];
+        inbin = sm.sh[2];
         need -= (int)above;
-        prefix |= (u64)d << shift;
-        mask |= (u64)dmask << shift;
-        if ((int)inbin == need) break;
+        bprefix = prefix | ((u64)d << shift);
+        bmask = mask | ((u64)dmask << shift);
+        // keys strictly above the boundary bin stay in the (prefix, mask) test below
+        if ((int)inbin == need || inbin <= 32u) break;
+        prefix = bprefix;
+        mask = bmask;
     }
-    // everything at or above the selected prefix: exactly k keys
-    if (tid == 0) sm.sh[3] = 0;
-    __syncthreads();
+    // keys in bins above the boundary bin: (x & mask) == prefix and x's digit > d,
+    // i.e. (x & bmask) > bprefix; they are all kept.  Keys of the boundary bin
+    // go to a side list when the bin is small.
+    const bool small = (int)inbin != need;
     u64 mn = ~0ull;
-    for (int i = tid; i < count; i += kRrThreads) {
-        const u64 x = keys[i];
-        if ((x & mask) >= prefix) {
-            const uint32_t pos = atomicAdd(&sm.sh[3], 1u);
+    for (int base = 0; base < count; base += kRrThreads) {
+        const int i = base + tid;
+        u64 x = 0;
+        bool above = false, inb = false;
+        if (i < count) {
+            x = keys[i];
+            const u64 xm = x & bmask;
+            // bmask covers mask, so (x & bmask) orders keys by their selected prefix
+            above = small ? (xm > bprefix) : (xm >= bprefix);
+            inb = small && xm == bprefix;
+        }
+        const uint32_t pos = warp_append(&sm.sh[3], above);
+        if (above) {
             if (pos < (uint32_t)kMaxTopk) sm.tmp[pos] = x;
             mn = x < mn ? x : mn;
         }
+        const uint32_t bpos = warp_append(&sm.bcnt, inb);
+        if (inb && bpos < 32u) reinterpret_cast<u64 *>(sm.hist[pass ^ 1])[bpos] = x;
+    }
+    __syncthreads();
+    if (small && warp == 0) {
+        // sort the boundary bin (<= 32 keys) and keep its `need` best
+        const uint32_t nb = sm.bcnt;
+        u64 x = (lane < (int)nb) ? reinterpret_cast<const u64 *>(sm.hist[pass ^ 1])[lane] : 0ull;
+        x = warp_sort32_desc(x);
+        const uint32_t base = sm.sh[3];
+        if (lane < need && base + lane < (uint32_t)kMaxTopk) sm.tmp[base + lane] = x;
+        if (lane < need) mn = x < mn ? x : mn;
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
         const u64 y = __shfl_xor_sync(kFull, mn, o);
         mn = y < mn ? y : mn;
     }
+    __syncthreads();
     if (lane == 0) sm.red[0][warp] = mn;
     __syncthreads();
 #pragma unroll
@@ -202,37 +270,43 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
     if (tid < 16) sm.slev[tid] = (tid & 8) ? -a.lv.lev[tid & 7] : a.lv.lev[tid & 7];
     const int32_t *cand = a.cand + (size_t)bh * a.stride + m0;
     for (int i = tid; i < count; i += kRrThreads) ids[i] = cand[i];
-    const int q4 = lane & 3, sub = lane >> 2;          // group of the record, record of the warp step
-    float qr[32];
+    const int q8 = lane & 7, sub = lane >> 3;          // 16-byte piece of the record, record of the warp step
+    float qr[16];
 #pragma unroll
-    for (int i = 0; i < 32; i++) qr[i] = a.qt[(size_t)bh * kD + 32 * q4 + i];
+    for (int i = 0; i < 16; i++) qr[i] = a.qt[(size_t)bh * kD + 16 * q8 + i];
     const float qnorm = a.qnorm[bh];
-    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes + 32 * q4;
+    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes;
     float *dest = a.dbg_est ? a.dbg_est + (size_t)bh * a.C + m0 : nullptr;
     __syncthreads();
 
-    // each warp step: 16 records, two 16-byte loads per lane per record group
+    // each warp step: 16 records, one coalesced 16-byte load per lane per record
+    const bool odd = (q8 & 1) != 0;
     for (int r0 = warp * 16; r0 < count; r0 += kRrWarps * 16) {
-        uint4 nv[2], wv[2];
-        int32_t id[2];
+        uint4 v[4];
+        int32_t id[4];
 #pragma unroll
-        for (int u = 0; u < 2; u++) {
-            const int r = r0 + 8 * u + sub;
+        for (int u = 0; u < 4; u++) {
+            const int r = r0 + 4 * u + sub;
             id[u] = ids[r < count ? r : 0];
-            const uint4 *p = reinterpret_cast<const uint4 *>(rec + (size_t)id[u] * kRecBytes);
-            nv[u] = __ldg(p);
-            wv[u] = __ldg(p + 1);
+            v[u] = __ldg(reinterpret_cast<const uint4 *>(rec + (size_t)id[u] * kRecBytes) + q8);
         }
 #pragma unroll
-        for (int u = 0; u < 2; u++) {
-            float part = __uint_as_float(wv[u].x) * block_dot(sm.slev, nv[u].x, qr);
-            part = fmaf(__uint_as_float(wv[u].y), block_dot(sm.slev, nv[u].y, qr + 8), part);
-            part = fmaf(__uint_as_float(wv[u].z), block_dot(sm.slev, nv[u].z, qr + 16), part);
-            part = fmaf(__uint_as_float(wv[u].w), block_dot(sm.slev, nv[u].w, qr + 24), part);
+        for (int u = 0; u < 4; u++) {
+            // even lane of a pair: nibble words of blocks 4g..4g+3; odd lane: their
+            // weights.  Swap halves so lane q8 owns blocks 2 q8, 2 q8 + 1.
+            const uint32_t r0v = __shfl_xor_sync(kFull, odd ? v[u].x : v[u].z, 1);
+            const uint32_t r1v = __shfl_xor_sync(kFull, odd ? v[u].y : v[u].w, 1);
+            const uint32_t nib0 = odd ? r0v : v[u].x, nib1 = odd ? r1v : v[u].y;
+            const float w0 = __uint_as_float(odd ? v[u].z : r0v);
+            const float w1 = __uint_as_float(odd ? v[u].w : r1v);
+            const float d0 = block_dot(sm.slev, nib0, qr);
+            const float d1 = block_dot(sm.slev, nib1, qr + 8);
+            float part = fmaf(w0, d0, w1 * d1);
             part += __shfl_xor_sync(kFull, part, 1);
             part += __shfl_xor_sync(kFull, part, 2);
-            const int r = r0 + 8 * u + sub;
-            if (q4 == 0 && r < count) {
+            part += __shfl_xor_sync(kFull, part, 4);
+            const int r = r0 + 4 * u + sub;
+            if (q8 == 0 && r < count) {
                 const float est = qnorm * part;
                 keys[r] = make_key(est, id[u]);
                 if (dest) dest[r] = est;
@@ -267,10 +341,16 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
         const int64_t e1 = min(total, e0 + (cap - k));
         if (tid == 0) sm.cnt = (uint32_t)cnt;
         __syncthreads();
-        for (int64_t e = e0 + tid; e < e1; e += kRrThreads) {
-            const int64_t j = e / k, r = e - j * k;
-            const u64 x = __ldcg(a.partial + ((size_t)bh * a.max_slices + j) * a.topk_cap + r);
-            if (x != 0ull && x > tau) keys[atomicAdd(&sm.cnt, 1u)] = x;
+        for (int64_t eb = e0; eb < e1; eb += kRrThreads) {
+            const int64_t e = eb + tid;
+            u64 x = 0ull;
+            if (e < e1) {
+                const int64_t j = e / k, r = e - j * k;
+                x = __ldcg(a.partial + ((size_t)bh * a.max_slices + j) * a.topk_cap + r);
+            }
+            const bool take = x != 0ull && x > tau;
+            const uint32_t pos = warp_append(&sm.cnt, take);
+            if (take) keys[pos] = x;
         }
         __syncthreads();
         cnt = (int)sm.cnt;
