@@ -315,16 +315,18 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
     }
     __syncthreads();
 
-    // ---- Top-k set of the slice (unordered)
+    // ---- Top-k set of the slice (unordered) and its smallest key
     const int have = min(count, k);
+    u64 kth = 0ull;                  // a lower bound of the pair's k-th key (0: none)
     if (count > k) {
-        block_topk_select(sm, keys, count, k);
+        kth = block_topk_select(sm, keys, count, k);
     } else {
         for (int i = tid; i < count; i += kRrThreads) sm.tmp[i] = keys[i];
         __syncthreads();
     }
     u64 *part = a.partial + ((size_t)bh * a.max_slices + sl) * a.topk_cap;
     for (int i = tid; i < k; i += kRrThreads) part[i] = (i < have) ? sm.tmp[i] : 0ull;
+    if (tid == 0) a.slice_kth[(size_t)bh * a.max_slices + sl] = kth;
     __threadfence();
     __syncthreads();
     if (tid == 0) sm.last = (atomicAdd(&a.tickets[(size_t)bh * 2 + 1], 1u) == (unsigned)(a.nslices - 1));
@@ -332,10 +334,30 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
     if (!sm.last) return;
     __threadfence();
 
-    // ---- last CTA of the pair: merge the per-slice sets (keys[] is reused)
+    // ---- last CTA of the pair: merge the per-slice sets (keys[] is reused).
+    // A slice holding k keys >= its smallest kept key m_j proves the pair's
+    // k-th key >= m_j, so keys below max_j m_j are dropped as they are read.
     const int cap = a.slice;                   // room in keys[] (>= 2k by construction)
     int cnt = 0;
     u64 tau = 0ull;
+    {
+        u64 t = 0ull;
+        for (int j = tid; j < a.nslices; j += kRrThreads) {
+            const u64 m = __ldcg(a.slice_kth + (size_t)bh * a.max_slices + j);
+            t = m > t ? m : t;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const u64 y = __shfl_xor_sync(kFull, t, o);
+            t = y > t ? y : t;
+        }
+        if (lane == 0) sm.red[1][warp] = t;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < kRrWarps; w++) t = sm.red[1][w] > t ? sm.red[1][w] : t;
+        tau = t;
+        __syncthreads();
+    }
     const int64_t total = (int64_t)a.nslices * k;
     for (int64_t e0 = 0; e0 < total; e0 += cap - k) {
         const int64_t e1 = min(total, e0 + (cap - k));
@@ -348,7 +370,7 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
                 const int64_t j = e / k, r = e - j * k;
                 x = __ldcg(a.partial + ((size_t)bh * a.max_slices + j) * a.topk_cap + r);
             }
-            const bool take = x != 0ull && x > tau;
+            const bool take = x != 0ull && x >= tau;
             const uint32_t pos = warp_append(&sm.cnt, take);
             if (take) keys[pos] = x;
         }

@@ -44,6 +44,7 @@ struct pk_index {
     int32_t *sstar = nullptr;
     int32_t *cand = nullptr;
     unsigned long long *partial = nullptr;
+    unsigned long long *slice_kth = nullptr;
     int32_t max_slices = 1;
 
     int32_t *dev_err = nullptr;
@@ -174,6 +175,7 @@ void free_all(pk_index *ix)
     cudaFree(ix->sstar);
     cudaFree(ix->cand);
     cudaFree(ix->partial);
+    cudaFree(ix->slice_kth);
 
     cudaFree(ix->dev_err);
     cudaFree(ix->dev_err_detail);
@@ -355,6 +357,7 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     ra.topk_cap = ix->topk_cap;
     ra.tickets = ix->tickets;
     ra.partial = ix->partial;
+    ra.slice_kth = ix->slice_kth;
     ra.lv = ix->lv;
     ra.out_idx = out_idx;
     ra.out_score = out_score;
@@ -497,6 +500,7 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     const size_t MS = ix->max_slices;
     chk(dalloc(&ix->cand, BH * NC));
     chk(dalloc(&ix->partial, BH * MS * (size_t)ix->topk_cap));
+    chk(dalloc(&ix->slice_kth, BH * MS));
 
     chk(dalloc(&ix->dev_err, 1));
     chk(dalloc(&ix->dev_err_detail, 1));

@@ -106,6 +106,7 @@ struct RerankArgs {
     int32_t slice, nslices, max_slices, topk, topk_cap;
     uint32_t *tickets;
     unsigned long long *partial;   // [BH][max_slices][topk_cap]
+    unsigned long long *slice_kth; // [BH][max_slices] smallest key each slice kept
     Levels lv;
     int32_t *out_idx;        // [BH][topk]
     float *out_score;        // [BH][topk] or null
