@@ -155,6 +155,7 @@ def profiled_traffic(kernel: str, workload: str):
     files = {"collision_scan": ["k_collision_scan.cu", "pk_internal.cuh"],
              "rerank_topk": ["k_rerank_topk.cu", "pk_internal.cuh"],
              "compact": ["k_compact.cu", "pk_internal.cuh"],
+             "topk_merge": ["k_rerank_topk.cu", "pk_internal.cuh"],
              "query_prep": ["k_query_prep.cu", "pk_internal.cuh"],
              "gather_attend": ["k_gather_attend.cu", "pk_internal.cuh"]}.get(kernel)
     if not m or not hm or not files or hm.group(1) != src_hash(*files):
@@ -173,7 +174,9 @@ def alg_bytes(kernel: str, wl: dict, C: int, topk: int = 100):
     if kernel == "compact":
         return bh * (n + 4 * C)                      # S read + candidate ids written
     if kernel == "rerank_topk":
-        return bh * (132 * C + 8 * topk)             # ids + candidate records + result
+        return bh * (132 * C)                        # ids + candidate records
+    if kernel == "topk_merge":
+        return bh * 16 * topk * max(1, C // 1472)    # per-slice sets read + result (estimate)
     if kernel == "gather_attend":
         return bh * (2 * topk * 128 * 2 + G * 128 * (2 + 4))   # K/V rows + q + o
     raise KeyError(kernel)
@@ -428,7 +431,8 @@ def main():
         att = km.get("gather_attend", {})
         mil = {"workload": wl_m["name"], "steps_s": margs.steps * world / (rm["ms_total"] / 1000.0),
                "ms_per_step": rm["ms_total"] / margs.steps, "steps": margs.steps,
-               "search_us": sum(km[k]["avg_us"] for k in ("query_prep", "collision_scan", "compact", "rerank_topk")
+               "search_us": sum(km[k]["avg_us"] for k in ("query_prep", "collision_scan", "compact", "rerank_topk",
+                                          "topk_merge")
                                 if k in km),
                "attend_us": att.get("avg_us"), "recall_at_100": rm["recall"],
                "uva_bytes_per_step": link_bytes,
@@ -481,7 +485,7 @@ def main():
                      "unit": "GB/s", "frac": km[dom]["gbs"] / peak,
                      "traffic": profiled_traffic(dom, wl["name"]), "peak_source": peak_src},
         "kernels": km,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": 6 * args.steps,
         "clocks": res["clocks"],
         "e2e": res["e2e"],
         "cpu_baseline": res.get("cpu"),

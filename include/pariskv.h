@@ -202,10 +202,10 @@ pk_status pk_resolve(int64_t n, int64_t cand_budget, float collision_ratio, int3
 /* Per-kernel timing.  While tracing is on, the library records a CUDA event
  * pair on the launching stream around each of its kernels.  pk_trace_read
  * synchronises, then returns per kernel kind (0 encode, 1 query_prep,
- * 2 collision_scan, 3 compact, 4 rerank_topk, 5 gather_attend) the launch
- * count and the summed event time in ms; it clears the record. */
+ * 2 collision_scan, 3 compact, 4 rerank_topk, 5 topk_merge, 6 gather_attend)
+ * the launch count and the summed event time in ms; it clears the record. */
 enum { PK_K_ENCODE = 0, PK_K_QUERY_PREP = 1, PK_K_COLLISION_SCAN = 2, PK_K_COMPACT = 3,
-       PK_K_RERANK_TOPK = 4, PK_K_GATHER_ATTEND = 5, PK_K_COUNT = 6 };
+       PK_K_RERANK_TOPK = 4, PK_K_TOPK_MERGE = 5, PK_K_GATHER_ATTEND = 6, PK_K_COUNT = 7 };
 pk_status pk_trace_enable(pk_index *index, int32_t on);
 pk_status pk_trace_read(pk_index *index, int64_t *launches, double *total_ms);
 

@@ -21,7 +21,8 @@ PK_OK, PK_ERR_INVALID_ARG, PK_ERR_CAPACITY, PK_ERR_OOM, PK_ERR_CUDA, PK_ERR_TIME
     PK_ERR_DEVICE_CHECK, PK_ERR_UNSUPPORTED = range(8)
 PK_F32, PK_BF16 = 0, 1
 PK_KV_DEVICE, PK_KV_HOST_PINNED = 0, 1
-KERNELS = ("encode", "query_prep", "collision_scan", "compact", "rerank_topk", "gather_attend")
+KERNELS = ("encode", "query_prep", "collision_scan", "compact", "rerank_topk", "topk_merge",
+           "gather_attend")
 
 
 class pk_params(C.Structure):

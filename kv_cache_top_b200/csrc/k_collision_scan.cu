@@ -26,6 +26,7 @@
 namespace pk {
 
 constexpr int kScanThreads = 256;
+constexpr int kScanUnroll = 4;
 constexpr int kHistPad = 104;
 
 __device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], uint4 c)
@@ -74,33 +75,25 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
     uint8_t *S = a.S + (size_t)bh * a.n_cap + lo;
     uint8_t *dS = a.dbg_S ? a.dbg_S + (size_t)bh * a.n + lo : nullptr;
 
-    // each thread scores 4 consecutive keys per step (one packed 4-byte S
-    // store); every lane runs every step (the shuffles need the full warp):
-    // lanes past the end of the chunk score zero codes and store nothing
-    for (int64_t base = 0; base < cnt; base += 4 * kScanThreads) {
-        const int64_t i0 = base + 4 * tid;
-        uint4 c[4];
+    // every lane runs every iteration (the shuffles need the full warp);
+    // lanes past the end of the chunk compute on a zero code and store nothing
+    for (int64_t base = (int64_t)warp * 32 * kScanUnroll; base < cnt;
+         base += (int64_t)NW * 32 * kScanUnroll) {
+        uint4 c[kScanUnroll];
 #pragma unroll
-        for (int u = 0; u < 4; u++) c[u] = (i0 + u < cnt) ? __ldg(codes + i0 + u) : make_uint4(0, 0, 0, 0);
-        uint32_t sv[4];
-#pragma unroll
-        for (int u = 0; u < 4; u++) sv[u] = collision_score(tab, c[u]);
-        if (i0 + 3 < cnt) {
-            *reinterpret_cast<uint32_t *>(S + i0) = sv[0] | (sv[1] << 8) | (sv[2] << 16) | (sv[3] << 24);
-#pragma unroll
-            for (int u = 0; u < 4; u++) atomicAdd(&s_hist[warp][sv[u]], 1u);
-        } else {
-#pragma unroll
-            for (int u = 0; u < 4; u++)
-                if (i0 + u < cnt) {
-                    S[i0 + u] = (uint8_t)sv[u];
-                    atomicAdd(&s_hist[warp][sv[u]], 1u);
-                }
+        for (int u = 0; u < kScanUnroll; u++) {
+            const int64_t i = base + u * 32 + lane;
+            c[u] = (i < cnt) ? __ldcs(codes + i) : make_uint4(0, 0, 0, 0);
         }
-        if (dS) {
 #pragma unroll
-            for (int u = 0; u < 4; u++)
-                if (i0 + u < cnt) dS[i0 + u] = (uint8_t)sv[u];
+        for (int u = 0; u < kScanUnroll; u++) {
+            const int64_t i = base + u * 32 + lane;
+            const uint32_t s = collision_score(tab, c[u]);
+            if (i < cnt) {
+                S[i] = (uint8_t)s;
+                if (dS) dS[i] = (uint8_t)s;
+                atomicAdd(&s_hist[warp][s], 1u);
+            }
         }
     }
     __syncthreads();

@@ -15,12 +15,12 @@
 // request: no bank conflicts); q~ stays in registers.
 //
 // Scores never leave the chip: the CTA turns (score, id) into 64-bit keys
-// ordered by score desc then id asc and radix-selects its Top-k set; the last
-// CTA of the pair (ticket counter, no spin-wait) merges the per-slice sets and
-// sorts the final Top-k with one warp (README: "reranks those candidates with
-// a fused 4-bit approximate inner-product kernel and selects the final Top-k
-// KV indices").  Block barriers are few: each radix pass costs two, and
-// appends to shared lists take one atomic per warp.
+// ordered by score desc then id asc and radix-selects its Top-k set; a merge
+// kernel (one CTA per pair) selects the final Top-k from the per-slice sets
+// and sorts it with one warp (README: "reranks those candidates with a fused
+// 4-bit approximate inner-product kernel and selects the final Top-k KV
+// indices").  Block barriers are few: each radix pass costs two, and appends
+// to shared lists take one atomic per warp.
 #include "pk_internal.cuh"
 
 namespace pk {
@@ -317,47 +317,32 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
 
     // ---- Top-k set of the slice (unordered) and its smallest key
     const int have = min(count, k);
-    u64 kth = 0ull;                  // a lower bound of the pair's k-th key (0: none)
     if (count > k) {
-        kth = block_topk_select(sm, keys, count, k);
+        block_topk_select(sm, keys, count, k);
     } else {
         for (int i = tid; i < count; i += kRrThreads) sm.tmp[i] = keys[i];
         __syncthreads();
     }
     u64 *part = a.partial + ((size_t)bh * a.max_slices + sl) * a.topk_cap;
     for (int i = tid; i < k; i += kRrThreads) part[i] = (i < have) ? sm.tmp[i] : 0ull;
-    if (tid == 0) a.slice_kth[(size_t)bh * a.max_slices + sl] = kth;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sm.last = (atomicAdd(&a.tickets[(size_t)bh * 2 + 1], 1u) == (unsigned)(a.nslices - 1));
-    __syncthreads();
-    if (!sm.last) return;
-    __threadfence();
+}
 
-    // ---- last CTA of the pair: merge the per-slice sets (keys[] is reused).
-    // A slice holding k keys >= its smallest kept key m_j proves the pair's
-    // k-th key >= m_j, so keys below max_j m_j are dropped as they are read.
-    const int cap = a.slice;                   // room in keys[] (>= 2k by construction)
+// Merge of the per-slice Top-k sets of one pair into its final sorted Top-k.
+// One CTA per pair holds as many partial keys as its shared memory allows
+// (all of them in the usual case) and radix-selects once; larger merges run
+// in rounds that keep the best k seen so far.  The final order (score desc,
+// id asc) is produced by one warp.
+__global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
+{
+    extern __shared__ __align__(16) unsigned char s_dyn[];
+    __shared__ RrShared sm;
+    u64 *keys = reinterpret_cast<u64 *>(s_dyn);
+    const int bh = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int k = a.topk;
+    const int cap = a.cap;                     // keys[] capacity (>= 2k)
     int cnt = 0;
     u64 tau = 0ull;
-    {
-        u64 t = 0ull;
-        for (int j = tid; j < a.nslices; j += kRrThreads) {
-            const u64 m = __ldcg(a.slice_kth + (size_t)bh * a.max_slices + j);
-            t = m > t ? m : t;
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const u64 y = __shfl_xor_sync(kFull, t, o);
-            t = y > t ? y : t;
-        }
-        if (lane == 0) sm.red[1][warp] = t;
-        __syncthreads();
-#pragma unroll
-        for (int w = 0; w < kRrWarps; w++) t = sm.red[1][w] > t ? sm.red[1][w] : t;
-        tau = t;
-        __syncthreads();
-    }
     const int64_t total = (int64_t)a.nslices * k;
     for (int64_t e0 = 0; e0 < total; e0 += cap - k) {
         const int64_t e1 = min(total, e0 + (cap - k));
@@ -368,9 +353,9 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
             u64 x = 0ull;
             if (e < e1) {
                 const int64_t j = e / k, r = e - j * k;
-                x = __ldcg(a.partial + ((size_t)bh * a.max_slices + j) * a.topk_cap + r);
+                x = a.partial[((size_t)bh * a.max_slices + j) * a.topk_cap + r];
             }
-            const bool take = x != 0ull && x >= tau;
+            const bool take = x != 0ull && x > tau;
             const uint32_t pos = warp_append(&sm.cnt, take);
             if (take) keys[pos] = x;
         }
@@ -385,7 +370,6 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
     }
     const int got = min(cnt, k);
     if (got != k && tid == 0) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
-    // final order (score desc, id asc) by one warp
     int p2 = 1;
     while (p2 < k) p2 <<= 1;
     for (int i = tid; i < p2; i += kRrThreads) sm.tmp[i] = (i < got) ? keys[i] : 0ull;
@@ -398,7 +382,22 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
         a.out_idx[(size_t)bh * k + i] = live ? (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu)) : -1;
         if (a.out_score) a.out_score[(size_t)bh * k + i] = live ? unord_f32((uint32_t)(x >> 32)) : 0.0f;
     }
-    if (tid == 0) a.tickets[(size_t)bh * 2 + 1] = 0u;
+}
+
+size_t merge_smem(int cap) { return (size_t)cap * sizeof(u64); }
+
+cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s)
+{
+    static int attr_max = 0;
+    const size_t smem = merge_smem(a.cap);
+    if ((int)smem > attr_max) {
+        cudaError_t e = cudaFuncSetAttribute(k_topk_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)merge_smem(kMergeCap));
+        if (e != cudaSuccess) return e;
+        attr_max = (int)merge_smem(kMergeCap);
+    }
+    k_topk_merge<<<bh, kRrThreads, smem, s>>>(a);
+    return cudaGetLastError();
 }
 
 size_t rerank_smem(int slice) { return (size_t)slice * (sizeof(u64) + sizeof(int32_t)); }

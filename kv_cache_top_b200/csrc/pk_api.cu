@@ -44,7 +44,6 @@ struct pk_index {
     int32_t *sstar = nullptr;
     int32_t *cand = nullptr;
     unsigned long long *partial = nullptr;
-    unsigned long long *slice_kth = nullptr;
     int32_t max_slices = 1;
 
     int32_t *dev_err = nullptr;
@@ -175,7 +174,6 @@ void free_all(pk_index *ix)
     cudaFree(ix->sstar);
     cudaFree(ix->cand);
     cudaFree(ix->partial);
-    cudaFree(ix->slice_kth);
 
     cudaFree(ix->dev_err);
     cudaFree(ix->dev_err_detail);
@@ -355,16 +353,29 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     ra.max_slices = ix->max_slices;
     ra.topk = topk;
     ra.topk_cap = ix->topk_cap;
-    ra.tickets = ix->tickets;
     ra.partial = ix->partial;
-    ra.slice_kth = ix->slice_kth;
     ra.lv = ix->lv;
-    ra.out_idx = out_idx;
-    ra.out_score = out_score;
     ra.dbg_est = dbg ? dbg->cand_est : nullptr;
-    ra.dev_err = ix->dev_err;
     trace_begin(ix, PK_K_RERANK_TOPK, s);
     e = launch_rerank_topk(ra, ix->bh, s);
+    trace_end(ix, s);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    MergeArgs ma{};
+    ma.partial = ix->partial;
+    ma.nslices = ra.nslices;
+    ma.max_slices = ix->max_slices;
+    ma.topk = topk;
+    ma.topk_cap = ix->topk_cap;
+    {
+        const int64_t want = (int64_t)ra.nslices * topk;
+        ma.cap = (int32_t)std::max<int64_t>(2 * (int64_t)topk, std::min<int64_t>(want, kMergeCap));
+    }
+    ma.out_idx = out_idx;
+    ma.out_score = out_score;
+    ma.dev_err = ix->dev_err;
+    trace_begin(ix, PK_K_TOPK_MERGE, s);
+    e = launch_topk_merge(ma, ix->bh, s);
     trace_end(ix, s);
     return cuda_status(e);
 }
@@ -500,7 +511,6 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     const size_t MS = ix->max_slices;
     chk(dalloc(&ix->cand, BH * NC));
     chk(dalloc(&ix->partial, BH * MS * (size_t)ix->topk_cap));
-    chk(dalloc(&ix->slice_kth, BH * MS));
 
     chk(dalloc(&ix->dev_err, 1));
     chk(dalloc(&ix->dev_err_detail, 1));

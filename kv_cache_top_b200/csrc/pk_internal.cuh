@@ -23,6 +23,7 @@ constexpr int kMaxTopk = 1024;
 constexpr int kMaxGroup = 8;
 constexpr int kMaxSlice = 4096;  // candidates per rerank CTA (upper bound)
 constexpr int kAtRows = 32;      // selected rows per attention CTA (upper bound)
+constexpr int kMergeCap = 16384; // partial keys one merge CTA holds at once
 constexpr unsigned kFull = 0xffffffffu;
 
 // Device-check codes written to the index's error word (first one wins).
@@ -104,13 +105,16 @@ struct RerankArgs {
     const float *qnorm;
     int64_t stride, C;
     int32_t slice, nslices, max_slices, topk, topk_cap;
-    uint32_t *tickets;
-    unsigned long long *partial;   // [BH][max_slices][topk_cap]
-    unsigned long long *slice_kth; // [BH][max_slices] smallest key each slice kept
+    unsigned long long *partial;   // [BH][max_slices][topk_cap]  per-slice Top-k sets
     Levels lv;
+    float *dbg_est;          // [BH][C] or null
+};
+
+struct MergeArgs {
+    const unsigned long long *partial;
+    int32_t nslices, max_slices, topk, topk_cap, cap;
     int32_t *out_idx;        // [BH][topk]
     float *out_score;        // [BH][topk] or null
-    float *dbg_est;          // [BH][C] or null
     int32_t *dev_err;
 };
 
@@ -249,6 +253,7 @@ cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s);
 cudaError_t launch_collision_scan(const ScanArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_compact(const CompactArgs &a, int nchunks, int bh, cudaStream_t s);
 cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s);
+cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s);
 size_t rerank_smem(int slice);
 // host-side Lloyd-Max levels of the magnitude prior (closed-form integrals)
