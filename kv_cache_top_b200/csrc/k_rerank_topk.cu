@@ -219,24 +219,77 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
     return mn;
 }
 
-// One warp sorts sm.tmp[0..p2) descending in place (p2 a power of two <= 1024).
-__device__ void warp_sort_desc(u64 *v, int p2)
+// One warp sorts v[0..32 E) descending in place: E keys per lane in
+// registers (element e = E lane + i), bitonic network, shuffles for the
+// cross-lane stages -- no shared-memory round trips between stages.
+template <int E>
+__device__ void warp_sort_desc_reg(u64 *v)
 {
     const int lane = threadIdx.x & 31;
-    for (int kk = 2; kk <= p2; kk <<= 1) {
-        for (int j = kk >> 1; j > 0; j >>= 1) {
-            for (int i = lane; i < p2; i += 32) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const u64 x = v[i], y = v[ixj];
-                    const bool desc = (i & kk) == 0;
-                    if (desc ? (x < y) : (x > y)) {
-                        v[i] = y;
-                        v[ixj] = x;
+    constexpr int N = 32 * E;
+    u64 x[E];
+#pragma unroll
+    for (int i = 0; i < E; i++) x[i] = v[E * lane + i];
+#pragma unroll
+    for (int k = 2; k <= N; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j >= E) {
+                const int lx = j / E;
+#pragma unroll
+                for (int i = 0; i < E; i++) {
+                    const int e = E * lane + i;
+                    const u64 o = __shfl_xor_sync(kFull, x[i], lx);
+                    const bool keep_max = ((e & j) == 0) == ((e & k) == 0);
+                    x[i] = keep_max ? (o > x[i] ? o : x[i]) : (o < x[i] ? o : x[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < E; i++) {
+                    if ((i & j) == 0) {
+                        const int e = E * lane + i;
+                        const bool desc = (e & k) == 0;
+                        const u64 a = x[i], b = x[i ^ j];
+                        const u64 hi = a > b ? a : b, lo = a > b ? b : a;
+                        x[i] = desc ? hi : lo;
+                        x[i ^ j] = desc ? lo : hi;
                     }
                 }
             }
-            __syncwarp();
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < E; i++) v[E * lane + i] = x[i];
+}
+
+// One warp sorts v[0..p2) descending in place (p2 a power of two <= 1024).
+__device__ void warp_sort_desc(u64 *v, int p2)
+{
+    if (p2 <= 32) {
+        warp_sort_desc_reg<1>(v);      // callers pad to >= 32 entries with zeros
+    } else if (p2 == 64) {
+        warp_sort_desc_reg<2>(v);
+    } else if (p2 == 128) {
+        warp_sort_desc_reg<4>(v);
+    } else if (p2 == 256) {
+        warp_sort_desc_reg<8>(v);
+    } else {
+        const int lane = threadIdx.x & 31;
+        for (int kk = 2; kk <= p2; kk <<= 1) {
+            for (int j = kk >> 1; j > 0; j >>= 1) {
+                for (int i = lane; i < p2; i += 32) {
+                    const int ixj = i ^ j;
+                    if (ixj > i) {
+                        const u64 x = v[i], y = v[ixj];
+                        const bool desc = (i & kk) == 0;
+                        if (desc ? (x < y) : (x > y)) {
+                            v[i] = y;
+                            v[ixj] = x;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
         }
     }
 }
@@ -348,16 +401,24 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
         const int64_t e1 = min(total, e0 + (cap - k));
         if (tid == 0) sm.cnt = (uint32_t)cnt;
         __syncthreads();
-        for (int64_t eb = e0; eb < e1; eb += kRrThreads) {
-            const int64_t e = eb + tid;
-            u64 x = 0ull;
-            if (e < e1) {
-                const int64_t j = e / k, r = e - j * k;
-                x = a.partial[((size_t)bh * a.max_slices + j) * a.topk_cap + r];
+        constexpr int kB8 = 8;       // loads in flight per thread
+        for (int64_t eb = e0; eb < e1; eb += (int64_t)kB8 * kRrThreads) {
+            u64 x[kB8];
+#pragma unroll
+            for (int u = 0; u < kB8; u++) {
+                const int64_t e = eb + (int64_t)u * kRrThreads + tid;
+                x[u] = 0ull;
+                if (e < e1) {
+                    const int64_t j = e / k, r = e - j * k;
+                    x[u] = a.partial[((size_t)bh * a.max_slices + j) * a.topk_cap + r];
+                }
             }
-            const bool take = x != 0ull && x > tau;
-            const uint32_t pos = warp_append(&sm.cnt, take);
-            if (take) keys[pos] = x;
+#pragma unroll
+            for (int u = 0; u < kB8; u++) {
+                const bool take = x[u] != 0ull && x[u] > tau;
+                const uint32_t pos = warp_append(&sm.cnt, take);
+                if (take) keys[pos] = x[u];
+            }
         }
         __syncthreads();
         cnt = (int)sm.cnt;
@@ -370,7 +431,7 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
     }
     const int got = min(cnt, k);
     if (got != k && tid == 0) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
-    int p2 = 1;
+    int p2 = 32;
     while (p2 < k) p2 <<= 1;
     for (int i = tid; i < p2; i += kRrThreads) sm.tmp[i] = (i < got) ? keys[i] : 0ull;
     __syncthreads();

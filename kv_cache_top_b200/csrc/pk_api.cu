@@ -369,7 +369,8 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     ma.topk_cap = ix->topk_cap;
     {
         const int64_t want = (int64_t)ra.nslices * topk;
-        ma.cap = (int32_t)std::max<int64_t>(2 * (int64_t)topk, std::min<int64_t>(want, kMergeCap));
+        // room for every partial key at once (one select) when it fits
+        ma.cap = (int32_t)std::max<int64_t>(2 * (int64_t)topk, std::min<int64_t>(want + topk, kMergeCap));
     }
     ma.out_idx = out_idx;
     ma.out_score = out_score;
