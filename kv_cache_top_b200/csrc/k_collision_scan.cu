@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
 
     for (int i = tid; i < NW * kHistPad; i += kScanThreads) (&s_hist[0][0])[i] = 0u;
 
+    pdl_wait();                                   // bonus tables come from the query preparation
     uint32_t tab[kB];
     const uint32_t *bp = a.bonus_packed + (size_t)bh * kB * 32;
 #pragma unroll
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
 
     __threadfence();
     __syncthreads();
+    pdl_trigger();
     if (tid == 0) s_last = (atomicAdd(&a.tickets[(size_t)bh * 2 + 0], 1u) == (unsigned)(a.nchunks - 1));
     __syncthreads();
     if (!s_last) return;
@@ -178,7 +180,6 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
 namespace pk {
 cudaError_t launch_collision_scan(const ScanArgs &a, int bh, cudaStream_t s)
 {
-    k_collision_scan<<<dim3(a.nchunks, bh), kScanThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k_collision_scan, dim3(a.nchunks, bh), dim3(kScanThreads), 0, s, a);
 }
 }  // namespace pk

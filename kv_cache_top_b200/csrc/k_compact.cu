@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kCpThreads) k_compact(CompactArgs a)
     const int tid = threadIdx.x;
     const int64_t lo = (int64_t)chunk * a.chunk;
     const int64_t hi = min(lo + a.chunk, a.n);
+    pdl_wait();                                   // S, s* and chunk slots come from the scan
     const uint2 info = a.chunk_info[(size_t)bh * a.max_chunks + chunk];
     const uint32_t slot0 = info.x, quota = info.y;
     const uint32_t sstar = (uint32_t)a.sstar[bh];
@@ -104,12 +105,12 @@ __global__ void __launch_bounds__(kCpThreads) k_compact(CompactArgs a)
     }
     if (tid == kCpThreads - 1 && (int64_t)slot > room)
         devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, (long long)slot0);
+    pdl_trigger();
 }
 
 cudaError_t launch_compact(const CompactArgs &a, int nchunks, int bh, cudaStream_t s)
 {
-    k_compact<<<dim3(nchunks, bh), kCpThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k_compact, dim3(nchunks, bh), dim3(kCpThreads), 0, s, a);
 }
 
 }  // namespace pk

@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
         s_m[tid] = -INFINITY;
         s_l[tid] = 0.0f;
     }
+    pdl_wait();                                   // the selected ids may come from the search
     const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + (size_t)bh * a.stride * row_bytes;
     const unsigned char *Vb = reinterpret_cast<const unsigned char *>(a.V) + (size_t)bh * a.stride * row_bytes;
     const int d = tid & (kD - 1);
@@ -196,13 +197,15 @@ cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s)
     cfg.blockDim = dim3(kAtThreads, 1, 1);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = a.nsplit;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, k_gather_attend, a);
 }
 

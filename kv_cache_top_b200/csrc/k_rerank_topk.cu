@@ -8,11 +8,13 @@
 //
 // Work is split by candidate slices (not key ranges), so every CTA reranks
 // the same number of records wherever the candidates sit.  A CTA stages its
-// candidate ids in shared memory; eight lanes share a record (one coalesced
-// 128-byte load, 16 bytes per lane) and after one pair exchange each lane
-// owns two blocks (16 coordinates) with their weights.  The signed level of a
-// nibble comes from a 16-entry shared table (at most 16 distinct words per
-// request: no bank conflicts); q~ stays in registers.
+// candidate ids in shared memory; four lanes share a record, each loading one
+// 32-byte group (the nibbles of 4 blocks and their 4 weights) and decoding
+// its 32 coordinates with no exchange.  The signed level of a nibble comes
+// from a 16-entry shared table (at most 16 distinct words per request: no
+// bank conflicts), addressed by one byte permute per coordinate; q~ stays in
+// registers.  The kernel is issue-bound, so the layout minimises instructions
+// per record.
 //
 // Scores never leave the chip: the CTA turns (score, id) into 64-bit keys
 // ordered by score desc then id asc and radix-selects its Top-k set; a merge
@@ -299,16 +301,25 @@ __device__ __forceinline__ u64 make_key(float est, int32_t idx)
     return ((u64)ord_f32(__fadd_rn(est, 0.0f)) << 32) | (u64)(0xffffffffu - (uint32_t)idx);
 }
 
-// dot of one block's 8 nibbles (one u32) with 8 coordinates of q~
+// dot of one block's 8 nibbles (one u32: byte i holds coordinates 2i, 2i+1)
+// with 8 coordinates of q~.  lo/hi hold 4 x the low/high nibble of every byte,
+// i.e. the byte offsets of the signed levels in the 16-entry table; one byte
+// permute per coordinate then yields the address.
 __device__ __forceinline__ float block_dot(const float *slev, uint32_t nib, const float *q)
 {
+    const uint32_t lo = (nib << 2) & 0x3c3c3c3cu, hi = (nib >> 2) & 0x3c3c3c3cu;
+    const char *base = reinterpret_cast<const char *>(slev);
     float d = 0.0f;
 #pragma unroll
-    for (int jj = 0; jj < 8; jj++) d = fmaf(slev[(nib >> (4 * jj)) & 0xfu], q[jj], d);
+    for (int i = 0; i < 4; i++) {
+        const uint32_t o0 = __byte_perm(lo, 0u, 0x4440u + i), o1 = __byte_perm(hi, 0u, 0x4440u + i);
+        d = fmaf(*reinterpret_cast<const float *>(base + o0), q[2 * i], d);
+        d = fmaf(*reinterpret_cast<const float *>(base + o1), q[2 * i + 1], d);
+    }
     return d;
 }
 
-__global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
+__global__ void __launch_bounds__(kRrThreads, 4) k_rerank_topk(RerankArgs a)
 {
     extern __shared__ __align__(16) unsigned char s_dyn[];
     __shared__ RrShared sm;
@@ -321,45 +332,41 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
     const int count = (int)min((int64_t)a.slice, a.C - m0);
 
     if (tid < 16) sm.slev[tid] = (tid & 8) ? -a.lv.lev[tid & 7] : a.lv.lev[tid & 7];
+    pdl_wait();                                   // candidates come from the compaction
     const int32_t *cand = a.cand + (size_t)bh * a.stride + m0;
     for (int i = tid; i < count; i += kRrThreads) ids[i] = cand[i];
-    const int q8 = lane & 7, sub = lane >> 3;          // 16-byte piece of the record, record of the warp step
-    float qr[16];
+    const int q4 = lane & 3, sub = lane >> 2;          // 32-byte group of the record, record of the round
+    float qr[32];
 #pragma unroll
-    for (int i = 0; i < 16; i++) qr[i] = a.qt[(size_t)bh * kD + 16 * q8 + i];
+    for (int i = 0; i < 32; i++) qr[i] = a.qt[(size_t)bh * kD + 32 * q4 + i];
     const float qnorm = a.qnorm[bh];
-    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes;
+    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes + 32 * q4;
     float *dest = a.dbg_est ? a.dbg_est + (size_t)bh * a.C + m0 : nullptr;
     __syncthreads();
 
-    // each warp step: 16 records, one coalesced 16-byte load per lane per record
-    const bool odd = (q8 & 1) != 0;
+    // each warp step: 16 records in two rounds of 8; lane (record, group) loads
+    // the group's 16 B of nibbles and 16 B of weights
     for (int r0 = warp * 16; r0 < count; r0 += kRrWarps * 16) {
-        uint4 v[4];
-        int32_t id[4];
+        uint4 nv[2], wv[2];
+        int32_t id[2];
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const int r = r0 + 4 * u + sub;
+        for (int u = 0; u < 2; u++) {
+            const int r = r0 + 8 * u + sub;
             id[u] = ids[r < count ? r : 0];
-            v[u] = __ldg(reinterpret_cast<const uint4 *>(rec + (size_t)id[u] * kRecBytes) + q8);
+            const uint4 *p = reinterpret_cast<const uint4 *>(rec + (size_t)id[u] * kRecBytes);
+            nv[u] = __ldg(p);
+            wv[u] = __ldg(p + 1);
         }
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            // even lane of a pair: nibble words of blocks 4g..4g+3; odd lane: their
-            // weights.  Swap halves so lane q8 owns blocks 2 q8, 2 q8 + 1.
-            const uint32_t r0v = __shfl_xor_sync(kFull, odd ? v[u].x : v[u].z, 1);
-            const uint32_t r1v = __shfl_xor_sync(kFull, odd ? v[u].y : v[u].w, 1);
-            const uint32_t nib0 = odd ? r0v : v[u].x, nib1 = odd ? r1v : v[u].y;
-            const float w0 = __uint_as_float(odd ? v[u].z : r0v);
-            const float w1 = __uint_as_float(odd ? v[u].w : r1v);
-            const float d0 = block_dot(sm.slev, nib0, qr);
-            const float d1 = block_dot(sm.slev, nib1, qr + 8);
-            float part = fmaf(w0, d0, w1 * d1);
+        for (int u = 0; u < 2; u++) {
+            float part = __uint_as_float(wv[u].x) * block_dot(sm.slev, nv[u].x, qr);
+            part = fmaf(__uint_as_float(wv[u].y), block_dot(sm.slev, nv[u].y, qr + 8), part);
+            part = fmaf(__uint_as_float(wv[u].z), block_dot(sm.slev, nv[u].z, qr + 16), part);
+            part = fmaf(__uint_as_float(wv[u].w), block_dot(sm.slev, nv[u].w, qr + 24), part);
             part += __shfl_xor_sync(kFull, part, 1);
             part += __shfl_xor_sync(kFull, part, 2);
-            part += __shfl_xor_sync(kFull, part, 4);
-            const int r = r0 + 4 * u + sub;
-            if (q8 == 0 && r < count) {
+            const int r = r0 + 8 * u + sub;
+            if (q4 == 0 && r < count) {
                 const float est = qnorm * part;
                 keys[r] = make_key(est, id[u]);
                 if (dest) dest[r] = est;
@@ -378,6 +385,7 @@ __global__ void __launch_bounds__(kRrThreads) k_rerank_topk(RerankArgs a)
     }
     u64 *part = a.partial + ((size_t)bh * a.max_slices + sl) * a.topk_cap;
     for (int i = tid; i < k; i += kRrThreads) part[i] = (i < have) ? sm.tmp[i] : 0ull;
+    pdl_trigger();
 }
 
 // Merge of the per-slice Top-k sets of one pair into its final sorted Top-k.
@@ -396,6 +404,7 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
     const int cap = a.cap;                     // keys[] capacity (>= 2k)
     int cnt = 0;
     u64 tau = 0ull;
+    pdl_wait();                                   // per-slice sets come from the rerank
     const int64_t total = (int64_t)a.nslices * k;
     for (int64_t e0 = 0; e0 < total; e0 += cap - k) {
         const int64_t e1 = min(total, e0 + (cap - k));
@@ -443,6 +452,7 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
         a.out_idx[(size_t)bh * k + i] = live ? (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu)) : -1;
         if (a.out_score) a.out_score[(size_t)bh * k + i] = live ? unord_f32((uint32_t)(x >> 32)) : 0.0f;
     }
+    pdl_trigger();
 }
 
 size_t merge_smem(int cap) { return (size_t)cap * sizeof(u64); }
@@ -457,8 +467,7 @@ cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s)
         if (e != cudaSuccess) return e;
         attr_max = (int)merge_smem(kMergeCap);
     }
-    k_topk_merge<<<bh, kRrThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k_topk_merge, dim3(bh), dim3(kRrThreads), smem, s, a);
 }
 
 size_t rerank_smem(int slice) { return (size_t)slice * (sizeof(u64) + sizeof(int32_t)); }
@@ -473,8 +482,7 @@ cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s)
         if (e != cudaSuccess) return e;
         attr_max = (int)rerank_smem(kMaxSlice);
     }
-    k_rerank_topk<<<dim3(a.nslices, bh), kRrThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k_rerank_topk, dim3(a.nslices, bh), dim3(kRrThreads), smem, s, a);
 }
 
 }  // namespace pk

@@ -153,6 +153,14 @@ __device__ __forceinline__ float unord_f32(uint32_t k)
     return __uint_as_float(u);
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while its predecessor finishes; it must wait here
+// before touching the predecessor's outputs (a no-op for ordinary launches).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the dependent grid launch once every CTA of this grid has called this
+// (or exited); called after a CTA's main work.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Record a device-check failure (first writer wins) without trapping.
 __device__ __forceinline__ void devchk(int32_t *err, long long *detail, int32_t code, long long v)
 {
@@ -256,6 +264,24 @@ cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s);
 size_t rerank_smem(int slice);
+
+// Launch with programmatic stream serialisation (the kernel calls pdl_wait()
+// before reading what earlier kernels of the stream wrote).
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
 // host-side Lloyd-Max levels of the magnitude prior (closed-form integrals)
 int lloyd_max_levels(int m, int L, double *lev, double *thr);
 }  // namespace pk
