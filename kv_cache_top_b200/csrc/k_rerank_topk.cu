@@ -8,9 +8,11 @@
 //
 // Work is split by candidate slices (not key ranges), so every CTA reranks
 // the same number of records wherever the candidates sit.  A CTA stages its
-// candidate ids in shared memory; four lanes share a record, each loading one
-// 32-byte group (the nibbles of 4 blocks and their 4 weights) and decoding
-// its 32 coordinates with no exchange.  The signed level of a nibble comes
+// candidate ids in shared memory; each warp streams its records into a
+// private multi-stage shared-memory ring with asynchronous 16-byte copies
+// (several stages in flight per warp, no registers held), and four lanes
+// decode a record, each taking one 32-byte group (the nibbles of 4 blocks and
+// their 4 weights, 32 coordinates) with no exchange.  The signed level of a nibble comes
 // from a 16-entry shared table (at most 16 distinct words per request: no
 // bank conflicts), addressed by one byte permute per coordinate; q~ stays in
 // registers.  The kernel is issue-bound, so the layout minimises instructions
@@ -319,12 +321,28 @@ __device__ __forceinline__ float block_dot(const float *slev, uint32_t nib, cons
     return d;
 }
 
-__global__ void __launch_bounds__(kRrThreads, 4) k_rerank_topk(RerankArgs a)
+// 16-byte asynchronous global -> shared copy (L2 only, no register staging)
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+constexpr int kRrStages = 3;                       // per-warp pipeline depth
+constexpr int kRrStep = 16;                        // records per warp stage
+constexpr int kRecPad = 144;                       // shared-memory record stride (conflict-free)
+constexpr size_t kRrRingBytes = (size_t)kRrWarps * kRrStages * kRrStep * kRecPad;
+
+__global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
 {
     extern __shared__ __align__(16) unsigned char s_dyn[];
     __shared__ RrShared sm;
-    u64 *keys = reinterpret_cast<u64 *>(s_dyn);                         // [slice]
-    int32_t *ids = reinterpret_cast<int32_t *>(s_dyn + (size_t)a.slice * sizeof(u64));
+    unsigned char *ring_all = s_dyn;                                   // [warps][stages][16][144]
+    u64 *keys = reinterpret_cast<u64 *>(s_dyn + kRrRingBytes);         // [slice]
+    int32_t *ids = reinterpret_cast<int32_t *>(s_dyn + kRrRingBytes + (size_t)a.slice * sizeof(u64));
     const int bh = blockIdx.y, sl = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.topk;
@@ -340,39 +358,63 @@ __global__ void __launch_bounds__(kRrThreads, 4) k_rerank_topk(RerankArgs a)
 #pragma unroll
     for (int i = 0; i < 32; i++) qr[i] = a.qt[(size_t)bh * kD + 32 * q4 + i];
     const float qnorm = a.qnorm[bh];
-    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes + 32 * q4;
+    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes;
     float *dest = a.dbg_est ? a.dbg_est + (size_t)bh * a.C + m0 : nullptr;
     __syncthreads();
 
-    // each warp step: 16 records in two rounds of 8; lane (record, group) loads
-    // the group's 16 B of nibbles and 16 B of weights
-    for (int r0 = warp * 16; r0 < count; r0 += kRrWarps * 16) {
-        uint4 nv[2], wv[2];
-        int32_t id[2];
+    // Each warp streams its own records (warp w takes steps w, w + 8, ...,
+    // 16 records per step) through a private ring of kRrStages shared-memory
+    // stages: the copies of the next stages are in flight while one stage is
+    // decoded.  Copies are coalesced: lane l moves 16-byte pieces l, l+32,
+    // l+64, l+96 of the step's 2 KB.
+    unsigned char *ring = ring_all + (size_t)warp * kRrStages * kRrStep * kRecPad;
+    const int nsteps = (count + kRrStep - 1) / kRrStep;
+    auto issue = [&](int step_local, int stage) {
+        const int r0 = (warp + step_local * kRrWarps) * kRrStep;
+        if (r0 < count) {
 #pragma unroll
-        for (int u = 0; u < 2; u++) {
-            const int r = r0 + 8 * u + sub;
-            id[u] = ids[r < count ? r : 0];
-            const uint4 *p = reinterpret_cast<const uint4 *>(rec + (size_t)id[u] * kRecBytes);
-            nv[u] = __ldg(p);
-            wv[u] = __ldg(p + 1);
+            for (int u = 0; u < 4; u++) {
+                const int piece = lane + 32 * u;
+                const int j = piece >> 3, c = piece & 7;
+                const int r = r0 + j;
+                const int32_t id = ids[r < count ? r : 0];
+                cp_async16(ring + ((size_t)stage * kRrStep + j) * kRecPad + 16 * c,
+                           rec + (size_t)id * kRecBytes + 16 * c);
+            }
         }
+        cp_async_commit();                            // always one group per call
+    };
+    const int my_steps = (nsteps > warp) ? (nsteps - warp + kRrWarps - 1) / kRrWarps : 0;
+#pragma unroll
+    for (int s = 0; s < kRrStages - 1; s++) issue(s, s);
+    for (int t = 0; t < my_steps; t++) {
+        cp_async_wait<kRrStages - 2>();               // step t has landed (this lane's pieces)
+        __syncwarp();                                 // ... and every lane's
+        const int stage = t % kRrStages;
+        const int r0 = (warp + t * kRrWarps) * kRrStep;
+        const unsigned char *st = ring + (size_t)stage * kRrStep * kRecPad;
 #pragma unroll
         for (int u = 0; u < 2; u++) {
-            float part = __uint_as_float(wv[u].x) * block_dot(sm.slev, nv[u].x, qr);
-            part = fmaf(__uint_as_float(wv[u].y), block_dot(sm.slev, nv[u].y, qr + 8), part);
-            part = fmaf(__uint_as_float(wv[u].z), block_dot(sm.slev, nv[u].z, qr + 16), part);
-            part = fmaf(__uint_as_float(wv[u].w), block_dot(sm.slev, nv[u].w, qr + 24), part);
+            const int j = 8 * u + sub;
+            const uint4 *p = reinterpret_cast<const uint4 *>(st + (size_t)j * kRecPad + 32 * q4);
+            const uint4 nv = p[0], wv = p[1];
+            float part = __uint_as_float(wv.x) * block_dot(sm.slev, nv.x, qr);
+            part = fmaf(__uint_as_float(wv.y), block_dot(sm.slev, nv.y, qr + 8), part);
+            part = fmaf(__uint_as_float(wv.z), block_dot(sm.slev, nv.z, qr + 16), part);
+            part = fmaf(__uint_as_float(wv.w), block_dot(sm.slev, nv.w, qr + 24), part);
             part += __shfl_xor_sync(kFull, part, 1);
             part += __shfl_xor_sync(kFull, part, 2);
-            const int r = r0 + 8 * u + sub;
+            const int r = r0 + j;
             if (q4 == 0 && r < count) {
                 const float est = qnorm * part;
-                keys[r] = make_key(est, id[u]);
+                keys[r] = make_key(est, ids[r]);
                 if (dest) dest[r] = est;
             }
         }
+        __syncwarp();                                 // stage consumed before it is refilled
+        issue(t + kRrStages - 1, (t + kRrStages - 1) % kRrStages);
     }
+    cp_async_wait<0>();
     __syncthreads();
 
     // ---- Top-k set of the slice (unordered) and its smallest key
@@ -470,7 +512,7 @@ cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s)
     return launch_pdl(k_topk_merge, dim3(bh), dim3(kRrThreads), smem, s, a);
 }
 
-size_t rerank_smem(int slice) { return (size_t)slice * (sizeof(u64) + sizeof(int32_t)); }
+size_t rerank_smem(int slice) { return kRrRingBytes + (size_t)slice * (sizeof(u64) + sizeof(int32_t)); }
 
 cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s)
 {

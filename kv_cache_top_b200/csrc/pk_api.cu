@@ -133,7 +133,7 @@ int32_t slice_lo(const pk_index *ix) { return std::max<int32_t>(256, 2 * ix->top
 
 void slicing(const pk_index *ix, int64_t C, int32_t *slice, int32_t *nslices)
 {
-    const int64_t target = 4 * (int64_t)ix->num_sms;
+    const int64_t target = 2 * (int64_t)ix->num_sms;
     int64_t sl = ceil_div(ceil_div(C * ix->bh, target), 64) * 64;
     sl = std::max<int64_t>(sl, slice_lo(ix));
     sl = std::min<int64_t>(sl, kMaxSlice);
@@ -505,7 +505,7 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(dalloc(&ix->sstar, BH));
     {   // largest slice count any C <= n_cap can need
         const int64_t lo = slice_lo(ix);
-        const int64_t by_target = ceil_div(4 * (int64_t)ix->num_sms, ix->bh) + 1;
+        const int64_t by_target = ceil_div(2 * (int64_t)ix->num_sms, ix->bh) + 1;
         ix->max_slices = (int32_t)std::max<int64_t>(std::min<int64_t>(ceil_div(n_cap, lo), by_target),
                                                     ceil_div(n_cap, kMaxSlice)) + 1;
     }
