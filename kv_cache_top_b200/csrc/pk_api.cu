@@ -117,12 +117,15 @@ uint64_t splitmix64(uint64_t x)
     return z ^ (z >> 31);
 }
 
+// Key chunks of the scan and the compaction: at most one wave (4 resident
+// CTAs per SM) when the chunk-size cap allows, never fewer than
+// ceil(n / kMaxChunk) chunks.
 void chunking(const pk_index *ix, int64_t n, int32_t *nchunks, int64_t *chunk)
 {
-    int64_t nch = ceil_div(4 * (int64_t)ix->num_sms, ix->bh);
-    nch = std::max<int64_t>(1, std::min<int64_t>(nch, ceil_div(n, kMinChunk)));
+    int64_t nch = std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / ix->bh);
+    nch = std::min<int64_t>(nch, ceil_div(n, kMinChunk));
     nch = std::max<int64_t>(nch, ceil_div(n, kMaxChunk));
-    nch = std::min<int64_t>(nch, ix->max_chunks);
+    nch = std::max<int64_t>(1, std::min<int64_t>(nch, ix->max_chunks));
     int64_t ch = ceil_div(ceil_div(n, nch), 16) * 16;
     *chunk = ch;
     *nchunks = (int32_t)ceil_div(n, ch);
@@ -133,8 +136,10 @@ int32_t slice_lo(const pk_index *ix) { return std::max<int32_t>(256, 2 * ix->top
 
 void slicing(const pk_index *ix, int64_t C, int32_t *slice, int32_t *nslices)
 {
-    const int64_t target = 2 * (int64_t)ix->num_sms;
-    int64_t sl = ceil_div(ceil_div(C * ix->bh, target), 64) * 64;
+    // at most one wave (2 resident CTAs per SM) unless the slice-size cap forces more
+    int64_t ns = std::max<int64_t>(1, (2 * (int64_t)ix->num_sms) / ix->bh);
+    ns = std::max<int64_t>(ns, ceil_div(C, kMaxSlice));
+    int64_t sl = ceil_div(ceil_div(C, ns), 64) * 64;
     sl = std::max<int64_t>(sl, slice_lo(ix));
     sl = std::min<int64_t>(sl, kMaxSlice);
     *slice = (int32_t)sl;
@@ -469,7 +474,7 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
         delete ix;
         return cuda_status(e);
     }
-    ix->max_chunks = (int32_t)std::max<int64_t>(ceil_div(4 * (int64_t)ix->num_sms, ix->bh),
+    ix->max_chunks = (int32_t)std::max<int64_t>(std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / ix->bh),
                                                 ceil_div(n_cap, kMaxChunk) + 1);
 
     // SRHT sign diagonal and scale; Lloyd-Max levels
@@ -505,7 +510,7 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(dalloc(&ix->sstar, BH));
     {   // largest slice count any C <= n_cap can need
         const int64_t lo = slice_lo(ix);
-        const int64_t by_target = ceil_div(2 * (int64_t)ix->num_sms, ix->bh) + 1;
+        const int64_t by_target = std::max<int64_t>(1, (2 * (int64_t)ix->num_sms) / ix->bh);
         ix->max_slices = (int32_t)std::max<int64_t>(std::min<int64_t>(ceil_div(n_cap, lo), by_target),
                                                     ceil_div(n_cap, kMaxSlice)) + 1;
     }
