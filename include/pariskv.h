@@ -199,6 +199,31 @@ pk_status pk_magnitude_levels(int32_t m, int32_t L, float *levels, float *thresh
 pk_status pk_resolve(int64_t n, int64_t cand_budget, float collision_ratio, int32_t topk,
                      int64_t *C, int64_t *R);
 
+/* Candidate selection that allocates nothing.  (No counterpart on the pages:
+ * it is a deployment aid for the candidate step of pk_search.)
+ *
+ * For callers that cannot allocate device memory at the moment they need a
+ * candidate set -- code recorded into a CUDA graph (cudaMalloc cannot be
+ * captured), serving runtimes whose memory pool is fully reserved up front,
+ * or decode threads that must not take allocator locks -- this computes, from
+ * one row of collision scores, the same Top-C candidate ids in the same
+ * ascending order as the candidate step of pk_search (higher score first,
+ * then lower id; ids written in ascending order).
+ *   S     [n] u8 device (or pinned host) scores; scores from pk_search_debug
+ *         lie in [0, 96]; any byte value is accepted.
+ *   n     1 <= n <= 4,194,304 (PK_ERR_CAPACITY above that; nothing runs).
+ *   C     1 <= C <= n.
+ *   cand  [C] i32 device, 4-byte aligned: the candidate ids.
+ * Scratch: a static device array of 266,496 bytes that every GPU loading the
+ * library holds until the process exits; no cudaMalloc, cudaFree or other
+ * allocating call is made.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current, so make it
+ * once before any stream capture.  All calls share the array: calls whose
+ * work overlaps on the GPU (different streams or host threads) race on it;
+ * calls on one stream are ordered and safe.  Asynchronous on `stream`. */
+pk_status pk_select_candidates_noalloc(const uint8_t *S, int64_t n, int64_t C, int32_t *cand,
+                                       void *stream);
+
 /* Per-kernel timing.  While tracing is on, the library records a CUDA event
  * pair on the launching stream around each of its kernels.  pk_trace_read
  * synchronises, then returns per kernel kind (0 encode, 1 query_prep,

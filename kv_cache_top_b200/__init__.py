@@ -21,7 +21,7 @@ __all__ = [
     "PkError", "pk_default_params", "pk_build_index", "pk_append", "pk_search", "pk_search_debug",
     "pk_attend", "pk_free", "pk_status_str", "pk_last_device_error", "pk_get_info",
     "pk_export_index", "pk_magnitude_levels", "pk_resolve", "pk_trace_enable", "pk_trace_read",
-    "pk_params", "pk_info", "pk_debug_out", "PK_F32", "PK_BF16", "PK_KV_DEVICE",
+    "pk_select_candidates_noalloc", "pk_params", "pk_info", "pk_debug_out", "PK_F32", "PK_BF16", "PK_KV_DEVICE",
     "PK_KV_HOST_PINNED", "KERNELS", "lib",
 ]
 
@@ -146,3 +146,10 @@ def pk_trace_read(index):
     ms = np.zeros(len(KERNELS), np.float64)
     _check(lib.pk_trace_read(index, n.ctypes.data, ms.ctypes.data), "pk_trace_read")
     return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(KERNELS)}
+
+
+def pk_select_candidates_noalloc(S, n: int, C: int, cand, stream=None):
+    """Top-C candidate ids of one score row with no device allocation (see
+    include/pariskv.h): for callers that cannot allocate at that moment."""
+    _check(lib.pk_select_candidates_noalloc(_ptr(S), int(n), int(C), _ptr(cand), _stream(stream)),
+           "pk_select_candidates_noalloc")

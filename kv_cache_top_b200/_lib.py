@@ -15,6 +15,7 @@ EXPORTS = (
     "pk_default_params", "pk_build_index", "pk_append", "pk_search", "pk_search_debug",
     "pk_attend", "pk_free", "pk_status_str", "pk_last_device_error", "pk_get_info",
     "pk_export_index", "pk_magnitude_levels", "pk_resolve", "pk_trace_enable", "pk_trace_read",
+    "pk_select_candidates_noalloc",
 )
 
 PK_OK, PK_ERR_INVALID_ARG, PK_ERR_CAPACITY, PK_ERR_OOM, PK_ERR_CUDA, PK_ERR_TIMEOUT, \
@@ -89,4 +90,6 @@ def load() -> C.CDLL:
     lib.pk_trace_enable.argtypes = [P, I32]
     lib.pk_trace_read.restype = st
     lib.pk_trace_read.argtypes = [P, P, P]
+    lib.pk_select_candidates_noalloc.restype = st
+    lib.pk_select_candidates_noalloc.argtypes = [P, I64, I64, P, P]
     return lib
