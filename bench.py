@@ -69,6 +69,25 @@ def dist_env():
         int(os.environ.get("LOCAL_RANK", 0))
 
 
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of per-rank timings (one all-reduce, every rank calls
+    it in the same order).  At world == 1 the values come back unchanged."""
+    vals = [float(v) for v in values]
+    if world <= 1:
+        return vals
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time (weak scaling: each rank owns the same amount of work)."""
+    return units_per_rank * world / (ms_max / 1000.0)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -292,18 +311,20 @@ def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
             i_host.copy_(idx, non_blocking=True)
             evs[i][1].record(stream)
         torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in evs) / ks
-        e2e = {"value": 1000.0 / e2e_ms, "unit": "steps/s", "ms_per_step": e2e_ms,
+        e2e_ms = sum(a.elapsed_time(b) for a, b in evs)
+        e2e = {"steps": ks, "ms_total": e2e_ms,
                "h2d_bytes_per_step": q_dev.numel() * q_dev.element_size(),
                "d2h_bytes_per_step": out.numel() * 4 + idx.numel() * 4}
 
     clocks = sampler.stop() if rank == 0 else None
 
-    # max over ranks of the device time
-    if world > 1:
-        t = torch.tensor([ms_clean], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_clean = float(t.item())
+    # max over ranks of the device times (every rank takes the same step)
+    ms_clean, e2e_max = max_over_ranks([ms_clean, e2e["ms_total"] if e2e else 0.0], world, dev)
+    if e2e:
+        e2e = {"value": job_rate(e2e["steps"], world, e2e_max), "unit": "steps/s",
+               "ms_per_step": e2e_max / e2e["steps"],
+               "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+               "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
 
     res = dict(ms_total=ms_clean, wall=wall_clean, kern=kern, recall=recall, C=C, R=R, info=info,
                e2e=e2e, clocks=clocks, ms_traced=ms_traced)
@@ -429,7 +450,7 @@ def main():
         km = kernel_table(rm["kern"], margs.steps, wl_m, rm["C"], peak)
         link_bytes = wl_m["batch"] * wl_m["H"] * 100 * 2 * 128 * 2
         att = km.get("gather_attend", {})
-        mil = {"workload": wl_m["name"], "steps_s": margs.steps * world / (rm["ms_total"] / 1000.0),
+        mil = {"workload": wl_m["name"], "steps_s": job_rate(margs.steps, world, rm["ms_total"]),
                "ms_per_step": rm["ms_total"] / margs.steps, "steps": margs.steps,
                "search_us": sum(km[k]["avg_us"] for k in ("query_prep", "collision_scan", "compact", "rerank_topk",
                                           "topk_merge")
@@ -442,8 +463,6 @@ def main():
                if att and rm.get("h2d_gbs") else None,
                "kernels": km, "cand_budget": rm["C"], "collision_budget": rm["R"],
                "cpu_baseline": rm.get("cpu")}
-        if world > 1:
-            pass
 
     if world > 1:
         torch.distributed.barrier()
@@ -456,7 +475,7 @@ def main():
     dom = max(km, key=lambda k: km[k]["share"])
     step_bytes = sum(alg_bytes(k, wl, res["C"]) for k in km)
     ms_per_step = res["ms_total"] / args.steps
-    value = args.steps * world / (res["ms_total"] / 1000.0)
+    value = job_rate(args.steps, world, res["ms_total"])
     line = {
         "metric": METRIC,
         "value": value,
