@@ -14,13 +14,14 @@
 // Hot loop: 16 B of codes per key read with 128-bit streaming loads; the 16
 // bonus tables (4 bits x 256 centres = one 32-bit register per lane per
 // block) live in registers and are read with warp shuffles, which have no
-// bank conflicts whatever the codes are.  Lane l's word of block b holds in
-// nibble t the bonus of centre 32 t + l, so a code byte c is used as it is:
-// its low 5 bits pick the lane (the shuffle ignores higher bits), and
-// 4 (c >> 5) -- all four computed at once per 32-bit code word -- is the
-// shift of a wrap-mode funnel shift (which ignores bits above 4).  Two
-// extracted bonuses (each <= 6) are added before one mask, since their sum
-// still fits in the low nibble.
+// bank conflicts whatever the codes are.  Lane l's word of block b holds the
+// bonus of centre 32 t + l in the 4 bits starting at bit 4 t + r(l), rotated
+// by r(l) = (l >> 3) & 3, so a code byte c is used as it is: its low 5 bits
+// pick the lane (the shuffle ignores higher bits), and bits 3..7 of c, i.e.
+// 4 (c >> 5) + r(c & 31), are exactly the rotate amount that brings the
+// bonus to bit 0 (a wrap-mode funnel shift ignores bits above 4) -- one shift
+// of the code word per code.  Two extracted bonuses (each <= 6) are added
+// before one mask, since their sum still fits in the low nibble.
 #include "pk_internal.cuh"
 
 namespace pk {
@@ -36,15 +37,14 @@ __device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], u
 #pragma unroll
     for (int q = 0; q < 4; q++) {
         const uint32_t w = wds[q];
-        const uint32_t A = (w >> 3) & 0x1c1c1c1cu;      // byte k: 4 * (c_k >> 5)
         const uint32_t v0 = __shfl_sync(kFull, tab[4 * q + 0], (int)w);
         const uint32_t v1 = __shfl_sync(kFull, tab[4 * q + 1], (int)(w >> 8));
         const uint32_t v2 = __shfl_sync(kFull, tab[4 * q + 2], (int)(w >> 16));
         const uint32_t v3 = __shfl_sync(kFull, tab[4 * q + 3], (int)(w >> 24));
-        const uint32_t x0 = __funnelshift_r(v0, 0u, A);
-        const uint32_t x1 = __funnelshift_r(v1, 0u, A >> 8);
-        const uint32_t x2 = __funnelshift_r(v2, 0u, A >> 16);
-        const uint32_t x3 = __funnelshift_r(v3, 0u, A >> 24);
+        const uint32_t x0 = __funnelshift_r(v0, v0, w >> 3);
+        const uint32_t x1 = __funnelshift_r(v1, v1, w >> 11);
+        const uint32_t x2 = __funnelshift_r(v2, v2, w >> 19);
+        const uint32_t x3 = __funnelshift_r(v3, v3, w >> 27);
         s += ((x0 + x1) & 0xfu) + ((x2 + x3) & 0xfu);
     }
     return s;

@@ -11,134 +11,190 @@
 //     better-ranked buckets (from the occupancy table), and a bucket inside
 //     the top-rho fraction (P(c) < R = ceil(rho n)) gets bonus 6 - floor(6P/R).
 //
-// Grid (16 blocks, pairs), one warp per CTA: the warp rotates the query, ranks
-// the 256 centres of its block with a register bitonic sort (8 keys per lane,
-// shuffles only, no block barriers), scans the bucket sizes in rank order and
-// packs the bonus table 4 bits per centre in the layout the collision scan
-// keeps in registers -- lane l's word holds, in nibble t, the bonus of centre
-// 32 t + l.
+// Grid (8, pairs): a CTA of 256 threads takes 2 blocks, one 128-thread half
+// per block.  The kernel is a latency chain, so its steps are laid out for a
+// short critical path with little repeated work: every global load is issued
+// up front (no load waits on another), warp 0 aggregates and rotates the
+// query once and shares it through shared memory, each half ranks the 256
+// centres of its block by a bitonic sort holding 2 keys per thread (shuffles
+// inside a warp; shared memory for the 3 stages that cross warps), a scan
+// over the half turns bucket sizes in rank order into P(c), and one warp per
+// half packs the bonus table 4 bits per centre in the layout the collision
+// scan keeps in registers -- lane l's word holds the bonus of centre 32 t + l
+// in the 4 bits starting at bit (4 t + r(l)) mod 32, r(l) = (l >> 3) & 3.
 #include "pk_internal.cuh"
 
 namespace pk {
 
-__global__ void __launch_bounds__(32) k_query_prep(PrepArgs a)
-{
-    const int b = blockIdx.x, bh = blockIdx.y;
-    const int lane = threadIdx.x;
-    const int b_seq = bh / a.H, h = bh - b_seq * a.H;
-    __shared__ uint8_t s_bonus[kNC];
+constexpr int kQpHalf = 128;                  // threads per block of centres
+constexpr int kQpBlocks = 2;                  // blocks per CTA
+constexpr int kQpThreads = kQpHalf * kQpBlocks;
+constexpr int kQpWarps = kQpThreads / 32;
 
-    if (b == 0) {   // reset the per-call counters of the collision scan and the rerank
-        for (int i = lane; i < kBins; i += 32) a.head_hist[(size_t)bh * kBins + i] = 0u;
-        if (lane < 2) a.tickets[(size_t)bh * 2 + lane] = 0u;
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ void load_heads(float (&qv)[4][kMaxGroup], const T *qp, int G, int lane)
+{
+#pragma unroll
+    for (int r = 0; r < 4; r++)
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; g++) {
+            const int gg = g < G ? g : G - 1;          // in bounds; unused when g >= G
+            qv[r][g] = to_f32(qp[lane + 32 * r + gg * kD]);
+        }
+}
+
+__device__ __forceinline__ uint32_t tier_bonus(uint32_t P, unsigned long long R)
+{
+    // 6 - floor(6P/R) for P < R, else 0: floor(6P/R) = #{j = 1..5 : 6P >= jR},
+    // exact in integers without a division
+    if ((unsigned long long)P >= R) return 0u;
+    const unsigned long long p6 = 6ull * P;
+    return 6u - (uint32_t)(p6 >= R) - (uint32_t)(p6 >= 2 * R) - (uint32_t)(p6 >= 3 * R) -
+           (uint32_t)(p6 >= 4 * R) - (uint32_t)(p6 >= 5 * R);
+}
+
+__global__ void __launch_bounds__(kQpThreads) k_query_prep(PrepArgs a)
+{
+    typedef unsigned long long u64;
+    const int bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int half = tid / kQpHalf, t = tid % kQpHalf;      // t: thread within the half
+    const int b = kQpBlocks * blockIdx.x + half;             // this half's block
+    const int b_seq = bh / a.H, h = bh - b_seq * a.H;
+    __shared__ uint32_t s_occ[kQpBlocks][kNC];
+    __shared__ u64 s_key[2][kQpBlocks][kNC];
+    __shared__ float s_x[kD];
+    __shared__ uint32_t s_ws[kQpWarps];
+    __shared__ uint8_t s_bonus[kQpBlocks][kNC];
+
+    if (blockIdx.x == 0) {   // reset the per-call counters of the collision scan and the rerank
+        for (int i = tid; i < kBins; i += kQpThreads) a.head_hist[(size_t)bh * kBins + i] = 0u;
+        if (tid < 2) a.tickets[(size_t)bh * 2 + tid] = 0u;
     }
-    float x[4];
-    {
+    // global loads: 2 bucket sizes per thread; warp 0 the G query heads
+    const uint32_t *occ = a.occ + ((size_t)bh * kB + b) * kNC;
+    const uint32_t o0 = occ[t], o1 = occ[t + kQpHalf];
+    if (warp == 0) {
+        float qv[4][kMaxGroup];
         const int64_t base = ((int64_t)b_seq * a.H * a.G + (int64_t)h * a.G) * kD;
+        if (a.is_bf16)
+            load_heads(qv, reinterpret_cast<const __nv_bfloat16 *>(a.q) + base, a.G, lane);
+        else
+            load_heads(qv, reinterpret_cast<const float *>(a.q) + base, a.G, lane);
+        float x[4];
 #pragma unroll
         for (int r = 0; r < 4; r++) {
-            const int64_t j = base + lane + 32 * r;
-            float acc = ld_as_f32(a.q, j, a.is_bf16);
-            for (int g = 1; g < a.G; g++) acc = __fadd_rn(acc, ld_as_f32(a.q, j + (int64_t)g * kD, a.is_bf16));
+            float acc = qv[r][0];
+#pragma unroll
+            for (int g = 1; g < kMaxGroup; g++)
+                if (g < a.G) acc = __fadd_rn(acc, qv[r][g]);
             x[r] = acc;
         }
-    }
-    const float nrm = warp_rotate128(x, a.rot, lane);
-    if (b == 0) {
+        const float nrm = warp_rotate128(x, a.rot, lane);
 #pragma unroll
-        for (int r = 0; r < 4; r++) {
-            a.qt[(size_t)bh * kD + lane + 32 * r] = x[r];
-            if (a.dbg_qt) a.dbg_qt[(size_t)bh * kD + lane + 32 * r] = x[r];
-        }
-        if (lane == 0) {
-            a.qnorm[bh] = nrm;
-            if (a.dbg_qnorm) a.dbg_qnorm[bh] = nrm;
+        for (int r = 0; r < 4; r++) s_x[lane + 32 * r] = x[r];
+        if (blockIdx.x == 0) {
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                a.qt[(size_t)bh * kD + lane + 32 * r] = x[r];
+                if (a.dbg_qt) a.dbg_qt[(size_t)bh * kD + lane + 32 * r] = x[r];
+            }
+            if (lane == 0) {
+                a.qnorm[bh] = nrm;
+                if (a.dbg_qnorm) a.dbg_qnorm[bh] = nrm;
+            }
         }
     }
-    // coordinates 8b..8b+7 live in register b/4 of lanes 8(b%4)..8(b%4)+7
+    s_occ[half][t] = o0;
+    s_occ[half][t + kQpHalf] = o1;
+    __syncthreads();
     float xq[kM];
-    {
-        float src = x[0];
 #pragma unroll
-        for (int r = 1; r < 4; r++) src = (b / 4 == r) ? x[r] : src;
-#pragma unroll
-        for (int j = 0; j < kM; j++) xq[j] = __shfl_sync(kFull, src, 8 * (b % 4) + j);
-    }
-    // element e = 8 lane + i starts as centre c = e; sort key (ascending order =
+    for (int j = 0; j < kM; j++) xq[j] = s_x[kM * b + j];
+    // element e = 2 t + i starts as centre c = e; sort key (ascending order =
     // rank order): high 32 bits = ~ord(L) (L desc), low 8 bits = c (c asc)
-    unsigned long long key[8];
+    u64 key[2];
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const int c = lane * 8 + i;
+    for (int i = 0; i < 2; i++) {
+        const int c = 2 * t + i;
         float L = 0.0f;
 #pragma unroll
         for (int j = 0; j < kM; j++) L = __fadd_rn(L, ((c >> j) & 1) ? -xq[j] : xq[j]);
         L = __fadd_rn(L, 0.0f);   // fold -0 into +0 so equal scores tie
-        key[i] = ((unsigned long long)(~ord_f32(L)) << 8) | (unsigned)c;
+        key[i] = ((u64)(~ord_f32(L)) << 8) | (unsigned)c;
     }
-    // bitonic sort, ascending, 256 elements over the warp
+    // bitonic sort, ascending, 256 elements over the half
+    int buf = 0;
 #pragma unroll
-    for (int k = 2; k <= 256; k <<= 1) {
+    for (int k = 2; k <= kNC; k <<= 1) {
 #pragma unroll
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
-            if (jj >= 8) {
-                const int lx = jj >> 3;
-#pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    const int e = lane * 8 + i;
-                    const unsigned long long o = __shfl_xor_sync(kFull, key[i], lx);
-                    const bool take_min = ((e & jj) == 0) == ((e & k) == 0);
-                    key[i] = take_min ? (o < key[i] ? o : key[i]) : (o > key[i] ? o : key[i]);
-                }
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j == 1) {                      // both elements in this thread
+                const bool up = ((2 * t) & k) == 0;
+                const u64 lo = key[0] < key[1] ? key[0] : key[1];
+                const u64 hi = key[0] < key[1] ? key[1] : key[0];
+                key[0] = up ? lo : hi;
+                key[1] = up ? hi : lo;
             } else {
+                u64 o[2];
+                if (j <= 32) {                 // partner thread t ^ (j/2), same warp
 #pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    if ((i & jj) == 0) {
-                        const int e = lane * 8 + i;
-                        const bool up = (e & k) == 0;
-                        const unsigned long long x0 = key[i], x1 = key[i ^ jj];
-                        const unsigned long long lo = x0 < x1 ? x0 : x1, hi = x0 < x1 ? x1 : x0;
-                        key[i] = up ? lo : hi;
-                        key[i ^ jj] = up ? hi : lo;
-                    }
+                    for (int i = 0; i < 2; i++) o[i] = __shfl_xor_sync(kFull, key[i], j >> 1);
+                } else {                       // partner in another warp of the half
+#pragma unroll
+                    for (int i = 0; i < 2; i++) s_key[buf][half][2 * t + i] = key[i];
+                    __syncthreads();
+#pragma unroll
+                    for (int i = 0; i < 2; i++) o[i] = s_key[buf][half][(2 * t + i) ^ j];
+                    buf ^= 1;
+                }
+#pragma unroll
+                for (int i = 0; i < 2; i++) {
+                    const int e = 2 * t + i;
+                    const bool take_min = ((e & j) == 0) == ((e & k) == 0);
+                    key[i] = take_min ? (o[i] < key[i] ? o[i] : key[i]) : (o[i] > key[i] ? o[i] : key[i]);
                 }
             }
         }
     }
-    // exclusive prefix of bucket sizes in rank order -> tier bonus
-    const uint32_t *occ = a.occ + ((size_t)bh * kB + b) * kNC;
-    uint32_t cnt[8], run = 0;
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        cnt[i] = occ[key[i] & 0xffu];
-        run += cnt[i];
-    }
-    uint32_t incl = run;
+    // exclusive prefix of bucket sizes in rank order (over the half) -> tier bonus
+    const int c0 = (int)(key[0] & 0xffu), c1 = (int)(key[1] & 0xffu);
+    const uint32_t n0 = s_occ[half][c0], n1 = s_occ[half][c1];   // visible: the sort passed barriers
+    uint32_t incl = n0 + n1;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const uint32_t y = __shfl_up_sync(kFull, incl, o);
         if (lane >= o) incl += y;
     }
-    uint32_t P = incl - run;
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-        const int c = (int)(key[i] & 0xffu);
-        uint32_t bon = 0;
-        if ((int64_t)P < a.R) bon = 6u - (uint32_t)((6ull * P) / (unsigned long long)a.R);
-        s_bonus[c] = (uint8_t)bon;
-        if (a.dbg_bonus) a.dbg_bonus[((size_t)bh * kB + b) * kNC + c] = (uint8_t)bon;
-        P += cnt[i];
+    if (lane == 31) s_ws[warp] = incl;
+    __syncthreads();
+    uint32_t P0 = incl - (n0 + n1);
+    for (int w = half * (kQpHalf / 32); w < warp; w++) P0 += s_ws[w];
+    const unsigned long long R = (unsigned long long)a.R;
+    const uint32_t bon0 = tier_bonus(P0, R), bon1 = tier_bonus(P0 + n0, R);
+    s_bonus[half][c0] = (uint8_t)bon0;
+    s_bonus[half][c1] = (uint8_t)bon1;
+    if (a.dbg_bonus) {
+        uint8_t *db = a.dbg_bonus + ((size_t)bh * kB + b) * kNC;
+        db[c0] = (uint8_t)bon0;
+        db[c1] = (uint8_t)bon1;
     }
-    __syncwarp();
-    uint32_t word = 0;
+    __syncthreads();
+    if (t < 32) {                              // first warp of each half
+        uint32_t word = 0;
 #pragma unroll
-    for (int t = 0; t < 8; t++) word |= (uint32_t)s_bonus[32 * t + lane] << (4 * t);
-    a.bonus_packed[((size_t)bh * kB + b) * 32 + lane] = word;
+        for (int tt = 0; tt < 8; tt++) word |= (uint32_t)s_bonus[half][32 * tt + lane] << (4 * tt);
+        const uint32_t rl = (uint32_t)(lane >> 3) & 3u;
+        a.bonus_packed[((size_t)bh * kB + b) * 32 + lane] = __funnelshift_l(word, word, rl);
+    }
 }
 
 cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s)
 {
-    k_query_prep<<<dim3(kB, a.bh), 32, 0, s>>>(a);
+    k_query_prep<<<dim3(kB / kQpBlocks, a.bh), kQpThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -303,6 +303,23 @@ __device__ __forceinline__ u64 make_key(float est, int32_t idx)
     return ((u64)ord_f32(__fadd_rn(est, 0.0f)) << 32) | (u64)(0xffffffffu - (uint32_t)idx);
 }
 
+// Descending rank of every key of v[0..m) (keys distinct): rank(x) =
+// #{y in v : y > x}.  Every thread walks the whole list in step (broadcast
+// shared-memory reads), so the pass costs m / blockDim compares per key and
+// no barrier; it sorts and selects at once for small m.
+template <typename Emit>
+__device__ __forceinline__ void rank_by_count(const u64 *v, int m, Emit emit)
+{
+    for (int i0 = 0; i0 < m; i0 += kRrThreads) {
+        const int i = i0 + (int)threadIdx.x;
+        const u64 x = (i < m) ? v[i] : ~0ull;
+        int r = 0;
+#pragma unroll 4
+        for (int j = 0; j < m; j++) r += (v[j] > x) ? 1 : 0;
+        if (i < m) emit(r, x);
+    }
+}
+
 // dot of one block's 8 nibbles (one u32: byte i holds coordinates 2i, 2i+1)
 // with 8 coordinates of q~.  lo/hi hold 4 x the low/high nibble of every byte,
 // i.e. the byte offsets of the signed levels in the 16-entry table; one byte
@@ -425,33 +442,74 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
         for (int i = tid; i < count; i += kRrThreads) sm.tmp[i] = keys[i];
         __syncthreads();
     }
+    // the slice's set, sorted descending (zeros pad a slice shorter than k)
     u64 *part = a.partial + ((size_t)bh * a.max_slices + sl) * a.topk_cap;
-    for (int i = tid; i < k; i += kRrThreads) part[i] = (i < have) ? sm.tmp[i] : 0ull;
+    rank_by_count(sm.tmp, have, [&](int r, u64 x) { part[r] = x; });
+    for (int i = have + tid; i < k; i += kRrThreads) part[i] = 0ull;
     pdl_trigger();
 }
 
-// Merge of the per-slice Top-k sets of one pair into its final sorted Top-k.
-// One CTA per pair holds as many partial keys as its shared memory allows
-// (all of them in the usual case) and radix-selects once; larger merges run
-// in rounds that keep the best k seen so far.  The final order (score desc,
-// id asc) is produced by one warp.
+// Merge of the per-slice Top-k lists of one pair into its final sorted
+// Top-k.  Each list arrives sorted descending (zero = padding).  Let q =
+// ceil(k / nslices): the q best keys of every list are nslices q >= k keys of
+// the union, so the k-th best key of the union is at least
+//     LB = min over lists of (the list's q-th key).
+// Only keys >= LB can be in the Top-k, and every key above a survivor is a
+// survivor too, so a survivor's rank among the survivors is its rank in the
+// union: ranking the survivors by counting yields the Top-k already sorted.
+// When too many keys survive (scores concentrated in few slices), a radix
+// select over all keys keeps k first and those k are ranked.  Inputs larger
+// than the shared-memory capacity run in rounds that keep the best k seen.
+constexpr int kRankDirect = 512;   // largest survivor count ranked directly
+
+__device__ __forceinline__ void merge_emit(const MergeArgs &a, int bh, int k, int r, u64 x)
+{
+    if (r >= k) return;
+    a.out_idx[(size_t)bh * k + r] = (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu));
+    if (a.out_score) a.out_score[(size_t)bh * k + r] = unord_f32((uint32_t)(x >> 32));
+}
+
 __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
 {
     extern __shared__ __align__(16) unsigned char s_dyn[];
     __shared__ RrShared sm;
     u64 *keys = reinterpret_cast<u64 *>(s_dyn);
     const int bh = blockIdx.x;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.topk;
     const int cap = a.cap;                     // keys[] capacity (>= 2k)
     int cnt = 0;
     u64 tau = 0ull;
-    pdl_wait();                                   // per-slice sets come from the rerank
+    pdl_wait();                                   // per-slice lists come from the rerank
     const int64_t total = (int64_t)a.nslices * k;
+    const u64 *plist = a.partial + (size_t)bh * a.max_slices * a.topk_cap;
+    u64 lb = 0ull;
+    if (total <= cap) {                           // lower bound of the k-th key (see above)
+        const int q = (k + a.nslices - 1) / a.nslices;
+        u64 v = ~0ull;
+        for (int s = tid; s < a.nslices; s += kRrThreads) {
+            const u64 y = plist[(size_t)s * a.topk_cap + (q - 1)];
+            v = y < v ? y : v;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            const u64 y = __shfl_xor_sync(kFull, v, o);
+            v = y < v ? y : v;
+        }
+        if (lane == 0) sm.red[0][warp] = v;
+    }
     for (int64_t e0 = 0; e0 < total; e0 += cap - k) {
         const int64_t e1 = min(total, e0 + (cap - k));
-        if (tid == 0) sm.cnt = (uint32_t)cnt;
+        if (tid == 0) {
+            sm.cnt = (uint32_t)cnt;
+            sm.bcnt = 0u;
+        }
         __syncthreads();
+        if (total <= cap) {
+            lb = sm.red[0][0];
+#pragma unroll
+            for (int w = 1; w < kRrWarps; w++) lb = sm.red[0][w] < lb ? sm.red[0][w] : lb;
+        }
         constexpr int kB8 = 8;       // loads in flight per thread
         for (int64_t eb = e0; eb < e1; eb += (int64_t)kB8 * kRrThreads) {
             u64 x[kB8];
@@ -461,7 +519,7 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
                 x[u] = 0ull;
                 if (e < e1) {
                     const int64_t j = e / k, r = e - j * k;
-                    x[u] = a.partial[((size_t)bh * a.max_slices + j) * a.topk_cap + r];
+                    x[u] = plist[(size_t)j * a.topk_cap + r];
                 }
             }
 #pragma unroll
@@ -469,10 +527,25 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
                 const bool take = x[u] != 0ull && x[u] > tau;
                 const uint32_t pos = warp_append(&sm.cnt, take);
                 if (take) keys[pos] = x[u];
+                const bool surv = take && x[u] >= lb;
+                const uint32_t sp = warp_append(&sm.bcnt, surv);
+                if (surv && sp < (uint32_t)kMaxTopk) sm.tmp[sp] = x[u];
             }
         }
         __syncthreads();
         cnt = (int)sm.cnt;
+        const int m = (int)sm.bcnt;
+        if (total <= cap && m <= (kRankDirect > k ? kRankDirect : k)) {
+            // survivors hold the whole Top-k: rank them, emit ranks < k
+            if (m < k && tid == 0) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, m);
+            rank_by_count(sm.tmp, m, [&](int r, u64 x) { merge_emit(a, bh, k, r, x); });
+            for (int i = m + tid; i < k; i += kRrThreads) {
+                a.out_idx[(size_t)bh * k + i] = -1;
+                if (a.out_score) a.out_score[(size_t)bh * k + i] = 0.0f;
+            }
+            pdl_trigger();
+            return;
+        }
         if (cnt > k) {
             tau = block_topk_select(sm, keys, cnt, k);
             for (int i = tid; i < k; i += kRrThreads) keys[i] = sm.tmp[i];
@@ -482,17 +555,10 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
     }
     const int got = min(cnt, k);
     if (got != k && tid == 0) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
-    int p2 = 32;
-    while (p2 < k) p2 <<= 1;
-    for (int i = tid; i < p2; i += kRrThreads) sm.tmp[i] = (i < got) ? keys[i] : 0ull;
-    __syncthreads();
-    if (warp == 0) warp_sort_desc(sm.tmp, p2);
-    __syncthreads();
-    for (int i = tid; i < k; i += kRrThreads) {
-        const u64 x = sm.tmp[i];
-        const bool live = i < got;
-        a.out_idx[(size_t)bh * k + i] = live ? (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu)) : -1;
-        if (a.out_score) a.out_score[(size_t)bh * k + i] = live ? unord_f32((uint32_t)(x >> 32)) : 0.0f;
+    rank_by_count(keys, got, [&](int r, u64 x) { merge_emit(a, bh, k, r, x); });
+    for (int i = got + tid; i < k; i += kRrThreads) {
+        a.out_idx[(size_t)bh * k + i] = -1;
+        if (a.out_score) a.out_score[(size_t)bh * k + i] = 0.0f;
     }
     pdl_trigger();
 }
