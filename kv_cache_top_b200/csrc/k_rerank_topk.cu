@@ -450,23 +450,55 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
 }
 
 // Merge of the per-slice Top-k lists of one pair into its final sorted
-// Top-k.  Each list arrives sorted descending (zero = padding).  Let q =
-// ceil(k / nslices): the q best keys of every list are nslices q >= k keys of
-// the union, so the k-th best key of the union is at least
-//     LB = min over lists of (the list's q-th key).
-// Only keys >= LB can be in the Top-k, and every key above a survivor is a
-// survivor too, so a survivor's rank among the survivors is its rank in the
-// union: ranking the survivors by counting yields the Top-k already sorted.
-// When too many keys survive (scores concentrated in few slices), a radix
-// select over all keys keeps k first and those k are ranked.  Inputs larger
-// than the shared-memory capacity run in rounds that keep the best k seen.
-constexpr int kRankDirect = 512;   // largest survivor count ranked directly
-
+// Top-k.  Each list arrives sorted descending (zero = padding; real keys are
+// distinct).  When the lists fit in shared memory (the usual case) a tree of
+// pairwise merges halves their number per level, each merge keeping its k
+// best: output position d of merge(A, B) comes from the co-rank of d (merge
+// path) -- the first d outputs are A[0..i) and B[0..d-i) for the i found by
+// binary search -- so every output is computed independently in log2(k)
+// steps and a level costs one barrier, whatever the score distribution.
+// Larger inputs run in rounds of radix select that keep the best k seen.
 __device__ __forceinline__ void merge_emit(const MergeArgs &a, int bh, int k, int r, u64 x)
 {
-    if (r >= k) return;
-    a.out_idx[(size_t)bh * k + r] = (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu));
-    if (a.out_score) a.out_score[(size_t)bh * k + r] = unord_f32((uint32_t)(x >> 32));
+    const bool live = x != 0ull;
+    a.out_idx[(size_t)bh * k + r] = live ? (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu)) : -1;
+    if (a.out_score) a.out_score[(size_t)bh * k + r] = live ? unord_f32((uint32_t)(x >> 32)) : 0.0f;
+}
+
+// Lists s = 0..ns-1 of k keys at src + s k; returns the buffer holding the
+// merged list (k keys).  src needs ns k keys, dst (ns + 1) / 2 k keys.  All
+// threads of the block call it.
+__device__ const u64 *merge_tree(u64 *src, u64 *dst, int ns, int k)
+{
+    while (ns > 1) {
+        const int np = (ns + 1) / 2;
+        const int tasks = np * k;
+        for (int t = threadIdx.x; t < tasks; t += kRrThreads) {
+            const int m = t / k, d = t - m * k;
+            const u64 *A = src + (size_t)(2 * m) * k;
+            u64 out;
+            if (2 * m + 1 >= ns) {
+                out = A[d];                       // odd list out: carried up
+            } else {
+                const u64 *B = A + k;
+                int lo = 0, hi = d;               // d < k: i in [0, d]
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (A[mid] > B[d - 1 - mid]) lo = mid + 1;
+                    else hi = mid;
+                }
+                const u64 x = A[lo], y = B[d - lo];
+                out = y > x ? y : x;
+            }
+            dst[(size_t)m * k + d] = out;
+        }
+        __syncthreads();
+        u64 *t = src;
+        src = dst;
+        dst = t;
+        ns = np;
+    }
+    return src;
 }
 
 __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
@@ -475,41 +507,35 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
     __shared__ RrShared sm;
     u64 *keys = reinterpret_cast<u64 *>(s_dyn);
     const int bh = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int k = a.topk;
     const int cap = a.cap;                     // keys[] capacity (>= 2k)
-    int cnt = 0;
-    u64 tau = 0ull;
     pdl_wait();                                   // per-slice lists come from the rerank
     const int64_t total = (int64_t)a.nslices * k;
     const u64 *plist = a.partial + (size_t)bh * a.max_slices * a.topk_cap;
-    u64 lb = 0ull;
-    if (total <= cap) {                           // lower bound of the k-th key (see above)
-        const int q = (k + a.nslices - 1) / a.nslices;
-        u64 v = ~0ull;
-        for (int s = tid; s < a.nslices; s += kRrThreads) {
-            const u64 y = plist[(size_t)s * a.topk_cap + (q - 1)];
-            v = y < v ? y : v;
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            const u64 y = __shfl_xor_sync(kFull, v, o);
-            v = y < v ? y : v;
-        }
-        if (lane == 0) sm.red[0][warp] = v;
-    }
-    for (int64_t e0 = 0; e0 < total; e0 += cap - k) {
-        const int64_t e1 = min(total, e0 + (cap - k));
-        if (tid == 0) {
-            sm.cnt = (uint32_t)cnt;
-            sm.bcnt = 0u;
+    if (total <= cap) {
+#pragma unroll 4
+        for (int e = tid; e < (int)total; e += kRrThreads) {
+            const int sl = e / k, r = e - sl * k;
+            keys[e] = plist[(size_t)sl * a.topk_cap + r];
         }
         __syncthreads();
-        if (total <= cap) {
-            lb = sm.red[0][0];
-#pragma unroll
-            for (int w = 1; w < kRrWarps; w++) lb = sm.red[0][w] < lb ? sm.red[0][w] : lb;
+        const u64 *res = merge_tree(keys, keys + cap, a.nslices, k);
+        if (tid == 0 && res[k - 1] == 0ull) {
+            int got = 0;
+            while (got < k && res[got] != 0ull) got++;
+            devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
         }
+        for (int d = tid; d < k; d += kRrThreads) merge_emit(a, bh, k, d, res[d]);
+        pdl_trigger();
+        return;
+    }
+    int cnt = 0;
+    u64 tau = 0ull;
+    for (int64_t e0 = 0; e0 < total; e0 += cap - k) {
+        const int64_t e1 = min(total, e0 + (cap - k));
+        if (tid == 0) sm.cnt = (uint32_t)cnt;
+        __syncthreads();
         constexpr int kB8 = 8;       // loads in flight per thread
         for (int64_t eb = e0; eb < e1; eb += (int64_t)kB8 * kRrThreads) {
             u64 x[kB8];
@@ -527,25 +553,10 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
                 const bool take = x[u] != 0ull && x[u] > tau;
                 const uint32_t pos = warp_append(&sm.cnt, take);
                 if (take) keys[pos] = x[u];
-                const bool surv = take && x[u] >= lb;
-                const uint32_t sp = warp_append(&sm.bcnt, surv);
-                if (surv && sp < (uint32_t)kMaxTopk) sm.tmp[sp] = x[u];
             }
         }
         __syncthreads();
         cnt = (int)sm.cnt;
-        const int m = (int)sm.bcnt;
-        if (total <= cap && m <= (kRankDirect > k ? kRankDirect : k)) {
-            // survivors hold the whole Top-k: rank them, emit ranks < k
-            if (m < k && tid == 0) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, m);
-            rank_by_count(sm.tmp, m, [&](int r, u64 x) { merge_emit(a, bh, k, r, x); });
-            for (int i = m + tid; i < k; i += kRrThreads) {
-                a.out_idx[(size_t)bh * k + i] = -1;
-                if (a.out_score) a.out_score[(size_t)bh * k + i] = 0.0f;
-            }
-            pdl_trigger();
-            return;
-        }
         if (cnt > k) {
             tau = block_topk_select(sm, keys, cnt, k);
             for (int i = tid; i < k; i += kRrThreads) keys[i] = sm.tmp[i];
@@ -556,14 +567,13 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
     const int got = min(cnt, k);
     if (got != k && tid == 0) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
     rank_by_count(keys, got, [&](int r, u64 x) { merge_emit(a, bh, k, r, x); });
-    for (int i = got + tid; i < k; i += kRrThreads) {
-        a.out_idx[(size_t)bh * k + i] = -1;
-        if (a.out_score) a.out_score[(size_t)bh * k + i] = 0.0f;
-    }
+    for (int i = got + tid; i < k; i += kRrThreads) merge_emit(a, bh, k, i, 0ull);
     pdl_trigger();
 }
 
-size_t merge_smem(int cap) { return (size_t)cap * sizeof(u64); }
+// dynamic shared memory of the merge: cap keys for the lists, (cap + 1) / 2 + k
+// for the first level of the merge tree
+size_t merge_smem(int cap) { return ((size_t)cap + (cap + 1) / 2 + 64 + 1024) * sizeof(u64); }
 
 cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s)
 {

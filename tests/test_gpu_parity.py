@@ -148,6 +148,25 @@ def test_duplicate_keys_tie_rule(pk):
         pk.pk_free(h)
 
 
+@pytest.mark.parametrize("n,width", [(32768, 150), (262144, 150)])
+def test_clustered_top_keys_merge(pk, n, width):
+    """Keys n0..n0+width-1 are made close to the query, so the whole Top-k sits
+    in one rerank slice: the per-slice lists are far from interleaved and the
+    merge must leave its usual short-prefix case (the larger n also gives
+    many slices and a weak prefix bound)."""
+    w = workloads.llama_layer(1, n, H=1, G=1, seed=width + n, device="cuda")
+    K = w["K"].clone()
+    q = w["q"][0]
+    n0 = n // 3
+    K[0, 0, n0:n0 + width] = (3.0 * q[0, 0].float() + 0.2 * K[0, 0, n0:n0 + width].float()).to(K.dtype)
+    h = build(pk, K, w["V"], n, 1, 1, 1)
+    try:
+        idx = check_pairs(pk, h, K, w["V"], q, [0], 1, 1, 1, n, 100)
+        assert ((idx[0] >= n0) & (idx[0] < n0 + width)).sum() >= 90
+    finally:
+        pk.pk_free(h)
+
+
 def test_append_matches_oracle(pk):
     """pk_append encodes new decode keys with the fixed codebook: the index
     after appends equals an index built over all keys at once."""
