@@ -223,6 +223,114 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
     return mn;
 }
 
+// Keep the k largest of keys[0..count) (k < count <= kMaxSlice; keys
+// distinct) in sm.tmp[0..k), any order, in one counting pass.  Scores of one
+// query span both signs and a few octaves, so bits of the key spread them
+// poorly; instead bin b(v) = min(255, floor((v - vmin) 256 / (vmax - vmin)))
+// of the score v, which never decreases as the key grows, so every key in a
+// bin above the boundary bin is kept.  The upper tail is sparse, so the bin
+// holding the k-th key usually has a few keys; one warp sorts it.  Keys are
+// held in registers, each warp histograms into its own 256 counters (hist,
+// 8 KB of free scratch), and appends take one atomic per warp.  Returns
+// false -- with nothing written to sm.tmp -- when the scores are all equal or
+// the boundary bin holds more than 32 keys that must be split; the caller
+// then runs the radix select.  All threads of the block call it.
+__device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int count, int k, uint32_t *hist)
+{
+    constexpr int kPer = kMaxSlice / kRrThreads;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    u64 x[kPer];
+    float vmin = INFINITY, vmax = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kPer; u++) {
+        const int i = tid + u * kRrThreads;
+        x[u] = (i < count) ? keys[i] : 0ull;
+        if (i < count) {
+            const float v = unord_f32((uint32_t)(x[u] >> 32));
+            vmin = fminf(vmin, v);
+            vmax = fmaxf(vmax, v);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        vmin = fminf(vmin, __shfl_xor_sync(kFull, vmin, o));
+        vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, o));
+    }
+    uint32_t *wh = hist + warp * 256;
+#pragma unroll
+    for (int i = 0; i < 8; i++) wh[lane + 32 * i] = 0u;
+    float *red = reinterpret_cast<float *>(&sm.red[0][0]);
+    if (lane == 0) {
+        red[warp] = vmin;
+        red[kRrWarps + warp] = vmax;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kRrWarps; w++) {
+        vmin = fminf(vmin, red[w]);
+        vmax = fmaxf(vmax, red[kRrWarps + w]);
+    }
+    const float range = vmax - vmin;
+    const float scale = 256.0f / range;
+    if (!(range > 0.0f) || !(range < INFINITY) || !(scale < INFINITY)) {
+        __syncthreads();
+        return false;
+    }
+    auto bin_of = [&](u64 key) {
+        const float v = unord_f32((uint32_t)(key >> 32));
+        return min(255, (int)((v - vmin) * scale));
+    };
+#pragma unroll
+    for (int u = 0; u < kPer; u++)
+        if (tid + u * kRrThreads < count) atomicAdd(&wh[bin_of(x[u])], 1u);
+    __syncthreads();
+    // thread tid takes bin 255 - tid: keys in higher bins by an exclusive scan
+    uint32_t hv = 0;
+#pragma unroll
+    for (int w = 0; w < kRrWarps; w++) hv += hist[w * 256 + 255 - tid];
+    uint32_t tot;
+    const uint32_t above = block_excl_scan<kRrThreads>(hv, reinterpret_cast<uint32_t *>(&sm.hist[0][0]), &tot);
+    if (above < (uint32_t)k && above + hv >= (uint32_t)k) {
+        sm.sh[0] = 255 - tid;
+        sm.sh[1] = above;
+        sm.sh[2] = hv;
+    }
+    if (tid == 0) {
+        sm.sh[3] = 0u;
+        sm.bcnt = 0u;
+    }
+    __syncthreads();
+    const int bstar = (int)sm.sh[0];
+    const int need = k - (int)sm.sh[1];
+    const int inbin = (int)sm.sh[2];
+    const bool small = inbin != need;          // the boundary bin must be split
+    if (small && inbin > 32) {
+        __syncthreads();
+        return false;
+    }
+    u64 *side = reinterpret_cast<u64 *>(&sm.hist[1][0]);   // <= 32 keys
+#pragma unroll
+    for (int u = 0; u < kPer; u++) {
+        const bool live = tid + u * kRrThreads < count;
+        const int bq = live ? bin_of(x[u]) : -1;
+        const bool keep = live && (small ? bq > bstar : bq >= bstar);
+        const uint32_t pos = warp_append(&sm.sh[3], keep);
+        if (keep) sm.tmp[pos] = x[u];
+        const bool inb = live && small && bq == bstar;
+        const uint32_t bp = warp_append(&sm.bcnt, inb);
+        if (inb) side[bp] = x[u];
+    }
+    __syncthreads();
+    if (small && warp == 0) {
+        u64 y = (lane < inbin) ? side[lane] : 0ull;
+        y = warp_sort32_desc(y);
+        const uint32_t base = sm.sh[3];
+        if (lane < need) sm.tmp[base + lane] = y;
+    }
+    __syncthreads();
+    return true;
+}
+
 // One warp sorts v[0..32 E) descending in place: E keys per lane in
 // registers (element e = E lane + i), bitonic network, shuffles for the
 // cross-lane stages -- no shared-memory round trips between stages.
@@ -437,7 +545,9 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
     // ---- Top-k set of the slice (unordered) and its smallest key
     const int have = min(count, k);
     if (count > k) {
-        block_topk_select(sm, keys, count, k);
+        // the ring is free now: 8 KB of it hold the per-warp histograms
+        if (!block_topk_select_linear(sm, keys, count, k, reinterpret_cast<uint32_t *>(ring_all)))
+            block_topk_select(sm, keys, count, k);
     } else {
         for (int i = tid; i < count; i += kRrThreads) sm.tmp[i] = keys[i];
         __syncthreads();
