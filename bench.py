@@ -11,8 +11,8 @@ budgets.  The line also carries the metric's 1M point (n = 1048576, 8 KV
 heads, K/V in pinned host memory read through UVA) under "million_token".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload throughput|million|llama|tiny] [--no-million]
-                  [--no-cpu-baseline] [--no-e2e] [--no-dense]
+                  [--workload throughput|million|llama|tiny|drift] [--no-million]
+                  [--no-cpu-baseline] [--no-e2e] [--no-dense] [--drift-steps T]
 
 For N > 1 launch under torch.distributed.run: every rank runs its own copy of
 the workload (pairs shard with no data-path collective: weak scaling); the
@@ -45,6 +45,9 @@ WORKLOADS = {
     "million": dict(name="million_1x1048576_uva", batch=1, n=1 << 20, H=8, G=4, cand=0, kv_host=True),
     "llama": dict(name="llama_1x32768", batch=1, n=32768, H=8, G=4, cand=2048, kv_host=False),
     "tiny": dict(name="tiny_1x4096", batch=1, n=4096, H=1, G=1, cand=512, kv_host=False),
+    # prefill 65536 keys per KV head, then 16384 decode steps of append + search
+    "drift": dict(name="drift_65536+16384", batch=1, n=65536, H=8, G=1, cand=0, kv_host=False,
+                  steps=16384, recall_every=256),
 }
 
 
@@ -61,6 +64,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--drift-steps", type=int, default=0,
+                    help="decode steps of the drift workload (default: all 16384)")
     return ap.parse_args()
 
 
@@ -437,6 +442,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     peak, peak_src = load_peaks()
     wl = WORKLOADS[args.workload]
+    if args.workload == "drift":
+        if world > 1:
+            raise SystemExit("the drift mode runs on one GPU")
+        return run_drift(args, wl, peak)
     want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
     res = run_ours(args, wl, rank, world, local_rank, want_cpu, peak)
 
@@ -518,6 +527,58 @@ def main():
     print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+# ------------------------------------------------------------ drift mode
+def run_drift(args, wl, peaks):
+    """Append + search per decode step over a drifting key stream (one KV
+    head group per step, G = 1); Recall@100 against the exact Top-100 of
+    <k_i, q> in fp64 over all keys so far, every `recall_every` steps."""
+    import torch
+    import kv_cache_top_b200 as pk
+    import workloads
+    dev = torch.device("cuda", 0)
+    n0, T, H, every = wl["n"], wl["steps"], wl["H"], wl["recall_every"]
+    if args.drift_steps > 0:
+        T = max(every, (min(args.drift_steps, T) // every) * every)
+    w = workloads.drift_stream(n0, T, H=H, seed=args.seed, device=dev)
+    p = pk.pk_default_params(batch=1, n_kv_heads=H, group=1, topk=100, n_cap=n0 + T, kv_dtype=pk.PK_BF16)
+    h = pk.pk_build_index(w["K"], w["V"], n0, p)
+    idx = torch.empty(H, 100, dtype=torch.int32, device=dev)
+    Kall = torch.cat([w["K"][0].double(), w["k_new"][:, 0, :, 0].permute(1, 0, 2).double()], dim=1)  # [H][n0+T][D]
+    stream = torch.cuda.current_stream()
+    for t in range(min(args.warmup, 8)):          # warm-up searches without appends
+        pk.pk_search(h, w["q"][0], 100, idx)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(T)]
+    recalls = []
+    for t in range(T):
+        ev[t][0].record(stream)
+        pk.pk_append(h, w["k_new"][t], w["v_new"][t], 1)
+        pk.pk_search(h, w["q"][t], 100, idx)
+        ev[t][1].record(stream)
+        if (t + 1) % every == 0:
+            n = n0 + t + 1
+            s = torch.einsum("hnd,hd->hn", Kall[:, :n], w["q"][t][0].double())
+            ex = torch.topk(s, 100, dim=1).indices
+            got = idx.long()
+            r = [len(set(ex[i].tolist()) & set(got[i].tolist())) / 100.0 for i in range(H)]
+            recalls.append((t + 1, sum(r) / H))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    pk.pk_free(h)
+    ms_tot = sum(ms)
+    line = {"metric": "append+search steps/s under key drift; Recall@100 every %d steps" % every,
+            "value": T / (ms_tot / 1000.0), "unit": "steps/s", "n_gpus": 1, "steps": T, "warmup": args.warmup,
+            "ms_per_step": ms_tot / T, "ms_per_step_median": statistics.median(ms), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl["name"], "n_prefill": n0, "kv_heads": H, "q_heads": H, "head_dim": 128,
+                       "topk": 100, "step": "pk_append (1 key per KV head) + pk_search",
+                       "l2": "not flushed (each step touches the index once)"},
+            "recall_at_100": [{"step": a, "recall": b} for a, b in recalls],
+            "recall_at_100_mean": sum(b for _, b in recalls) / max(1, len(recalls)),
+            "gpu_launches": None}
+    print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------- reference arm

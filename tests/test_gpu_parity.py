@@ -187,6 +187,31 @@ def test_append_matches_oracle(pk):
         pk.pk_free(h)
 
 
+def test_drift_stream_append_then_search(pk):
+    """Drift config: prefill 65536 keys per KV head (8 heads, G = 1) from
+    N(mu_0, diag sigma^2), then decode steps that each append one key drawn
+    from a distribution whose mean moves towards mu_1 and search with a query
+    from the same step law.  The codebook stays fixed; after 256 and 512
+    steps the whole path (occupancy, tiers, candidates, rerank, Top-k,
+    attention) still matches the oracle built over all keys at once."""
+    n0, T, H = 65536, 512, 8
+    w = workloads.drift_stream(n0, T, H=H, seed=7, device="cuda")
+    h = build(pk, w["K"], w["V"], n0, 1, H, 1, n_cap=n0 + T)
+    try:
+        idx = torch.empty(H, 100, dtype=torch.int32, device="cuda")
+        for t in range(T):
+            pk.pk_append(h, w["k_new"][t], w["v_new"][t], 1)
+            pk.pk_search(h, w["q"][t], 100, idx)
+            if t + 1 in (256, 512):
+                n = n0 + t + 1
+                K = torch.cat([w["K"], w["k_new"][:t + 1, 0, :, 0].permute(1, 0, 2).unsqueeze(0)], dim=2)
+                V = torch.cat([w["V"], w["v_new"][:t + 1, 0, :, 0].permute(1, 0, 2).unsqueeze(0)], dim=2)
+                assert pk.pk_get_info(h).n == n
+                check_pairs(pk, h, K, V, w["q"][t], [0, 5], 1, H, 1, n, 100, check_encode=(t + 1 == T))
+    finally:
+        pk.pk_free(h)
+
+
 def test_host_pinned_kv_store(pk):
     """K/V kept in pinned host memory and read through UVA by the attention."""
     w = workloads.llama_layer(1, 20000, H=2, G=4, seed=3, device="cuda")
