@@ -513,7 +513,7 @@ def main():
                      "unit": "GB/s", "frac": km[dom]["gbs"] / peak,
                      "traffic": profiled_traffic(dom, wl["name"]), "peak_source": peak_src},
         "kernels": km,
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": sum(v["launches"] for v in km.values()),
         "clocks": res["clocks"],
         "e2e": res["e2e"],
         "cpu_baseline": res.get("cpu"),
