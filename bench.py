@@ -12,7 +12,7 @@ heads, K/V in pinned host memory read through UVA) under "million_token".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload throughput|million|llama|tiny|drift] [--no-million]
-                  [--no-cpu-baseline] [--no-e2e] [--no-dense] [--drift-steps T]
+                  [--no-cpu-baseline] [--no-e2e] [--no-dense] [--graph] [--drift-steps T]
 
 For N > 1 launch under torch.distributed.run: every rank runs its own copy of
 the workload (pairs shard with no data-path collective: weak scaling); the
@@ -63,6 +63,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time one CUDA-graph launch per step instead of eager launches")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--drift-steps", type=int, default=0,
                     help="decode steps of the drift workload (default: all 16384)")
@@ -256,6 +258,26 @@ def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
         step(i)
     torch.cuda.synchronize()
 
+    # one CUDA graph per query of the pool: a step is then one graph launch
+    # (the library's programmatic dependent launches become graph edges)
+    graphs = None
+    if args.graph:
+        graphs = []
+        for i in range(nq):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(i)
+            graphs.append(g)
+        for i in range(min(args.warmup, nq)):
+            graphs[i].replay()
+        torch.cuda.synchronize()
+
+    def timed_step(i, trace):
+        if graphs is not None and not trace:
+            graphs[i % nq].replay()
+        else:
+            step(i)
+
     sampler = ClockSampler(None)
     if rank == 0:
         try:
@@ -280,7 +302,7 @@ def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
         for i in range(args.steps):
             flush.zero_()                      # L2 flush outside the timed events
             evs[i][0].record(stream)
-            step(i)
+            timed_step(i, trace)
             evs[i][1].record(stream)
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
@@ -332,7 +354,8 @@ def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
                "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
 
     res = dict(ms_total=ms_clean, wall=wall_clean, kern=kern, recall=recall, C=C, R=R, info=info,
-               e2e=e2e, clocks=clocks, ms_traced=ms_traced)
+               e2e=e2e, clocks=clocks, ms_traced=ms_traced, graph=graphs is not None)
+    del graphs
 
     # dense-attention comparator on the same tensors (HBM workloads only)
     if rank == 0 and not wl["kv_host"] and not args.no_dense:
@@ -505,6 +528,7 @@ def main():
                    "kv_dtype": "bf16", "index": "16 B codes + 128 B 4-bit record per key",
                    "l2": "flushed between timed steps (256 MiB write outside the events)",
                    "queries": "fresh query per step from a 64-query pool",
+                   "launch": "one CUDA graph per step" if res["graph"] else "eager launches",
                    "parallelism": "replicas: each rank its own %d pairs" % (wl["batch"] * wl["H"])},
         "recall_at_100": res["recall"],
         "hbm": {"alg_bytes_per_step": step_bytes, "gbs": step_bytes / ms_per_step / 1e6,
