@@ -309,17 +309,26 @@ __device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int coun
         return false;
     }
     u64 *side = reinterpret_cast<u64 *>(&sm.hist[1][0]);   // <= 32 keys
+    // positions by one block scan of per-thread counts (kept keys in the
+    // high half, boundary-bin keys in the low half), then plain stores
+    uint32_t keepm = 0, inbm = 0;
 #pragma unroll
     for (int u = 0; u < kPer; u++) {
         const bool live = tid + u * kRrThreads < count;
         const int bq = live ? bin_of(x[u]) : -1;
-        const bool keep = live && (small ? bq > bstar : bq >= bstar);
-        const uint32_t pos = warp_append(&sm.sh[3], keep);
-        if (keep) sm.tmp[pos] = x[u];
-        const bool inb = live && small && bq == bstar;
-        const uint32_t bp = warp_append(&sm.bcnt, inb);
-        if (inb) side[bp] = x[u];
+        if (live && (small ? bq > bstar : bq >= bstar)) keepm |= 1u << u;
+        if (live && small && bq == bstar) inbm |= 1u << u;
     }
+    uint32_t tot2;
+    const uint32_t ex2 = block_excl_scan<kRrThreads>(((uint32_t)__popc(keepm) << 16) | (uint32_t)__popc(inbm),
+                                                     reinterpret_cast<uint32_t *>(&sm.hist[0][0]), &tot2);
+    uint32_t pos = ex2 >> 16, bp = ex2 & 0xffffu;
+#pragma unroll
+    for (int u = 0; u < kPer; u++) {
+        if (keepm & (1u << u)) sm.tmp[pos++] = x[u];
+        if (inbm & (1u << u)) side[bp++] = x[u];
+    }
+    if (tid == 0) sm.sh[3] = tot2 >> 16;
     __syncthreads();
     if (small && warp == 0) {
         u64 y = (lane < inbin) ? side[lane] : 0ull;
