@@ -15,7 +15,23 @@ from . import _lib
 from ._lib import (KERNELS, PK_BF16, PK_F32, PK_KV_DEVICE, PK_KV_HOST_PINNED, PK_OK, pk_debug_out,
                    pk_info, pk_params)
 
-lib = _lib.load()
+_handle = None
+
+
+def _L():
+    """The loaded library: loaded on first use, so that importing the package
+    (e.g. to build it) does not need it; every API call fails loudly (an
+    ImportError) when it is missing."""
+    global _handle
+    if _handle is None:
+        _handle = _lib.load()
+    return _handle
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _L()
+    raise AttributeError("module %r has no attribute %r" % (__name__, name))
 
 __all__ = [
     "PkError", "pk_default_params", "pk_build_index", "pk_append", "pk_search", "pk_search_debug",
@@ -56,12 +72,12 @@ def _stream(stream):
 
 
 def pk_status_str(status: int) -> str:
-    return lib.pk_status_str(status).decode()
+    return _L().pk_status_str(status).decode()
 
 
 def pk_default_params(**kw) -> pk_params:
     p = pk_params()
-    lib.pk_default_params(C.byref(p))
+    _L().pk_default_params(C.byref(p))
     for k, v in kw.items():
         if not hasattr(p, k):
             raise AttributeError("pk_params has no field %r" % k)
@@ -71,17 +87,17 @@ def pk_default_params(**kw) -> pk_params:
 
 def pk_build_index(K, V, n: int, params: pk_params, stream=None) -> C.c_void_p:
     h = C.c_void_p()
-    _check(lib.pk_build_index(_ptr(K), _ptr(V), int(n), C.byref(params), _stream(stream), C.byref(h)),
+    _check(_L().pk_build_index(_ptr(K), _ptr(V), int(n), C.byref(params), _stream(stream), C.byref(h)),
            "pk_build_index")
     return h
 
 
 def pk_append(index, k_new, v_new, n_new: int, stream=None):
-    _check(lib.pk_append(index, _ptr(k_new), _ptr(v_new), int(n_new), _stream(stream)), "pk_append")
+    _check(_L().pk_append(index, _ptr(k_new), _ptr(v_new), int(n_new), _stream(stream)), "pk_append")
 
 
 def pk_search(index, q, topk: int, out_idx, out_score=None, stream=None):
-    _check(lib.pk_search(index, _ptr(q), int(topk), _ptr(out_idx), _ptr(out_score), _stream(stream)),
+    _check(_L().pk_search(index, _ptr(q), int(topk), _ptr(out_idx), _ptr(out_score), _stream(stream)),
            "pk_search")
 
 
@@ -90,66 +106,66 @@ def pk_search_debug(index, q, topk: int, out_idx, out_score=None, dbg: dict | No
     d = pk_debug_out()
     for k, v in (dbg or {}).items():
         setattr(d, k, _ptr(v))
-    _check(lib.pk_search_debug(index, _ptr(q), int(topk), _ptr(out_idx), _ptr(out_score), C.byref(d),
+    _check(_L().pk_search_debug(index, _ptr(q), int(topk), _ptr(out_idx), _ptr(out_score), C.byref(d),
                                _stream(stream)), "pk_search_debug")
 
 
 def pk_attend(index, q, sel_idx, topk: int, out, stream=None):
-    _check(lib.pk_attend(index, _ptr(q), _ptr(sel_idx), int(topk), _ptr(out), _stream(stream)),
+    _check(_L().pk_attend(index, _ptr(q), _ptr(sel_idx), int(topk), _ptr(out), _stream(stream)),
            "pk_attend")
 
 
 def pk_free(index):
-    lib.pk_free(index)
+    _L().pk_free(index)
 
 
 def pk_last_device_error(index):
     """(status, detail): waits for the device, then reads and clears the
     index's device-check word."""
     det = C.c_int64(0)
-    st = lib.pk_last_device_error(index, C.byref(det))
+    st = _L().pk_last_device_error(index, C.byref(det))
     return st, det.value
 
 
 def pk_get_info(index) -> pk_info:
     info = pk_info()
-    _check(lib.pk_get_info(index, C.byref(info)), "pk_get_info")
+    _check(_L().pk_get_info(index, C.byref(info)), "pk_get_info")
     return info
 
 
 def pk_export_index(index, codes=None, records=None, occ=None, stream=None):
-    _check(lib.pk_export_index(index, _ptr(codes), _ptr(records), _ptr(occ), _stream(stream)),
+    _check(_L().pk_export_index(index, _ptr(codes), _ptr(records), _ptr(occ), _stream(stream)),
            "pk_export_index")
 
 
 def pk_magnitude_levels(m: int = 8, L: int = 8):
     lev = np.empty(L, np.float32)
     thr = np.empty(L - 1, np.float32)
-    _check(lib.pk_magnitude_levels(m, L, lev.ctypes.data, thr.ctypes.data), "pk_magnitude_levels")
+    _check(_L().pk_magnitude_levels(m, L, lev.ctypes.data, thr.ctypes.data), "pk_magnitude_levels")
     return lev, thr
 
 
 def pk_resolve(n: int, cand_budget: int = 0, collision_ratio: float = 0.0, topk: int = 100):
     c = C.c_int64()
     r = C.c_int64()
-    _check(lib.pk_resolve(n, cand_budget, collision_ratio, topk, C.byref(c), C.byref(r)), "pk_resolve")
+    _check(_L().pk_resolve(n, cand_budget, collision_ratio, topk, C.byref(c), C.byref(r)), "pk_resolve")
     return c.value, r.value
 
 
 def pk_trace_enable(index, on: bool = True):
-    _check(lib.pk_trace_enable(index, 1 if on else 0), "pk_trace_enable")
+    _check(_L().pk_trace_enable(index, 1 if on else 0), "pk_trace_enable")
 
 
 def pk_trace_read(index):
     """{kernel: (launches, total_ms)} since the last read (synchronises)."""
     n = np.zeros(len(KERNELS), np.int64)
     ms = np.zeros(len(KERNELS), np.float64)
-    _check(lib.pk_trace_read(index, n.ctypes.data, ms.ctypes.data), "pk_trace_read")
+    _check(_L().pk_trace_read(index, n.ctypes.data, ms.ctypes.data), "pk_trace_read")
     return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(KERNELS)}
 
 
 def pk_select_candidates_noalloc(S, n: int, C: int, cand, stream=None):
     """Top-C candidate ids of one score row with no device allocation (see
     include/pariskv.h): for callers that cannot allocate at that moment."""
-    _check(lib.pk_select_candidates_noalloc(_ptr(S), int(n), int(C), _ptr(cand), _stream(stream)),
+    _check(_L().pk_select_candidates_noalloc(_ptr(S), int(n), int(C), _ptr(cand), _stream(stream)),
            "pk_select_candidates_noalloc")

@@ -455,15 +455,6 @@ __device__ __forceinline__ float block_dot(const float *slev, uint32_t nib, cons
     return d;
 }
 
-// 16-byte asynchronous global -> shared copy (L2 only, no register staging)
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
-{
-    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 constexpr int kRrStages = 3;                       // per-warp pipeline depth
 constexpr int kRrStep = 16;                        // records per warp stage

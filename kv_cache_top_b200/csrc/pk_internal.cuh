@@ -110,14 +110,6 @@ struct RerankArgs {
     float *dbg_est;          // [BH][C] or null
 };
 
-struct MergeArgs {
-    const unsigned long long *partial;
-    int32_t nslices, max_slices, topk, topk_cap, cap;
-    int32_t *out_idx;        // [BH][topk]
-    float *out_score;        // [BH][topk] or null
-    int32_t *dev_err;
-};
-
 struct AttendArgs {
     const void *q;           // [batch][H*G][D]
     const int32_t *idx;      // [BH][topk]
@@ -132,12 +124,31 @@ struct AttendArgs {
     long long *dev_err_detail;
 };
 
+struct MergeArgs {
+    const unsigned long long *partial;
+    int32_t nslices, max_slices, topk, topk_cap, cap;
+    int32_t *out_idx;        // [BH][topk]
+    float *out_score;        // [BH][topk] or null
+    int32_t *dev_err;
+};
+
+
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float ld_as_f32(const void *p, int64_t i, int is_bf16)
 {
     if (is_bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
     return reinterpret_cast<const float *>(p)[i];
 }
+
+// 16-byte asynchronous global -> shared copy (L2 only, no register staging)
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Map an fp32 value to an unsigned key whose integer order is the float order.
 // -0.0 must already be folded into +0.0 by the caller (x + 0.0f).
