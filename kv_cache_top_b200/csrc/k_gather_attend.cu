@@ -12,10 +12,11 @@
 // CTA takes a contiguous share of the selected rows, 32 rows per tile, and
 // issues every 16-byte load of a tile's K and V rows before using any, so a
 // tile costs one round trip over the host link and several SMs pull rows at
-// once.  Each CTA keeps an online softmax (max, sum, weighted V) in fp32; CTA
-// rank 0 then merges the partials of its cluster through distributed shared
-// memory with the log-sum-exp rule.  Ids outside [0, n) are skipped and
-// recorded in the device-check word (no trap).
+// once.  Each CTA keeps an online softmax (max, sum, weighted V) in fp32, then
+// pushes its partial into CTA rank 0's shared memory with distributed-shared-
+// memory stores (no remote round trip), and rank 0 merges the partials with
+// the log-sum-exp rule.  Ids outside [0, n) are skipped and recorded in the
+// device-check word (no trap).
 #include <cooperative_groups.h>
 
 #include "pk_internal.cuh"
@@ -30,13 +31,20 @@ constexpr int kAtLoads = kAtRows * 32 / kAtThreads;   // 16-byte loads per threa
 
 __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
 {
-    __shared__ __align__(16) unsigned char sK[kAtRows * kD * 4];
-    __shared__ __align__(16) unsigned char sV[kAtRows * kD * 4];
+    // the K and V tiles; after the row loop rank 0 reuses them for the
+    // cluster's partial accumulators [8][kMaxGroup][kD] (32 KB)
+    __shared__ __align__(16) unsigned char s_kv[2 * kAtRows * kD * 4];
+    unsigned char *sK = s_kv;
+    unsigned char *sV = s_kv + kAtRows * kD * 4;
     __shared__ int32_t s_idx[kAtRows];
     __shared__ float s_q[kMaxGroup][kD];
     __shared__ float s_p[kMaxGroup][kAtRows];
     __shared__ float s_m[kMaxGroup], s_l[kMaxGroup], s_alpha[kMaxGroup];
-    __shared__ float s_acc[kMaxGroup][kD];
+    // rank 0 only: every CTA's partial (running max, sum, accumulator), pushed
+    // here with distributed-shared-memory stores before the cluster barrier
+    __shared__ float s_pm[8][kMaxGroup], s_pl[8][kMaxGroup];
+    static_assert(8 * kMaxGroup * kD * 4 <= 2 * kAtRows * kD * 4, "partials fit in the row tiles");
+    float (*s_pacc)[kMaxGroup][kD] = reinterpret_cast<float (*)[kMaxGroup][kD]>(s_kv);
 
     cg::cluster_group cluster = cg::this_cluster();
     const int sp = (int)cluster.block_rank(), bh = blockIdx.y;
@@ -161,33 +169,41 @@ __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
             }
         }
     }
+    // ---- push this CTA's partial into rank 0 (remote stores: no round trip)
+    float *pm = cluster.map_shared_rank(&s_pm[0][0], 0);
+    float *pl = cluster.map_shared_rank(&s_pl[0][0], 0);
+    float *pacc = cluster.map_shared_rank(&s_pacc[0][0][0], 0);
+    cluster.sync();                                   // every CTA is done with its rows (and s_m, s_l)
+    if (tid < G) {
+        pm[sp * kMaxGroup + tid] = s_m[tid];
+        pl[sp * kMaxGroup + tid] = s_l[tid];
+    }
 #pragma unroll
     for (int i = 0; i < kMaxGroup / 2; i++) {
         const int g = gsel + 2 * i;
-        if (g < G) s_acc[g][d] = acc[i];
+        if (g < G) pacc[((size_t)sp * kMaxGroup + g) * kD + d] = acc[i];
     }
-    // ---- merge the cluster's partials in CTA rank 0 (distributed shared memory)
-    cluster.sync();
+    cluster.sync();                                   // every partial has landed in rank 0
     if (sp == 0) {
+        // log-sum-exp merge of the nsp partials, from local shared memory
 #pragma unroll
         for (int i = 0; i < kMaxGroup / 2; i++) {
             const int g = gsel + 2 * i;
             if (g >= G) continue;
             float M = -INFINITY;
-            for (int r = 0; r < nsp; r++) M = fmaxf(M, *cluster.map_shared_rank(&s_m[g], r));
+            for (int r = 0; r < nsp; r++) M = fmaxf(M, s_pm[r][g]);
             float num = 0.0f, den = 0.0f;
             if (M != -INFINITY) {
                 for (int r = 0; r < nsp; r++) {
-                    const float mr = *cluster.map_shared_rank(&s_m[g], r);
+                    const float mr = s_pm[r][g];
                     const float f = (mr == -INFINITY) ? 0.0f : expf(mr - M);
-                    num = fmaf(f, *cluster.map_shared_rank(&s_acc[g][d], r), num);
-                    den = fmaf(f, *cluster.map_shared_rank(&s_l[g], r), den);
+                    num = fmaf(f, s_pacc[r][g][d], num);
+                    den = fmaf(f, s_pl[r][g], den);
                 }
             }
             a.out[qbase + (int64_t)g * kD + d] = (den > 0.0f) ? num / den : 0.0f;
         }
     }
-    cluster.sync();   // peers keep their shared memory until rank 0 has read it
 }
 
 cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s)
