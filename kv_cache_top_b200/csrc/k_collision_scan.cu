@@ -77,23 +77,47 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
     uint8_t *dS = a.dbg_S ? a.dbg_S + (size_t)bh * a.n + lo : nullptr;
 
     // every lane runs every iteration (the shuffles need the full warp);
-    // lanes past the end of the chunk compute on a zero code and store nothing
-    for (int64_t base = (int64_t)warp * 32 * kScanUnroll; base < cnt;
-         base += (int64_t)NW * 32 * kScanUnroll) {
+    // lanes past the end of the chunk compute on a zero code and store
+    // nothing.  Offsets within the chunk are 32-bit (a chunk is < 2^31 keys),
+    // and iterations that lie wholly inside the chunk skip the per-key checks.
+    const uint32_t ucnt = (uint32_t)cnt;
+    uint32_t *hw = s_hist[warp];
+    for (uint32_t base = (uint32_t)warp * 32 * kScanUnroll + lane; base < ucnt + lane;
+         base += (uint32_t)NW * 32 * kScanUnroll) {
+        const bool full = base - lane + 32 * kScanUnroll <= ucnt;
         uint4 c[kScanUnroll];
+        if (full) {
 #pragma unroll
-        for (int u = 0; u < kScanUnroll; u++) {
-            const int64_t i = base + u * 32 + lane;
-            c[u] = (i < cnt) ? __ldcs(codes + i) : make_uint4(0, 0, 0, 0);
+            for (int u = 0; u < kScanUnroll; u++) c[u] = __ldcs(codes + base + u * 32);
+        } else {
+#pragma unroll
+            for (int u = 0; u < kScanUnroll; u++) {
+                const uint32_t i = base + u * 32;
+                c[u] = (i < ucnt) ? __ldcs(codes + i) : make_uint4(0, 0, 0, 0);
+            }
         }
+        uint32_t sc[kScanUnroll];
 #pragma unroll
-        for (int u = 0; u < kScanUnroll; u++) {
-            const int64_t i = base + u * 32 + lane;
-            const uint32_t s = collision_score(tab, c[u]);
-            if (i < cnt) {
-                S[i] = (uint8_t)s;
-                if (dS) dS[i] = (uint8_t)s;
-                atomicAdd(&s_hist[warp][s], 1u);
+        for (int u = 0; u < kScanUnroll; u++) sc[u] = collision_score(tab, c[u]);
+        if (full) {
+#pragma unroll
+            for (int u = 0; u < kScanUnroll; u++) {
+                S[base + u * 32] = (uint8_t)sc[u];
+                atomicAdd(&hw[sc[u]], 1u);
+            }
+            if (dS) {
+#pragma unroll
+                for (int u = 0; u < kScanUnroll; u++) dS[base + u * 32] = (uint8_t)sc[u];
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < kScanUnroll; u++) {
+                const uint32_t i = base + u * 32;
+                if (i < ucnt) {
+                    S[i] = (uint8_t)sc[u];
+                    if (dS) dS[i] = (uint8_t)sc[u];
+                    atomicAdd(&hw[sc[u]], 1u);
+                }
             }
         }
     }
