@@ -61,3 +61,13 @@ def test_reference_arm_world2_rank0_only():
     assert line["unit"] == "steps/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_parallel_cpu_baseline_uses_several_cores():
+    """bench.py's all-cores oracle baseline (spawn-started workers, one pair
+    each, timed together) on a tiny workload."""
+    wl = dict(bench.WORKLOADS["tiny"], batch=2, H=2)
+    r = bench.cpu_baseline_parallel(wl, 0, queries=2, max_workers=2)
+    assert r["kind"] == "oracle" and r["unit"] == "steps/s"
+    assert r["cores"] == min(2, os.cpu_count() or 1)
+    assert r["value"] > 0
