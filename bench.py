@@ -475,7 +475,7 @@ def _oracle_worker(job):
     return queries, time.perf_counter() - t0
 
 
-def cpu_baseline_parallel(wl, seed, queries=16, max_workers=32):
+def cpu_baseline_parallel(wl, seed, queries=64, max_workers=32):
     """The oracle on all host cores: one process (spawn-started, so it is safe
     after GPU use) per core, each on its own sampled pair, all timing their
     searches at once.  Throughput = searches done / the slowest worker's time."""
