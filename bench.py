@@ -11,7 +11,7 @@ budgets.  The line also carries the metric's 1M point (n = 1048576, 8 KV
 heads, K/V in pinned host memory read through UVA) under "million_token".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload throughput|million|llama|tiny|drift] [--no-million]
+                  [--workload throughput|million|llama|tiny|drift|sweep] [--no-million]
                   [--no-cpu-baseline] [--no-e2e] [--no-dense] [--graph] [--drift-steps T]
 
 For N > 1 launch under torch.distributed.run: every rank runs its own copy of
@@ -45,6 +45,10 @@ WORKLOADS = {
     "million": dict(name="million_1x1048576_uva", batch=1, n=1 << 20, H=8, G=4, cand=0, kv_host=True),
     "llama": dict(name="llama_1x32768", batch=1, n=32768, H=8, G=4, cand=2048, kv_host=False),
     "tiny": dict(name="tiny_1x4096", batch=1, n=4096, H=1, G=1, cand=512, kv_host=False),
+    # Recall@100 and step time over a grid of candidate / collision ratios
+    "sweep": dict(name="ratio_sweep", batch=1, n=0, H=8, G=4, cand=0, kv_host=False,
+                  ns=(32768, 131072, 524288, 1048576), betas=(0.02, 0.05, 0.1, 0.2),
+                  rhos=(0.05, 0.1, 0.2, 0.35, 0.5), queries=8),
     # prefill 65536 keys per KV head, then 16384 decode steps of append + search
     "drift": dict(name="drift_65536+16384", batch=1, n=65536, H=8, G=1, cand=0, kv_host=False,
                   steps=16384, recall_every=256),
@@ -525,6 +529,10 @@ def main():
         if world > 1:
             raise SystemExit("the drift mode runs on one GPU")
         return run_drift(args, wl, peak)
+    if args.workload == "sweep":
+        if world > 1:
+            raise SystemExit("the sweep runs on one GPU")
+        return run_sweep(args, wl)
     want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
     res = run_ours(args, wl, rank, world, local_rank, want_cpu, peak)
 
@@ -659,6 +667,65 @@ def run_drift(args, wl, peaks):
             "recall_at_100_mean": sum(b for _, b in recalls) / max(1, len(recalls)),
             "gpu_launches": None}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ ratio sweep
+def run_sweep(args, wl):
+    """Recall@100 (against the exact Top-100 of <k_i, q_agg>, fp32) and the
+    search + attend time per step for candidate ratio beta (C = ceil(beta n))
+    and collision ratio rho, plus the ratio table's own choice, at several n
+    (1 sequence x 8 KV heads, Llama-shaped keys, K/V in HBM)."""
+    import torch
+    import kv_cache_top_b200 as pk
+    import workloads
+    dev = torch.device("cuda", 0)
+    H, G, topk, nq = wl["H"], wl["G"], 100, wl["queries"]
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    grid = []
+    for n in wl["ns"]:
+        w = workloads.llama_layer(1, n, H=H, G=G, seed=args.seed, device=dev, n_queries=nq)
+        exact = []
+        for qi in range(nq):
+            qa = w["q"][qi].float().view(H, G, 128).sum(1)
+            s_ = torch.einsum("hnd,hd->hn", w["K"][0].float(), qa)
+            exact.append(torch.topk(s_, topk, dim=1).indices.cpu())
+        idx = torch.empty(H, topk, dtype=torch.int32, device=dev)
+        out = torch.empty(1, H * G, 128, dtype=torch.float32, device=dev)
+        points = [(0.0, 0.0)] + [(b, r) for b in wl["betas"] for r in wl["rhos"]]
+        for beta, rho in points:
+            cand = math.ceil(beta * n) if beta > 0 else 0
+            p = pk.pk_default_params(batch=1, n_kv_heads=H, group=G, topk=topk, cand_budget=cand,
+                                     collision_ratio=rho, kv_dtype=pk.PK_BF16)
+            h = pk.pk_build_index(w["K"], w["V"], n, p)
+            C, R = pk.pk_resolve(n, cand, rho, topk)
+            rec = []
+            for qi in range(nq):
+                pk.pk_search(h, w["q"][qi], topk, idx)
+                got = idx.cpu()
+                rec += [len(set(exact[qi][i].tolist()) & set(got[i].tolist())) / topk for i in range(H)]
+            ev = []
+            for i in range(3 + 10):
+                flush.zero_()
+                a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a_.record(stream)
+                pk.pk_search(h, w["q"][i % nq], topk, idx)
+                pk.pk_attend(h, w["q"][i % nq], idx, topk, out)
+                b_.record(stream)
+                ev.append((a_, b_))
+            torch.cuda.synchronize()
+            ms = statistics.median([a_.elapsed_time(b_) for a_, b_ in ev[3:]])
+            grid.append({"n": n, "beta": beta if beta > 0 else "table", "rho": rho if rho > 0 else "table",
+                         "C": C, "R": R, "recall_at_100": sum(rec) / len(rec), "ms_per_step": ms})
+            pk.pk_free(h)
+        del w
+        torch.cuda.empty_cache()
+    print(json.dumps({"metric": "Recall@100 and step time vs candidate / collision ratio",
+                      "unit": "recall", "data": "synthetic", "dtype": "f32",
+                      "config": {"workload": wl["name"], "batch": 1, "kv_heads": H, "q_heads": H * G,
+                                 "head_dim": 128, "topk": topk, "queries": nq,
+                                 "step": "pk_search + pk_attend for all 8 KV heads, L2 flushed, median of 10"},
+                      "grid": grid}), flush=True)
 
 
 # ---------------------------------------------------------- reference arm

@@ -134,6 +134,24 @@ def test_edge_and_ragged_sizes(pk, n, cand, topk, batch, H, G):
         pk.pk_free(h)
 
 
+@pytest.mark.parametrize("beta,rho", [(0.02, 0.35), (0.2, 0.05)])
+def test_explicit_budgets(pk, beta, rho):
+    """Budgets away from the ratio table (the sweep's grid points): C =
+    ceil(beta n) and R = ceil(rho n) reach the tiers, the threshold and the
+    rerank unchanged."""
+    n = 30000
+    w = workloads.llama_layer(1, n, H=2, G=4, seed=int(1000 * beta + 100 * rho), device="cuda")
+    C = math.ceil(beta * n)
+    h = build(pk, w["K"], w["V"], n, 1, 2, 4, cand_budget=C, collision_ratio=rho)
+    try:
+        Cr, Rr = pk.pk_resolve(n, C, rho, 100)
+        assert Cr == C and Rr == math.ceil(float(np.float32(rho)) * n)   # rho travels as fp32
+        check_pairs(pk, h, w["K"], w["V"], w["q"][0], [0, 1], 1, 2, 4, n, 100, cand_budget=C,
+                    collision_ratio=rho)
+    finally:
+        pk.pk_free(h)
+
+
 def test_duplicate_keys_tie_rule(pk):
     """Many identical keys: equal scores everywhere, so the lower-id rule
     decides the candidate set and the Top-k, bit-exactly."""
