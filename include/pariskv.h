@@ -170,6 +170,24 @@ pk_status pk_search_debug(pk_index *index, const void *q, int32_t topk, int32_t 
 pk_status pk_attend(pk_index *index, const void *q, const int32_t *sel_idx, int32_t topk,
                     float *out, void *stream);
 
+/* Exact attention over the selected rows together with rows kept densely on
+ * the GPU outside the index -- the sink tokens and the recent local window --
+ * under one softmax (README, step 3: attention "over sink tokens, local
+ * tokens, and retrieved tokens"; slides, Fig. 5: sink and local tokens stay
+ * on the GPU for dense attention while the retrieval region is searched).
+ *   q, sel_idx, topk, out  as for pk_attend, except that topk may be 0
+ *            (dense rows only; sel_idx may then be NULL).
+ *   dense_K, dense_V  [BH][dense_stride][D] kv_dtype, device (or mapped host),
+ *            16-byte aligned, owned by the caller; rows 0..dense_len-1 of every
+ *            pair are attended (their order does not matter).
+ *   dense_len  0 <= dense_len <= dense_stride; topk + dense_len >= 1.
+ * o_g = sum over the topk selected rows and the dense rows of
+ * softmax(scale <q_g, k>) v.  Errors: PK_ERR_INVALID_ARG for a bad pointer,
+ * alignment or size; selected ids outside [0, n) as for pk_attend. */
+pk_status pk_attend_dense(pk_index *index, const void *q, const int32_t *sel_idx, int32_t topk,
+                          const void *dense_K, const void *dense_V, int64_t dense_stride,
+                          int32_t dense_len, float *out, void *stream);
+
 /* Free everything the index owns (synchronises the device first). NULL is ok. */
 void pk_free(pk_index *index);
 

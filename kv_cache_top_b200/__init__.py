@@ -37,7 +37,7 @@ __all__ = [
     "PkError", "pk_default_params", "pk_build_index", "pk_append", "pk_search", "pk_search_debug",
     "pk_attend", "pk_free", "pk_status_str", "pk_last_device_error", "pk_get_info",
     "pk_export_index", "pk_magnitude_levels", "pk_resolve", "pk_trace_enable", "pk_trace_read",
-    "pk_select_candidates_noalloc", "pk_params", "pk_info", "pk_debug_out", "PK_F32", "PK_BF16", "PK_KV_DEVICE",
+    "pk_select_candidates_noalloc", "pk_attend_dense", "pk_params", "pk_info", "pk_debug_out", "PK_F32", "PK_BF16", "PK_KV_DEVICE",
     "PK_KV_HOST_PINNED", "KERNELS", "lib",
 ]
 
@@ -113,6 +113,14 @@ def pk_search_debug(index, q, topk: int, out_idx, out_score=None, dbg: dict | No
 def pk_attend(index, q, sel_idx, topk: int, out, stream=None):
     _check(_L().pk_attend(index, _ptr(q), _ptr(sel_idx), int(topk), _ptr(out), _stream(stream)),
            "pk_attend")
+
+
+def pk_attend_dense(index, q, sel_idx, topk: int, dense_K, dense_V, dense_len: int, out, stream=None):
+    """Attention over the selected rows and the dense (sink + local) rows of
+    dense_K/dense_V [BH][stride][D] under one softmax."""
+    dstride = dense_K.shape[-2] if dense_K is not None and hasattr(dense_K, "shape") else 0
+    _check(_L().pk_attend_dense(index, _ptr(q), _ptr(sel_idx), int(topk), _ptr(dense_K), _ptr(dense_V),
+                                int(dstride), int(dense_len), _ptr(out), _stream(stream)), "pk_attend_dense")
 
 
 def pk_free(index):

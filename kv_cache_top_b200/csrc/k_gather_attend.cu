@@ -3,7 +3,10 @@
 // o_g = sum_r softmax_r(scale <q_g, K[sel_r]>) V[sel_r] for every query head
 // g of the KV head (ParisKV slides, "The target is high-score KV indices at
 // each decode step", Sec. 3 Eqs. 1-3: "recompute softmax and value
-// aggregation using the selected full-precision KV").  The K/V rows are read
+// aggregation using the selected full-precision KV").  Optionally the rows
+// kept densely on the GPU outside the index -- the sink and recent local
+// tokens -- join the same softmax (README, step 3: attention "over sink
+// tokens, local tokens, and retrieved tokens"; slides, Fig. 5 layout).  The K/V rows are read
 // where the index keeps them: HBM, or pinned host memory through UVA (README,
 // "Attention: fetch only selected KV pairs ... from pinned CPU memory via
 // UVA").
@@ -55,8 +58,10 @@ __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
     const int es = a.is_bf16 ? 2 : 4;
     const int row_bytes = kD * es;
     const int vpr = row_bytes / 16;
-    const int per = (a.topk + nsp - 1) / nsp;
-    const int r_beg = min(a.topk, sp * per), r_end = min(a.topk, r_beg + per);
+    // the pair's rows: the topk selected ids, then the dlen dense rows
+    const int nrows = a.topk + a.dlen;
+    const int per = (nrows + nsp - 1) / nsp;
+    const int r_beg = min(nrows, sp * per), r_end = min(nrows, r_beg + per);
 
     const int64_t qbase = ((int64_t)b_seq * a.H * G + (int64_t)h * G) * kD;
     for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][i % kD] = ld_as_f32(a.q, qbase + i, a.is_bf16);
@@ -67,6 +72,8 @@ __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
     pdl_wait();                                   // the selected ids may come from the search
     const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + (size_t)bh * a.stride * row_bytes;
     const unsigned char *Vb = reinterpret_cast<const unsigned char *>(a.V) + (size_t)bh * a.stride * row_bytes;
+    const unsigned char *dKb = a.dlen ? reinterpret_cast<const unsigned char *>(a.dK) + (size_t)bh * a.dstride * row_bytes : nullptr;
+    const unsigned char *dVb = a.dlen ? reinterpret_cast<const unsigned char *>(a.dV) + (size_t)bh * a.dstride * row_bytes : nullptr;
     const int d = tid & (kD - 1);
     const int gsel = tid >> 7;
     float acc[kMaxGroup / 2];
@@ -76,11 +83,18 @@ __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
     for (int t0 = r_beg; t0 < r_end; t0 += kAtRows) {
         const int rows = min(kAtRows, r_end - t0);
         __syncthreads();                                  // previous tile fully consumed
+        // row slot code: a selected id (>= 0), -1 (id out of range: skipped),
+        // or -2 - j for dense row j
         if (tid < rows) {
-            const int32_t id = a.idx[(size_t)bh * a.topk + t0 + tid];
-            const bool ok = id >= 0 && (int64_t)id < a.n;
-            if (!ok) devchk(a.dev_err, a.dev_err_detail, DEVCHK_BAD_INDEX, id);
-            s_idx[tid] = ok ? id : -1;
+            const int rr = t0 + tid;
+            if (rr < a.topk) {
+                const int32_t id = a.idx[(size_t)bh * a.topk + rr];
+                const bool ok = id >= 0 && (int64_t)id < a.n;
+                if (!ok) devchk(a.dev_err, a.dev_err_detail, DEVCHK_BAD_INDEX, id);
+                s_idx[tid] = ok ? id : -1;
+            } else {
+                s_idx[tid] = -2 - (rr - a.topk);
+            }
         }
         __syncthreads();
         // ---- gather: every load of the tile in flight at once
@@ -96,6 +110,10 @@ __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
                 if (id >= 0) {
                     kr[u] = *reinterpret_cast<const uint4 *>(Kb + (size_t)id * row_bytes + 16 * c);
                     vr[u] = *reinterpret_cast<const uint4 *>(Vb + (size_t)id * row_bytes + 16 * c);
+                } else if (id <= -2) {
+                    const size_t j = (size_t)(-2 - id);
+                    kr[u] = *reinterpret_cast<const uint4 *>(dKb + j * row_bytes + 16 * c);
+                    vr[u] = *reinterpret_cast<const uint4 *>(dVb + j * row_bytes + 16 * c);
                 }
             }
         }
@@ -124,7 +142,7 @@ __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
                           kx[2] * s_q[g][4 * lane + 2] + kx[3] * s_q[g][4 * lane + 3];
 #pragma unroll
                 for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
-                if (lane == 0) s_p[g][r] = (s_idx[r] >= 0) ? s * a.scale : -INFINITY;
+                if (lane == 0) s_p[g][r] = (s_idx[r] != -1) ? s * a.scale : -INFINITY;
             }
         }
         __syncthreads();

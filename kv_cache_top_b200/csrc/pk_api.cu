@@ -386,6 +386,45 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     return cuda_status(e);
 }
 
+pk_status attend_impl(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t topk, const void *dK,
+                      const void *dV, int64_t dstride, int32_t dlen, float *out, cudaStream_t s)
+{
+    if (!ix || !q || !out) return PK_ERR_INVALID_ARG;
+    if (topk < 0 || topk > ix->topk_cap || dlen < 0 || topk + (int64_t)dlen < 1) return PK_ERR_INVALID_ARG;
+    if (topk > 0 && (!sel_idx || !device_accessible(sel_idx) || !aligned(sel_idx, 4))) return PK_ERR_INVALID_ARG;
+    if (!device_accessible(q) || !device_accessible(out)) return PK_ERR_INVALID_ARG;
+    if (!aligned(q, ix->es) || !aligned(out, 4)) return PK_ERR_INVALID_ARG;
+    if (dlen > 0) {   // dense rows are read 16 bytes at a time
+        if (!dK || !dV || dstride < dlen || !device_accessible(dK) || !device_accessible(dV) ||
+            !aligned(dK, 16) || !aligned(dV, 16))
+            return PK_ERR_INVALID_ARG;
+    }
+    AttendArgs a{};
+    a.dK = dK;
+    a.dV = dV;
+    a.dstride = dstride;
+    a.dlen = dlen;
+    a.q = q;
+    a.idx = sel_idx;
+    a.K = ix->K;
+    a.V = ix->V;
+    a.out = out;
+    a.n = ix->n;
+    a.stride = ix->stride;
+    a.H = ix->p.n_kv_heads;
+    a.G = ix->p.group;
+    a.topk = topk;
+    a.is_bf16 = ix->p.kv_dtype == PK_BF16;
+    a.scale = ix->scale;
+    a.nsplit = splitting(ix, topk + dlen);
+    a.dev_err = ix->dev_err;
+    a.dev_err_detail = ix->dev_err_detail;
+    trace_begin(ix, PK_K_GATHER_ATTEND, s);
+    cudaError_t e = launch_gather_attend(a, ix->bh, s);
+    trace_end(ix, s);
+    return cuda_status(e);
+}
+
 }  // namespace
 
 // ======================================================================
@@ -583,32 +622,16 @@ pk_status pk_search_debug(pk_index *ix, const void *q, int32_t topk, int32_t *ou
 pk_status pk_attend(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t topk, float *out,
                     void *stream)
 {
-    if (!ix || !q || !sel_idx || !out) return PK_ERR_INVALID_ARG;
-    if (topk < 1 || topk > ix->topk_cap) return PK_ERR_INVALID_ARG;
-    if (!device_accessible(q) || !device_accessible(sel_idx) || !device_accessible(out))
-        return PK_ERR_INVALID_ARG;
-    if (!aligned(q, ix->es) || !aligned(sel_idx, 4) || !aligned(out, 4)) return PK_ERR_INVALID_ARG;
-    AttendArgs a{};
-    a.q = q;
-    a.idx = sel_idx;
-    a.K = ix->K;
-    a.V = ix->V;
-    a.out = out;
-    a.n = ix->n;
-    a.stride = ix->stride;
-    a.H = ix->p.n_kv_heads;
-    a.G = ix->p.group;
-    a.topk = topk;
-    a.is_bf16 = ix->p.kv_dtype == PK_BF16;
-    a.scale = ix->scale;
-    a.nsplit = splitting(ix, topk);
-    a.dev_err = ix->dev_err;
-    a.dev_err_detail = ix->dev_err_detail;
-    cudaStream_t s = (cudaStream_t)stream;
-    trace_begin(ix, PK_K_GATHER_ATTEND, s);
-    cudaError_t e = launch_gather_attend(a, ix->bh, s);
-    trace_end(ix, s);
-    return cuda_status(e);
+    if (topk < 1) return PK_ERR_INVALID_ARG;
+    return attend_impl(ix, q, sel_idx, topk, nullptr, nullptr, 0, 0, out, (cudaStream_t)stream);
+}
+
+pk_status pk_attend_dense(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t topk,
+                          const void *dense_K, const void *dense_V, int64_t dense_stride,
+                          int32_t dense_len, float *out, void *stream)
+{
+    return attend_impl(ix, q, sel_idx, topk, dense_K, dense_V, dense_stride, dense_len, out,
+                       (cudaStream_t)stream);
 }
 
 void pk_free(pk_index *ix)

@@ -122,6 +122,11 @@ struct AttendArgs {
     float scale;
     int32_t *dev_err;
     long long *dev_err_detail;
+    // dense rows kept outside the index (sink and local tokens), attended
+    // under the same softmax: [BH][dstride][D] kv_dtype, rows 0..dlen-1
+    const void *dK, *dV;
+    int64_t dstride;
+    int32_t dlen;
 };
 
 struct MergeArgs {

@@ -232,6 +232,21 @@ def attend(q, K, V, idx, scale: float):
     return o
 
 
+def attend_union(q, K, V, idx, Kd, Vd, scale: float):
+    """Attention of q [G][D] over the selected rows idx of (K, V) together
+    with every row of the dense set (Kd, Vd) [m][D] -- the sink and local
+    tokens kept on the GPU -- under one softmax (README, step 3: attention
+    over sink, local and retrieved tokens; slides, Fig. 5).  The union of
+    the two row sets is attended by `attend` above."""
+    K = _c(K, np.float32)
+    Kd = _c(np.reshape(Kd, (-1, K.shape[1])), np.float32)
+    Vd = _c(np.reshape(Vd, (-1, K.shape[1])), np.float32)
+    Ku = np.concatenate([K, Kd])
+    Vu = np.concatenate([_c(V, np.float32), Vd])
+    idx_u = np.concatenate([np.asarray(idx, np.int64), K.shape[0] + np.arange(Kd.shape[0])])
+    return attend(q, Ku, Vu, idx_u, scale)
+
+
 def ratio_table(n: int):
     b = np.empty(1, np.float64)
     r = np.empty(1, np.float64)

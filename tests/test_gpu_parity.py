@@ -230,6 +230,65 @@ def test_drift_stream_append_then_search(pk):
         pk.pk_free(h)
 
 
+@pytest.mark.parametrize("kind,topk,dlen,kv_location", [
+    ("llama", 100, 80, 0),      # 16 sink + 64 local rows beside the Top-100
+    ("llama", 0, 80, 0),        # dense rows only
+    ("llama", 100, 80, 1),      # index K/V in pinned host memory, dense rows on the GPU
+    ("tiny", 100, 33, 0),       # fp32 rows, ragged dense count
+])
+def test_attend_with_dense_rows(pk, kind, topk, dlen, kv_location):
+    """pk_attend_dense: the selected rows and the caller's dense (sink +
+    local) rows under one softmax, against the oracle's attention over the
+    union of the two row sets; with no dense rows it is pk_attend."""
+    if kind == "tiny":
+        w = workloads.tiny(seed=1, device="cuda")
+        batch, H, G, n = 1, 1, 1, 4096
+        q = w["q"][5]
+        cand = 512
+    else:
+        batch, H, G, n = 2, 2, 4, 20000
+        w = workloads.llama_layer(batch, n, H=H, G=G, seed=41, device="cuda")
+        q = w["q"][0]
+        cand = 0
+    h = build(pk, w["K"], w["V"], n, batch, H, G, cand_budget=cand, kv_location=kv_location)
+    try:
+        BH = batch * H
+        g = torch.Generator(device="cuda").manual_seed(5)
+        dstride = dlen + 16
+        dK = torch.randn(batch, H, dstride, 128, generator=g, device="cuda").to(w["K"].dtype)
+        dV = torch.randn(batch, H, dstride, 128, generator=g, device="cuda").to(w["K"].dtype)
+        idx = torch.empty(BH, 100, dtype=torch.int32, device="cuda")
+        pk.pk_search(h, q, 100, idx)
+        out = torch.full((batch, H * G, 128), float("nan"), dtype=torch.float32, device="cuda")
+        pk.pk_attend_dense(h, q, idx if topk else None, topk, dK, dV, dlen, out)
+        out0 = torch.empty_like(out)
+        out1 = torch.empty_like(out)
+        pk.pk_attend_dense(h, q, idx, 100, dK, dV, 0, out0)
+        pk.pk_attend(h, q, idx, 100, out1)
+        torch.cuda.synchronize()
+        st, det = pk.pk_last_device_error(h)
+        assert st == 0, (st, det)
+        assert torch.equal(out0, out1)
+        o = out.cpu().numpy()
+        ids = idx.cpu().numpy()
+        tol = 1e-4 if kind == "tiny" else parity.ATTN_ABS
+        for p in range(BH):
+            b, hh = divmod(p, H)
+            qg = workloads.to_np_f32(q[b, hh * G:(hh + 1) * G])
+            ref = parity.oracle.attend_union(qg, workloads.to_np_f32(w["K"][b, hh, :n]),
+                                             workloads.to_np_f32(w["V"][b, hh, :n]), ids[p][:topk],
+                                             workloads.to_np_f32(dK[b, hh, :dlen]),
+                                             workloads.to_np_f32(dV[b, hh, :dlen]), 1.0 / math.sqrt(128))
+            assert np.abs(o[b, hh * G:(hh + 1) * G] - ref).max() <= tol
+        with pytest.raises(pk.PkError):          # nothing to attend
+            pk.pk_attend_dense(h, q, None, 0, dK, dV, 0, out)
+        mis = torch.empty(dK.numel() + 8, dtype=dK.dtype, device="cuda")[1:1 + dK.numel()].view(dK.shape)
+        with pytest.raises(pk.PkError):          # dense rows not 16-byte aligned
+            pk.pk_attend_dense(h, q, idx, 100, mis, dV, dlen, out)
+    finally:
+        pk.pk_free(h)
+
+
 def test_host_pinned_kv_store(pk):
     """K/V kept in pinned host memory and read through UVA by the attention."""
     w = workloads.llama_layer(1, 20000, H=2, G=4, seed=3, device="cuda")

@@ -441,6 +441,39 @@ def test_attention_full_selection_equals_dense_attention():
     np.testing.assert_allclose(o, ref, atol=1e-12)
 
 
+def test_attention_over_selected_and_dense_rows():
+    """Sink/local rows kept outside the index join the retrieved rows under
+    one softmax: with no dense rows it is the selected-row attention, with no
+    selected rows it is attention over the dense rows, moving a row between
+    the two sets changes nothing, and the result is torch's attention over
+    the union of rows (fp64)."""
+    rng = np.random.default_rng(23)
+    n, m, k = 500, 40, 60
+    K = rng.standard_normal((n, D)).astype(np.float32)
+    V = rng.standard_normal((n, D)).astype(np.float32)
+    Kd = rng.standard_normal((m, D)).astype(np.float32)
+    Vd = rng.standard_normal((m, D)).astype(np.float32)
+    q = rng.standard_normal((4, D)).astype(np.float32)
+    idx = rng.choice(n, k, replace=False).astype(np.int32)
+    sc = 1.0 / math.sqrt(D)
+    o = oracle.attend_union(q, K, V, idx, Kd, Vd, sc)
+    np.testing.assert_array_equal(oracle.attend_union(q, K, V, idx, Kd[:0], Vd[:0], sc),
+                                  oracle.attend(q, K, V, idx, sc))
+    np.testing.assert_allclose(oracle.attend_union(q, K, V, idx[:0], Kd, Vd, sc),
+                               oracle.attend(q, Kd, Vd, np.arange(m), sc), atol=1e-14)
+    # move selected row idx[0] into the dense set
+    o2 = oracle.attend_union(q, K, V, idx[1:], np.concatenate([Kd, K[idx[:1]]]),
+                             np.concatenate([Vd, V[idx[:1]]]), sc)
+    np.testing.assert_allclose(o, o2, atol=1e-14)
+    Ku = np.concatenate([K[idx], Kd])
+    Vu = np.concatenate([V[idx], Vd])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).double()[None, :, None, :],
+        torch.from_numpy(Ku).double()[None, None].expand(1, 4, k + m, D),
+        torch.from_numpy(Vu).double()[None, None].expand(1, 4, k + m, D))[0, :, 0, :].numpy()
+    np.testing.assert_allclose(o, ref, atol=1e-12)
+
+
 # ------------------------------------------------------------ parameters
 def test_ratio_table_golden(golden):
     for ln in golden("ratio_table.txt"):
