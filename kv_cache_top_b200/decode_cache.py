@@ -1,0 +1,115 @@
+"""Sink / local / update-buffer layout for long decoding.
+
+ParisKV keeps recent tokens dense while older tokens are indexed and
+offloaded (README, "Long-generation support": a sink/local/update-buffer
+layout; slides, Fig. 5: sink and recent local tokens stay on the GPU for
+dense attention, new tokens enter an update buffer, and a full buffer
+triggers encoding and offload of the oldest local tokens; attention runs over
+sink, local and retrieved tokens).  This module is that policy, written on
+the library's C-ABI (pk_build_index, pk_append, pk_search, pk_attend_dense):
+encoding, retrieval and attention run in the library's kernels; the buffer
+bookkeeping (placing a new token in the dense buffer, moving the tail after
+re-indexing) is plain tensor copies.
+
+Positions 0 .. T-1 of every (sequence, KV head) pair are split into
+  sink             [0, sink)             kept on the GPU, attended densely;
+  retrieval zone   [sink, z)             in the ParisKV index (codes and
+                                         records on the GPU, K/V in the index
+                                         store -- pinned host memory when
+                                         offloaded); searched for the Top-k;
+  dense tail       [z, T)                kept on the GPU, attended densely.
+The tail holds between `local` and `local + update` tokens.  When a new token
+would make it longer, its oldest `update` tokens are encoded into the index
+with one pk_append, and the zone grows by `update`.  Where the pages leave
+the boundary rule open, this is the reading: re-indexing moves exactly
+`update` tokens at a time and never lets the tail drop below `local`.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (PK_BF16, PK_F32, PK_KV_DEVICE, PK_KV_HOST_PINNED, pk_append, pk_attend_dense,
+               pk_build_index, pk_default_params, pk_free, pk_get_info, pk_search)
+
+
+class DecodeCache:
+    """K, V: the prefill [batch][H][T0][D] (bf16 or fp32, on the GPU).
+    sink, local, update: the layout sizes (pages: sink 4-64, local 256-512,
+    update interval 256-512).  max_len: the largest T the cache will see
+    (sizes the index).  The index is built over [sink, T0 - local), which
+    must hold at least `topk` tokens."""
+
+    def __init__(self, K, V, *, group: int, sink: int = 64, local: int = 512, update: int = 512,
+                 max_len: int, topk: int = 100, offload: bool = False, **params):
+        assert K.dim() == 4 and K.shape == V.shape and K.shape[-1] == 128
+        self.batch, self.H, T0, D = K.shape
+        self.G, self.sink, self.local, self.update, self.topk = group, sink, local, update, topk
+        if T0 - sink - local < max(1, topk):
+            raise ValueError("the prefill must be longer than sink + local + topk tokens")
+        self.dtype = K.dtype
+        z = T0 - local                                    # zone end
+        p = pk_default_params(batch=self.batch, n_kv_heads=self.H, group=group, topk=topk,
+                              n_cap=max(max_len - sink - local, z - sink),
+                              kv_dtype=PK_BF16 if K.dtype == torch.bfloat16 else PK_F32,
+                              kv_location=PK_KV_HOST_PINNED if offload else PK_KV_DEVICE, **params)
+        self.index = pk_build_index(K[:, :, sink:z].contiguous(), V[:, :, sink:z].contiguous(), z - sink, p)
+        cap = sink + local + update
+        self.dK = torch.zeros(self.batch, self.H, cap, D, dtype=K.dtype, device=K.device)
+        self.dV = torch.zeros_like(self.dK)
+        self.dK[:, :, :sink] = K[:, :, :sink]
+        self.dV[:, :, :sink] = V[:, :, :sink]
+        self.dK[:, :, sink:sink + local] = K[:, :, z:]
+        self.dV[:, :, sink:sink + local] = V[:, :, z:]
+        self.tail = local                                 # dense tail length
+        self.T = T0
+        self.zone_end = z
+        self.reindexed = 0
+        self.idx = torch.empty(self.batch * self.H, topk, dtype=torch.int32, device=K.device)
+        self.out = torch.empty(self.batch, self.H * group, D, dtype=torch.float32, device=K.device)
+
+    @property
+    def zone(self):
+        """(start, end) positions of the retrieval zone."""
+        return self.sink, self.zone_end
+
+    def _reindex(self):
+        s, u = self.sink, self.update
+        pk_append(self.index, self.dK[:, :, s:s + u].contiguous(), self.dV[:, :, s:s + u].contiguous(), u)
+        rest = self.tail - u
+        self.dK[:, :, s:s + rest] = self.dK[:, :, s + u:s + self.tail].clone()
+        self.dV[:, :, s:s + rest] = self.dV[:, :, s + u:s + self.tail].clone()
+        self.tail = rest
+        self.zone_end += u
+        self.reindexed += 1
+
+    def step(self, q, k_new, v_new):
+        """One decode step: add the new token k_new, v_new [batch][H][1][D] to
+        the dense tail (re-indexing first when the buffer is full), retrieve
+        the zone's Top-k for q [batch][H*G][D], and attend over sink + tail +
+        retrieved rows.  Returns the attention output [batch][H*G][D] fp32
+        (a buffer reused by the next step).  Everything runs on torch's current
+        stream, in order."""
+        if self.tail == self.local + self.update:
+            self._reindex()
+        r = self.sink + self.tail
+        self.dK[:, :, r:r + 1] = k_new
+        self.dV[:, :, r:r + 1] = v_new
+        self.tail += 1
+        self.T += 1
+        pk_search(self.index, q, self.topk, self.idx)
+        pk_attend_dense(self.index, q, self.idx, self.topk, self.dK, self.dV, self.sink + self.tail, self.out)
+        return self.out
+
+    def close(self):
+        if self.index is not None:
+            pk_free(self.index)
+            self.index = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def info(self):
+        return pk_get_info(self.index)

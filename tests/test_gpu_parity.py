@@ -289,6 +289,53 @@ def test_attend_with_dense_rows(pk, kind, topk, dlen, kv_location):
         pk.pk_free(h)
 
 
+@pytest.mark.parametrize("offload", [False, True])
+def test_decode_cache_sink_local_update(pk, offload):
+    """The sink/local/update-buffer layout over 160 decode steps (sink 16,
+    local 64, update 32; re-indexing every 32 steps): the retrieval zone
+    grows by whole update buffers, the dense tail stays within
+    (local, local + update], the Top-k over the zone matches the oracle's
+    search of the zone, and the output is the oracle's attention over sink +
+    tail + retrieved rows."""
+    from kv_cache_top_b200.decode_cache import DecodeCache
+    T0, steps, H, G = 4096, 160, 2, 2
+    sink, local, update = 16, 64, 32
+    w = workloads.llama_layer(1, T0 + steps, H=H, G=G, seed=77, device="cuda", n_queries=steps)
+    K, V = w["K"], w["V"]
+    cache = DecodeCache(K[:, :, :T0].contiguous(), V[:, :, :T0].contiguous(), group=G, sink=sink, local=local,
+                        update=update, max_len=T0 + steps, offload=offload)
+    try:
+        for t in range(steps):
+            out = cache.step(w["q"][t], K[:, :, T0 + t:T0 + t + 1].contiguous(),
+                             V[:, :, T0 + t:T0 + t + 1].contiguous())
+            if t not in (0, 31, 32, 100, steps - 1):
+                continue
+            torch.cuda.synchronize()
+            T = T0 + t + 1
+            z0, z1 = cache.zone
+            assert z0 == sink and (z1 - (T0 - local)) % update == 0
+            assert cache.info().n == z1 - z0 and cache.tail == T - z1 and local < cache.tail <= local + update
+            idx2 = torch.empty_like(cache.idx)
+            sc2 = torch.empty(H, 100, dtype=torch.float32, device="cuda")
+            pk.pk_search(cache.index, w["q"][t], 100, idx2, sc2)
+            torch.cuda.synchronize()
+            assert torch.equal(idx2, cache.idx)
+            idx, sc, o = idx2.cpu().numpy(), sc2.cpu().numpy(), out.cpu().numpy()
+            for p in range(H):
+                Kz = workloads.to_np_f32(K[0, p, z0:z1])
+                Vz = workloads.to_np_f32(V[0, p, z0:z1])
+                qg = workloads.to_np_f32(w["q"][t][0, p * G:(p + 1) * G])
+                enc, orc = parity.oracle_pair(Kz, qg, 100, 0)
+                parity.check_topk(idx[p], sc[p], orc, enc)
+                Kd = np.concatenate([workloads.to_np_f32(K[0, p, :sink]), workloads.to_np_f32(K[0, p, z1:T])])
+                Vd = np.concatenate([workloads.to_np_f32(V[0, p, :sink]), workloads.to_np_f32(V[0, p, z1:T])])
+                ref = parity.oracle.attend_union(qg, Kz, Vz, idx[p], Kd, Vd, 1.0 / math.sqrt(128))
+                assert np.abs(o[0, p * G:(p + 1) * G] - ref).max() <= parity.ATTN_ABS
+        assert cache.reindexed == 4          # at steps 32, 64, 96 and 128
+    finally:
+        cache.close()
+
+
 def test_host_pinned_kv_store(pk):
     """K/V kept in pinned host memory and read through UVA by the attention."""
     w = workloads.llama_layer(1, 20000, H=2, G=4, seed=3, device="cuda")
