@@ -11,7 +11,7 @@ budgets.  The line also carries the metric's 1M point (n = 1048576, 8 KV
 heads, K/V in pinned host memory read through UVA) under "million_token".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload throughput|million|llama|tiny|drift|sweep] [--no-million]
+                  [--workload throughput|million|llama|tiny|drift|sweep|longgen] [--no-million]
                   [--no-cpu-baseline] [--no-e2e] [--no-dense] [--graph] [--drift-steps T]
 
 For N > 1 launch under torch.distributed.run: every rank runs its own copy of
@@ -49,6 +49,9 @@ WORKLOADS = {
     "sweep": dict(name="ratio_sweep", batch=1, n=0, H=8, G=4, cand=0, kv_host=False,
                   ns=(32768, 131072, 524288, 1048576), betas=(0.02, 0.05, 0.1, 0.2),
                   rhos=(0.05, 0.1, 0.2, 0.35, 0.5), queries=8),
+    # sink / local / update-buffer decoding after an 8 x 131072 prefill
+    "longgen": dict(name="longgen_8x131072+1024", batch=8, n=131072, H=8, G=4, cand=0, kv_host=False,
+                    steps=1024, sink=64, local=512, update=512),
     # prefill 65536 keys per KV head, then 16384 decode steps of append + search
     "drift": dict(name="drift_65536+16384", batch=1, n=65536, H=8, G=1, cand=0, kv_host=False,
                   steps=16384, recall_every=256),
@@ -529,6 +532,10 @@ def main():
         if world > 1:
             raise SystemExit("the drift mode runs on one GPU")
         return run_drift(args, wl, peak)
+    if args.workload == "longgen":
+        if world > 1:
+            raise SystemExit("the long-generation mode runs on one GPU")
+        return run_longgen(args, wl)
     if args.workload == "sweep":
         if world > 1:
             raise SystemExit("the sweep runs on one GPU")
@@ -667,6 +674,54 @@ def run_drift(args, wl, peaks):
             "recall_at_100_mean": sum(b for _, b in recalls) / max(1, len(recalls)),
             "gpu_launches": None}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------ long generation
+def run_longgen(args, wl):
+    """Decode steps with the sink / local / update-buffer layout: each step
+    adds one token per pair to the dense tail (re-indexing `update` tokens
+    when the buffer is full), retrieves the zone's Top-k and attends over
+    sink + tail + retrieved rows.  CUDA events per step, L2 flushed between
+    steps; steps that re-index are reported apart."""
+    import torch
+    import workloads
+    from kv_cache_top_b200.decode_cache import DecodeCache
+    dev = torch.device("cuda", 0)
+    B, n, H, G, T = wl["batch"], wl["n"], wl["H"], wl["G"], wl["steps"]
+    w = workloads.llama_layer(B, n + T, H=H, G=G, seed=args.seed, device=dev, n_queries=64)
+    K, V, q = w["K"], w["V"], w["q"]
+    cache = DecodeCache(K[:, :, :n].contiguous(), V[:, :, :n].contiguous(), group=G, sink=wl["sink"],
+                        local=wl["local"], update=wl["update"], max_len=n + T)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    toks = [(K[:, :, n + t:n + t + 1].contiguous(), V[:, :, n + t:n + t + 1].contiguous()) for t in range(T)]
+    ev, reidx = [], []
+    for t in range(T):
+        flush.zero_()
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        will = cache.tail == cache.local + cache.update
+        a_.record(stream)
+        cache.step(q[t % 64], *toks[t])
+        b_.record(stream)
+        ev.append((a_, b_))
+        reidx.append(will)
+    torch.cuda.synchronize()
+    ms = [a_.elapsed_time(b_) for a_, b_ in ev]
+    plain = [m for m, r in zip(ms, reidx) if not r]
+    re_ms = [m for m, r in zip(ms, reidx) if r]
+    info = cache.info()
+    cache.close()
+    print(json.dumps({
+        "metric": "decode steps/s with the sink / local / update-buffer layout (retrieval + attention over "
+                  "sink, local and retrieved rows)",
+        "value": T / (sum(ms) / 1000.0), "unit": "steps/s", "n_gpus": 1, "steps": T, "higher_is_better": True,
+        "ms_per_step": sum(ms) / T, "ms_per_step_median": statistics.median(plain),
+        "reindex_steps": len(re_ms), "ms_per_reindex_step": (sum(re_ms) / len(re_ms)) if re_ms else None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl["name"], "batch": B, "prefill": n, "kv_heads": H, "q_heads": H * G,
+                   "sink": wl["sink"], "local": wl["local"], "update": wl["update"], "topk": 100,
+                   "zone_keys_at_end": info.n, "l2": "flushed between steps (outside the events)"}}),
+          flush=True)
 
 
 # ------------------------------------------------------------ ratio sweep
