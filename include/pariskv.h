@@ -188,6 +188,25 @@ pk_status pk_attend_dense(pk_index *index, const void *q, const int32_t *sel_idx
                           const void *dense_K, const void *dense_V, int64_t dense_stride,
                           int32_t dense_len, float *out, void *stream);
 
+/* Per-query-head retrieval for GQA: every query head of a pair searches the
+ * pair's index with its own query (no aggregation): its own bonus tables,
+ * collision scores, candidates and Top-k.  The pages retrieve with one query
+ * per KV head; this is the other reading of a GQA group, kept beside it to
+ * compare recall and cost.
+ *   q        [batch][H*G][D] kv_dtype.
+ *   out_idx  [batch][H*G][topk] i32 device: key ids of the pair's index,
+ *            best first for each query head; out_score likewise or NULL.
+ * The first call allocates a workspace for batch*H*G query units (kept
+ * until pk_free).  Errors as pk_search, and PK_ERR_OOM for that workspace. */
+pk_status pk_search_heads(pk_index *index, const void *q, int32_t topk, int32_t *out_idx,
+                          float *out_score, void *stream);
+
+/* Attention of every query head over its own selected rows (as returned by
+ * pk_search_heads): sel_idx [batch][H*G][topk] i32 device; out as for
+ * pk_attend.  Errors as pk_attend. */
+pk_status pk_attend_heads(pk_index *index, const void *q, const int32_t *sel_idx, int32_t topk,
+                          float *out, void *stream);
+
 /* Free everything the index owns (synchronises the device first). NULL is ok. */
 void pk_free(pk_index *index);
 

@@ -37,7 +37,8 @@ __all__ = [
     "PkError", "pk_default_params", "pk_build_index", "pk_append", "pk_search", "pk_search_debug",
     "pk_attend", "pk_free", "pk_status_str", "pk_last_device_error", "pk_get_info",
     "pk_export_index", "pk_magnitude_levels", "pk_resolve", "pk_trace_enable", "pk_trace_read",
-    "pk_select_candidates_noalloc", "pk_attend_dense", "pk_params", "pk_info", "pk_debug_out", "PK_F32", "PK_BF16", "PK_KV_DEVICE",
+    "pk_select_candidates_noalloc", "pk_attend_dense", "pk_search_heads", "pk_attend_heads",
+    "pk_params", "pk_info", "pk_debug_out", "PK_F32", "PK_BF16", "PK_KV_DEVICE",
     "PK_KV_HOST_PINNED", "KERNELS", "lib",
 ]
 
@@ -121,6 +122,18 @@ def pk_attend_dense(index, q, sel_idx, topk: int, dense_K, dense_V, dense_len: i
     dstride = dense_K.shape[-2] if dense_K is not None and hasattr(dense_K, "shape") else 0
     _check(_L().pk_attend_dense(index, _ptr(q), _ptr(sel_idx), int(topk), _ptr(dense_K), _ptr(dense_V),
                                 int(dstride), int(dense_len), _ptr(out), _stream(stream)), "pk_attend_dense")
+
+
+def pk_search_heads(index, q, topk: int, out_idx, out_score=None, stream=None):
+    """Per-query-head retrieval: out_idx [batch][H*G][topk]."""
+    _check(_L().pk_search_heads(index, _ptr(q), int(topk), _ptr(out_idx), _ptr(out_score), _stream(stream)),
+           "pk_search_heads")
+
+
+def pk_attend_heads(index, q, sel_idx, topk: int, out, stream=None):
+    """Attention of every query head over its own rows sel_idx [batch][H*G][topk]."""
+    _check(_L().pk_attend_heads(index, _ptr(q), _ptr(sel_idx), int(topk), _ptr(out), _stream(stream)),
+           "pk_attend_heads")
 
 
 def pk_free(index):

@@ -15,7 +15,7 @@ EXPORTS = (
     "pk_default_params", "pk_build_index", "pk_append", "pk_search", "pk_search_debug",
     "pk_attend", "pk_free", "pk_status_str", "pk_last_device_error", "pk_get_info",
     "pk_export_index", "pk_magnitude_levels", "pk_resolve", "pk_trace_enable", "pk_trace_read",
-    "pk_select_candidates_noalloc", "pk_attend_dense",
+    "pk_select_candidates_noalloc", "pk_attend_dense", "pk_search_heads", "pk_attend_heads",
 )
 
 PK_OK, PK_ERR_INVALID_ARG, PK_ERR_CAPACITY, PK_ERR_OOM, PK_ERR_CUDA, PK_ERR_TIMEOUT, \
@@ -72,6 +72,10 @@ def load() -> C.CDLL:
     lib.pk_search_debug.argtypes = [P, P, I32, P, P, C.POINTER(pk_debug_out), P]
     lib.pk_attend.restype = st
     lib.pk_attend.argtypes = [P, P, P, I32, P, P]
+    lib.pk_search_heads.restype = st
+    lib.pk_search_heads.argtypes = [P, P, I32, P, P, P]
+    lib.pk_attend_heads.restype = st
+    lib.pk_attend_heads.argtypes = [P, P, P, I32, P, P]
     lib.pk_attend_dense.restype = st
     lib.pk_attend_dense.argtypes = [P, P, P, I32, P, P, I64, I32, P, P]
     lib.pk_free.restype = None

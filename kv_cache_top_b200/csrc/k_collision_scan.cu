@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
     const int64_t lo = (int64_t)chunk * a.chunk;
     const int64_t hi = min(lo + a.chunk, a.n);
     const int64_t cnt = hi - lo;
-    const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes + ((size_t)bh * a.n_cap + lo) * kB);
+    const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes + ((size_t)index_pair(bh, a.kvg) * a.n_cap + lo) * kB);
     uint8_t *S = a.S + (size_t)bh * a.n_cap + lo;
     uint8_t *dS = a.dbg_S ? a.dbg_S + (size_t)bh * a.n + lo : nullptr;
 

@@ -70,10 +70,11 @@ __global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
         s_l[tid] = 0.0f;
     }
     pdl_wait();                                   // the selected ids may come from the search
-    const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + (size_t)bh * a.stride * row_bytes;
-    const unsigned char *Vb = reinterpret_cast<const unsigned char *>(a.V) + (size_t)bh * a.stride * row_bytes;
-    const unsigned char *dKb = a.dlen ? reinterpret_cast<const unsigned char *>(a.dK) + (size_t)bh * a.dstride * row_bytes : nullptr;
-    const unsigned char *dVb = a.dlen ? reinterpret_cast<const unsigned char *>(a.dV) + (size_t)bh * a.dstride * row_bytes : nullptr;
+    const size_t kp = (size_t)index_pair(bh, a.kvg);     // the index pair holding this unit's rows
+    const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + kp * a.stride * row_bytes;
+    const unsigned char *Vb = reinterpret_cast<const unsigned char *>(a.V) + kp * a.stride * row_bytes;
+    const unsigned char *dKb = a.dlen ? reinterpret_cast<const unsigned char *>(a.dK) + kp * a.dstride * row_bytes : nullptr;
+    const unsigned char *dVb = a.dlen ? reinterpret_cast<const unsigned char *>(a.dV) + kp * a.dstride * row_bytes : nullptr;
     const int d = tid & (kD - 1);
     const int gsel = tid >> 7;
     float acc[kMaxGroup / 2];

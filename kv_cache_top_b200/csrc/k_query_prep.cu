@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(kQpThreads) k_query_prep(PrepArgs a)
         if (tid < 2) a.tickets[(size_t)bh * 2 + tid] = 0u;
     }
     // global loads: 2 bucket sizes per thread; warp 0 the G query heads
-    const uint32_t *occ = a.occ + ((size_t)bh * kB + b) * kNC;
+    const uint32_t *occ = a.occ + ((size_t)index_pair(bh, a.kvg) * kB + b) * kNC;
     const uint32_t o0 = occ[t], o1 = occ[t + kQpHalf];
     if (warp == 0) {
         float qv[4][kMaxGroup];

@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
 #pragma unroll
     for (int i = 0; i < 32; i++) qr[i] = a.qt[(size_t)bh * kD + 32 * q4 + i];
     const float qnorm = a.qnorm[bh];
-    const uint8_t *rec = a.rec + (size_t)bh * a.stride * kRecBytes;
+    const uint8_t *rec = a.rec + (size_t)index_pair(bh, a.kvg) * a.stride * kRecBytes;
     float *dest = a.dbg_est ? a.dbg_est + (size_t)bh * a.C + m0 : nullptr;
     __syncthreads();
 

@@ -15,6 +15,21 @@ struct TraceRec {
     cudaEvent_t a, b;
 };
 
+// Search workspace for `units` query units: one per pair for the aggregated
+// query, G per pair for per-query-head search.
+struct Work {
+    int32_t units = 0;
+    int32_t max_chunks = 1, max_slices = 1;
+    float *qt = nullptr, *qnorm = nullptr;
+    uint32_t *bonus_packed = nullptr;
+    uint8_t *S = nullptr;
+    uint32_t *chunk_cum = nullptr, *head_hist = nullptr, *tickets = nullptr;
+    uint2 *chunk_info = nullptr;
+    int32_t *sstar = nullptr;
+    int32_t *cand = nullptr;
+    unsigned long long *partial = nullptr;
+};
+
 struct pk_index {
     pk_params p;
     int32_t bh = 0;
@@ -22,7 +37,6 @@ struct pk_index {
     int64_t stride = 0;          // rows per pair in every per-key array (n_cap rounded up to 16)
     int device = 0;
     int num_sms = 148;
-    int32_t max_chunks = 1;
     int32_t topk_cap = 100;
     int es = 2;
     float scale = 0.0f;
@@ -35,16 +49,9 @@ struct pk_index {
     // K/V store (device, or mapped pinned host)
     void *K = nullptr, *V = nullptr;
     bool kv_host = false;
-    // search workspace (device)
-    float *qt = nullptr, *qnorm = nullptr;
-    uint32_t *bonus_packed = nullptr;
-    uint8_t *S = nullptr;
-    uint32_t *chunk_cum = nullptr, *head_hist = nullptr, *tickets = nullptr;
-    uint2 *chunk_info = nullptr;
-    int32_t *sstar = nullptr;
-    int32_t *cand = nullptr;
-    unsigned long long *partial = nullptr;
-    int32_t max_slices = 1;
+    // search workspaces (device): w for the aggregated query, wh for
+    // per-query-head search (made on first use)
+    Work w, wh;
 
     int32_t *dev_err = nullptr;
     long long *dev_err_detail = nullptr;
@@ -120,12 +127,12 @@ uint64_t splitmix64(uint64_t x)
 // Key chunks of the scan and the compaction: at most one wave (4 resident
 // CTAs per SM) when the chunk-size cap allows, never fewer than
 // ceil(n / kMaxChunk) chunks.
-void chunking(const pk_index *ix, int64_t n, int32_t *nchunks, int64_t *chunk)
+void chunking(const pk_index *ix, const Work &w, int64_t n, int32_t *nchunks, int64_t *chunk)
 {
-    int64_t nch = std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / ix->bh);
+    int64_t nch = std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / w.units);
     nch = std::min<int64_t>(nch, ceil_div(n, kMinChunk));
     nch = std::max<int64_t>(nch, ceil_div(n, kMaxChunk));
-    nch = std::max<int64_t>(1, std::min<int64_t>(nch, ix->max_chunks));
+    nch = std::max<int64_t>(1, std::min<int64_t>(nch, w.max_chunks));
     int64_t ch = ceil_div(ceil_div(n, nch), 16) * 16;
     *chunk = ch;
     *nchunks = (int32_t)ceil_div(n, ch);
@@ -134,10 +141,10 @@ void chunking(const pk_index *ix, int64_t n, int32_t *nchunks, int64_t *chunk)
 // rerank work split: slices of the candidate list, ~3 CTAs per SM in total
 int32_t slice_lo(const pk_index *ix) { return std::max<int32_t>(256, 2 * ix->topk_cap); }
 
-void slicing(const pk_index *ix, int64_t C, int32_t *slice, int32_t *nslices)
+void slicing(const pk_index *ix, const Work &w, int64_t C, int32_t *slice, int32_t *nslices)
 {
     // at most one wave (2 resident CTAs per SM) unless the slice-size cap forces more
-    int64_t ns = std::max<int64_t>(1, (2 * (int64_t)ix->num_sms) / ix->bh);
+    int64_t ns = std::max<int64_t>(1, (2 * (int64_t)ix->num_sms) / w.units);
     ns = std::max<int64_t>(ns, ceil_div(C, kMaxSlice));
     int64_t sl = ceil_div(ceil_div(C, ns), 64) * 64;
     sl = std::max<int64_t>(sl, slice_lo(ix));
@@ -147,12 +154,67 @@ void slicing(const pk_index *ix, int64_t C, int32_t *slice, int32_t *nslices)
 }
 
 // attention work split: one cluster of up to 8 CTAs per pair, ~2 CTAs per SM
-int32_t splitting(const pk_index *ix, int32_t topk)
+int32_t splitting(const pk_index *ix, int32_t units, int32_t topk)
 {
-    int64_t ns = ceil_div(2 * (int64_t)ix->num_sms, ix->bh);
+    int64_t ns = ceil_div(2 * (int64_t)ix->num_sms, units);
     ns = std::max<int64_t>(1, std::min<int64_t>(ns, 8));
     ns = std::min<int64_t>(ns, topk);
     return (int32_t)ns;
+}
+
+void work_free(Work &w)
+{
+    cudaFree(w.qt);
+    cudaFree(w.qnorm);
+    cudaFree(w.bonus_packed);
+    cudaFree(w.S);
+    cudaFree(w.chunk_cum);
+    cudaFree(w.head_hist);
+    cudaFree(w.tickets);
+    cudaFree(w.chunk_info);
+    cudaFree(w.sstar);
+    cudaFree(w.cand);
+    cudaFree(w.partial);
+    w = Work{};
+}
+
+template <typename T>
+cudaError_t dalloc(T **p, size_t count);
+
+// Workspace for `units` query units of an index of capacity n_cap; the
+// counters start at zero.  On failure nothing stays allocated.
+cudaError_t work_alloc(pk_index *ix, Work &w, int32_t units, int64_t n_cap, cudaStream_t s)
+{
+    w.units = units;
+    w.max_chunks = (int32_t)std::max<int64_t>(std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / units),
+                                              ceil_div(n_cap, kMaxChunk) + 1);
+    {   // largest slice count any C <= n_cap can need
+        const int64_t lo = slice_lo(ix);
+        const int64_t by_target = std::max<int64_t>(1, (2 * (int64_t)ix->num_sms) / units);
+        w.max_slices = (int32_t)std::max<int64_t>(std::min<int64_t>(ceil_div(n_cap, lo), by_target),
+                                                  ceil_div(n_cap, kMaxSlice)) + 1;
+    }
+    const size_t U = units, NC = ix->stride, MC = w.max_chunks, MS = w.max_slices;
+    cudaError_t e = cudaSuccess;
+    auto chk = [&](cudaError_t x) { if (e == cudaSuccess) e = x; };
+    chk(dalloc(&w.qt, U * kD));
+    chk(dalloc(&w.qnorm, U));
+    chk(dalloc(&w.bonus_packed, U * kB * 32));
+    chk(dalloc(&w.S, U * NC));
+    chk(dalloc(&w.chunk_cum, U * MC * kCum));
+    chk(dalloc(&w.head_hist, U * kBins));
+    chk(dalloc(&w.tickets, U * 2));
+    chk(dalloc(&w.chunk_info, U * MC));
+    chk(dalloc(&w.sstar, U));
+    chk(dalloc(&w.cand, U * NC));
+    chk(dalloc(&w.partial, U * MS * (size_t)ix->topk_cap));
+    chk(cudaMemsetAsync(w.head_hist, 0, U * kBins * sizeof(uint32_t), s));
+    chk(cudaMemsetAsync(w.tickets, 0, U * 2 * sizeof(uint32_t), s));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        work_free(w);
+    }
+    return e;
 }
 
 void free_all(pk_index *ix)
@@ -168,17 +230,8 @@ void free_all(pk_index *ix)
         cudaFree(ix->K);
         cudaFree(ix->V);
     }
-    cudaFree(ix->qt);
-    cudaFree(ix->qnorm);
-    cudaFree(ix->bonus_packed);
-    cudaFree(ix->S);
-    cudaFree(ix->chunk_cum);
-    cudaFree(ix->head_hist);
-    cudaFree(ix->tickets);
-    cudaFree(ix->chunk_info);
-    cudaFree(ix->sstar);
-    cudaFree(ix->cand);
-    cudaFree(ix->partial);
+    work_free(ix->w);
+    work_free(ix->wh);
 
     cudaFree(ix->dev_err);
     cudaFree(ix->dev_err_detail);
@@ -262,8 +315,10 @@ pk_status copy_rows(pk_index *ix, void *store, const void *src, int64_t n_new, i
     return cuda_status(e);
 }
 
-pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_idx, float *out_score,
-                      const pk_debug_out *dbg, cudaStream_t s)
+// One search over work `w`: kvg query units per index pair (1: the
+// aggregated query of each pair; G: every query head of the pair).
+pk_status search_impl(pk_index *ix, Work &w, int32_t kvg, const void *q, int32_t topk, int32_t *out_idx,
+                      float *out_score, const pk_debug_out *dbg, cudaStream_t s)
 {
     if (!ix || !q || !out_idx) return PK_ERR_INVALID_ARG;
     if (topk < 1 || topk > ix->topk_cap) return PK_ERR_INVALID_ARG;
@@ -277,22 +332,23 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     resolve(ix->n, ix->p.cand_budget, ix->p.collision_ratio, topk, &C, &R);
     int32_t nchunks;
     int64_t chunk;
-    chunking(ix, ix->n, &nchunks, &chunk);
+    chunking(ix, w, ix->n, &nchunks, &chunk);
 
     PrepArgs pa{};
     pa.q = q;
-    pa.H = ix->p.n_kv_heads;
-    pa.G = ix->p.group;
+    pa.H = ix->p.n_kv_heads * kvg;        // per-head units: H*G units of one query head each
+    pa.G = ix->p.group / kvg;
+    pa.kvg = kvg;
     pa.is_bf16 = ix->p.kv_dtype == PK_BF16;
-    pa.bh = ix->bh;
+    pa.bh = w.units;
     pa.R = R;
     pa.occ = ix->occ;
     pa.rot = ix->rot;
-    pa.qt = ix->qt;
-    pa.qnorm = ix->qnorm;
-    pa.bonus_packed = ix->bonus_packed;
-    pa.head_hist = ix->head_hist;
-    pa.tickets = ix->tickets;
+    pa.qt = w.qt;
+    pa.qnorm = w.qnorm;
+    pa.bonus_packed = w.bonus_packed;
+    pa.head_hist = w.head_hist;
+    pa.tickets = w.tickets;
     if (dbg) {
         pa.dbg_bonus = dbg->bonus;
         pa.dbg_qt = dbg->qt;
@@ -305,71 +361,73 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
 
     ScanArgs sa{};
     sa.codes = ix->codes;
-    sa.bonus_packed = ix->bonus_packed;
+    sa.bonus_packed = w.bonus_packed;
+    sa.kvg = kvg;
     sa.n = ix->n;
     sa.n_cap = ix->stride;
     sa.chunk = chunk;
     sa.C = C;
     sa.nchunks = nchunks;
-    sa.S = ix->S;
-    sa.chunk_cum = ix->chunk_cum;
-    sa.head_hist = ix->head_hist;
-    sa.tickets = ix->tickets;
-    sa.chunk_info = ix->chunk_info;
-    sa.sstar = ix->sstar;
-    sa.max_chunks = ix->max_chunks;
+    sa.S = w.S;
+    sa.chunk_cum = w.chunk_cum;
+    sa.head_hist = w.head_hist;
+    sa.tickets = w.tickets;
+    sa.chunk_info = w.chunk_info;
+    sa.sstar = w.sstar;
+    sa.max_chunks = w.max_chunks;
     if (dbg) {
         sa.dbg_S = dbg->S;
         sa.dbg_hist = dbg->hist;
         sa.dbg_sstar = dbg->sstar;
     }
     trace_begin(ix, PK_K_COLLISION_SCAN, s);
-    e = launch_collision_scan(sa, ix->bh, s);
+    e = launch_collision_scan(sa, w.units, s);
     trace_end(ix, s);
     if (e != cudaSuccess) return cuda_status(e);
 
     CompactArgs ca{};
-    ca.S = ix->S;
-    ca.chunk_info = ix->chunk_info;
-    ca.sstar = ix->sstar;
+    ca.S = w.S;
+    ca.chunk_info = w.chunk_info;
+    ca.sstar = w.sstar;
     ca.n = ix->n;
     ca.stride = ix->stride;
     ca.chunk = chunk;
     ca.C = C;
-    ca.max_chunks = ix->max_chunks;
+    ca.max_chunks = w.max_chunks;
     ca.groups = (int32_t)ceil_div(chunk, 16 * 256);
-    ca.cand = ix->cand;
+    ca.cand = w.cand;
     ca.dbg_cand = dbg ? dbg->cand : nullptr;
     ca.dev_err = ix->dev_err;
     trace_begin(ix, PK_K_COMPACT, s);
-    e = launch_compact(ca, nchunks, ix->bh, s);
+    e = launch_compact(ca, nchunks, w.units, s);
     trace_end(ix, s);
     if (e != cudaSuccess) return cuda_status(e);
 
     RerankArgs ra{};
-    ra.cand = ix->cand;
+    ra.cand = w.cand;
+    ra.kvg = kvg;
     ra.rec = ix->rec;
-    ra.qt = ix->qt;
-    ra.qnorm = ix->qnorm;
+    ra.qt = w.qt;
+    ra.qnorm = w.qnorm;
     ra.stride = ix->stride;
     ra.C = C;
-    slicing(ix, C, &ra.slice, &ra.nslices);
-    if (ra.nslices > ix->max_slices) return PK_ERR_CAPACITY;
-    ra.max_slices = ix->max_slices;
+    slicing(ix, w, C, &ra.slice, &ra.nslices);
+    if (ra.nslices > w.max_slices) return PK_ERR_CAPACITY;
+    ra.max_slices = w.max_slices;
     ra.topk = topk;
     ra.topk_cap = ix->topk_cap;
-    ra.partial = ix->partial;
+    ra.partial = w.partial;
     ra.lv = ix->lv;
     ra.dbg_est = dbg ? dbg->cand_est : nullptr;
     trace_begin(ix, PK_K_RERANK_TOPK, s);
-    e = launch_rerank_topk(ra, ix->bh, s);
+    e = launch_rerank_topk(ra, w.units, s);
     trace_end(ix, s);
     if (e != cudaSuccess) return cuda_status(e);
 
     MergeArgs ma{};
-    ma.partial = ix->partial;
+    ma.partial = w.partial;
     ma.nslices = ra.nslices;
-    ma.max_slices = ix->max_slices;
+    ma.max_slices = w.max_slices;
     ma.topk = topk;
     ma.topk_cap = ix->topk_cap;
     {
@@ -381,13 +439,15 @@ pk_status search_impl(pk_index *ix, const void *q, int32_t topk, int32_t *out_id
     ma.out_score = out_score;
     ma.dev_err = ix->dev_err;
     trace_begin(ix, PK_K_TOPK_MERGE, s);
-    e = launch_topk_merge(ma, ix->bh, s);
+    e = launch_topk_merge(ma, w.units, s);
     trace_end(ix, s);
     return cuda_status(e);
 }
 
-pk_status attend_impl(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t topk, const void *dK,
-                      const void *dV, int64_t dstride, int32_t dlen, float *out, cudaStream_t s)
+// Attention for kvg query units per index pair (1: each pair's G query heads
+// over the pair's selected rows; G: each query head over its own rows).
+pk_status attend_impl(pk_index *ix, int32_t kvg, const void *q, const int32_t *sel_idx, int32_t topk,
+                      const void *dK, const void *dV, int64_t dstride, int32_t dlen, float *out, cudaStream_t s)
 {
     if (!ix || !q || !out) return PK_ERR_INVALID_ARG;
     if (topk < 0 || topk > ix->topk_cap || dlen < 0 || topk + (int64_t)dlen < 1) return PK_ERR_INVALID_ARG;
@@ -411,16 +471,18 @@ pk_status attend_impl(pk_index *ix, const void *q, const int32_t *sel_idx, int32
     a.out = out;
     a.n = ix->n;
     a.stride = ix->stride;
-    a.H = ix->p.n_kv_heads;
-    a.G = ix->p.group;
+    a.H = ix->p.n_kv_heads * kvg;
+    a.G = ix->p.group / kvg;
+    a.kvg = kvg;
     a.topk = topk;
     a.is_bf16 = ix->p.kv_dtype == PK_BF16;
     a.scale = ix->scale;
-    a.nsplit = splitting(ix, topk + dlen);
+    const int32_t units = ix->bh * kvg;
+    a.nsplit = splitting(ix, units, topk + dlen);
     a.dev_err = ix->dev_err;
     a.dev_err_detail = ix->dev_err_detail;
     trace_begin(ix, PK_K_GATHER_ATTEND, s);
-    cudaError_t e = launch_gather_attend(a, ix->bh, s);
+    cudaError_t e = launch_gather_attend(a, units, s);
     trace_end(ix, s);
     return cuda_status(e);
 }
@@ -513,8 +575,6 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
         delete ix;
         return cuda_status(e);
     }
-    ix->max_chunks = (int32_t)std::max<int64_t>(std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / ix->bh),
-                                                ceil_div(n_cap, kMaxChunk) + 1);
 
     // SRHT sign diagonal and scale; Lloyd-Max levels
     for (int r = 0; r < 4; r++) ix->rot.sign_mask[r] = 0;
@@ -532,30 +592,13 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
         for (int t = 0; t < kL - 1; t++) ix->lv.thr[t] = (float)thr[t];
     }
 
-    const size_t BH = ix->bh, NC = ix->stride, MC = ix->max_chunks;
+    const size_t BH = ix->bh, NC = ix->stride;
     e = cudaSuccess;
     auto chk = [&](cudaError_t x) { if (e == cudaSuccess) e = x; };
     chk(dalloc(&ix->codes, BH * NC * kB));
     chk(dalloc(&ix->rec, BH * NC * kRecBytes));
     chk(dalloc(&ix->occ, BH * kB * kNC));
-    chk(dalloc(&ix->qt, BH * kD));
-    chk(dalloc(&ix->qnorm, BH));
-    chk(dalloc(&ix->bonus_packed, BH * kB * 32));
-    chk(dalloc(&ix->S, BH * NC));
-    chk(dalloc(&ix->chunk_cum, BH * MC * kCum));
-    chk(dalloc(&ix->head_hist, BH * kBins));
-    chk(dalloc(&ix->tickets, BH * 2));
-    chk(dalloc(&ix->chunk_info, BH * MC));
-    chk(dalloc(&ix->sstar, BH));
-    {   // largest slice count any C <= n_cap can need
-        const int64_t lo = slice_lo(ix);
-        const int64_t by_target = std::max<int64_t>(1, (2 * (int64_t)ix->num_sms) / ix->bh);
-        ix->max_slices = (int32_t)std::max<int64_t>(std::min<int64_t>(ceil_div(n_cap, lo), by_target),
-                                                    ceil_div(n_cap, kMaxSlice)) + 1;
-    }
-    const size_t MS = ix->max_slices;
-    chk(dalloc(&ix->cand, BH * NC));
-    chk(dalloc(&ix->partial, BH * MS * (size_t)ix->topk_cap));
+    chk(work_alloc(ix, ix->w, ix->bh, n_cap, s));
 
     chk(dalloc(&ix->dev_err, 1));
     chk(dalloc(&ix->dev_err_detail, 1));
@@ -575,8 +618,6 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
         return PK_ERR_OOM;
     }
     chk(cudaMemsetAsync(ix->occ, 0, BH * kB * kNC * sizeof(uint32_t), s));
-    chk(cudaMemsetAsync(ix->head_hist, 0, BH * kBins * sizeof(uint32_t), s));
-    chk(cudaMemsetAsync(ix->tickets, 0, BH * 2 * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->dev_err, 0, sizeof(int32_t), s));
     chk(cudaMemsetAsync(ix->dev_err_detail, 0, sizeof(long long), s));
     if (e == cudaSuccess) st = copy_rows(ix, ix->K, K, n, 0, s);
@@ -610,28 +651,50 @@ pk_status pk_append(pk_index *ix, const void *k_new, const void *v_new, int64_t 
 pk_status pk_search(pk_index *ix, const void *q, int32_t topk, int32_t *out_idx, float *out_score,
                     void *stream)
 {
-    return search_impl(ix, q, topk, out_idx, out_score, nullptr, (cudaStream_t)stream);
+    if (!ix) return PK_ERR_INVALID_ARG;
+    return search_impl(ix, ix->w, 1, q, topk, out_idx, out_score, nullptr, (cudaStream_t)stream);
 }
 
 pk_status pk_search_debug(pk_index *ix, const void *q, int32_t topk, int32_t *out_idx,
                           float *out_score, const pk_debug_out *dbg, void *stream)
 {
-    return search_impl(ix, q, topk, out_idx, out_score, dbg, (cudaStream_t)stream);
+    if (!ix) return PK_ERR_INVALID_ARG;
+    return search_impl(ix, ix->w, 1, q, topk, out_idx, out_score, dbg, (cudaStream_t)stream);
 }
 
 pk_status pk_attend(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t topk, float *out,
                     void *stream)
 {
     if (topk < 1) return PK_ERR_INVALID_ARG;
-    return attend_impl(ix, q, sel_idx, topk, nullptr, nullptr, 0, 0, out, (cudaStream_t)stream);
+    return attend_impl(ix, 1, q, sel_idx, topk, nullptr, nullptr, 0, 0, out, (cudaStream_t)stream);
 }
 
 pk_status pk_attend_dense(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t topk,
                           const void *dense_K, const void *dense_V, int64_t dense_stride,
                           int32_t dense_len, float *out, void *stream)
 {
-    return attend_impl(ix, q, sel_idx, topk, dense_K, dense_V, dense_stride, dense_len, out,
+    return attend_impl(ix, 1, q, sel_idx, topk, dense_K, dense_V, dense_stride, dense_len, out,
                        (cudaStream_t)stream);
+}
+
+pk_status pk_search_heads(pk_index *ix, const void *q, int32_t topk, int32_t *out_idx, float *out_score,
+                          void *stream)
+{
+    if (!ix) return PK_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (ix->wh.units == 0) {      // the per-head workspace, made on first use
+        const cudaError_t e = work_alloc(ix, ix->wh, ix->bh * ix->p.group, ix->p.n_cap, s);
+        if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? PK_ERR_OOM : PK_ERR_CUDA;
+    }
+    return search_impl(ix, ix->wh, ix->p.group, q, topk, out_idx, out_score, nullptr, s);
+}
+
+pk_status pk_attend_heads(pk_index *ix, const void *q, const int32_t *sel_idx, int32_t topk, float *out,
+                          void *stream)
+{
+    if (!ix) return PK_ERR_INVALID_ARG;
+    if (topk < 1) return PK_ERR_INVALID_ARG;
+    return attend_impl(ix, ix->p.group, q, sel_idx, topk, nullptr, nullptr, 0, 0, out, (cudaStream_t)stream);
 }
 
 void pk_free(pk_index *ix)
@@ -664,7 +727,7 @@ pk_status pk_get_info(const pk_index *ix, pk_info *info)
     info->n = ix->n;
     info->n_cap = ix->p.n_cap;
     info->bh = ix->bh;
-    chunking(ix, ix->n, &info->nchunks, &info->chunk);
+    chunking(ix, ix->w, ix->n, &info->nchunks, &info->chunk);
     resolve(ix->n, ix->p.cand_budget, ix->p.collision_ratio, ix->p.topk, &info->cand, &info->coll);
     info->index_bytes = (int64_t)ix->bh * ix->stride * (kB + kRecBytes) + (int64_t)ix->bh * kB * kNC * 4;
     info->kv_bytes = 2 * (int64_t)ix->bh * ix->stride * kD * ix->es;

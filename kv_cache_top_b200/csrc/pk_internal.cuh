@@ -57,6 +57,7 @@ struct PrepArgs {
     const void *q;           // [batch][H*G][D]
     int32_t H, G, is_bf16, bh;
     int64_t R;               // collision budget ceil(rho n)
+    int32_t kvg;             // query units per index pair (1, or G for per-head search)
     const uint32_t *occ;
     RotConst rot;
     float *qt;               // [BH][D]
@@ -74,6 +75,7 @@ struct ScanArgs {
     const uint32_t *bonus_packed;
     int64_t n, n_cap, chunk, C;   // n_cap: row stride of the per-key arrays
     int32_t nchunks;
+    int32_t kvg;             // query units per index pair
     uint8_t *S;              // [BH][n_cap]
     uint32_t *chunk_cum;     // [BH][max_chunks][kCum]
     uint32_t *head_hist;     // [BH][kBins]
@@ -104,6 +106,7 @@ struct RerankArgs {
     const float *qt;
     const float *qnorm;
     int64_t stride, C;
+    int32_t kvg;             // query units per index pair
     int32_t slice, nslices, max_slices, topk, topk_cap;
     unsigned long long *partial;   // [BH][max_slices][topk_cap]  per-slice Top-k sets
     Levels lv;
@@ -119,6 +122,7 @@ struct AttendArgs {
     int64_t n, stride;
     int32_t H, G, topk, is_bf16;
     int32_t nsplit;          // CTAs (one cluster) per pair, 1..8
+    int32_t kvg;             // query units per index pair (K/V and dense rows of pair unit / kvg)
     float scale;
     int32_t *dev_err;
     long long *dev_err_detail;
@@ -139,6 +143,9 @@ struct MergeArgs {
 
 
 // ---------------------------------------------------------------- helpers
+// index pair of query unit u (the per-head search runs G units per pair)
+__device__ __forceinline__ int index_pair(int u, int kvg) { return kvg > 1 ? u / kvg : u; }
+
 __device__ __forceinline__ float ld_as_f32(const void *p, int64_t i, int is_bf16)
 {
     if (is_bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);

@@ -336,6 +336,41 @@ def test_decode_cache_sink_local_update(pk, offload):
         cache.close()
 
 
+@pytest.mark.parametrize("batch,H,G,n,kv_location", [(1, 2, 4, 20000, 0), (2, 1, 2, 9000, 1)])
+def test_per_query_head_search(pk, batch, H, G, n, kv_location):
+    """pk_search_heads / pk_attend_heads: each query head searches its pair's
+    index with its own query (the oracle's search with G = 1 on that head),
+    and attends over its own rows; the aggregated search is unchanged."""
+    w = workloads.llama_layer(batch, n, H=H, G=G, seed=n + 3, device="cuda")
+    q = w["q"][0]
+    h = build(pk, w["K"], w["V"], n, batch, H, G, kv_location=kv_location)
+    try:
+        U = batch * H * G
+        idx = torch.empty(U, 100, dtype=torch.int32, device="cuda")
+        sc = torch.empty(U, 100, dtype=torch.float32, device="cuda")
+        out = torch.full((batch, H * G, 128), float("nan"), dtype=torch.float32, device="cuda")
+        pk.pk_search_heads(h, q, 100, idx, sc)
+        pk.pk_attend_heads(h, q, idx, 100, out)
+        torch.cuda.synchronize()
+        st, det = pk.pk_last_device_error(h)
+        assert st == 0, (st, det)
+        ids, scs, o = idx.cpu().numpy(), sc.cpu().numpy(), out.cpu().numpy()
+        for u in range(U):
+            b, j = divmod(u, H * G)
+            hh = j // G
+            K_np = workloads.to_np_f32(w["K"][b, hh, :n])
+            V_np = workloads.to_np_f32(w["V"][b, hh, :n])
+            qh = workloads.to_np_f32(q[b, j:j + 1])
+            enc, orc = parity.oracle_pair(K_np, qh, 100, 0)
+            parity.check_topk(ids[u], scs[u], orc, enc)
+            ref = parity.oracle.attend(qh, K_np, V_np, ids[u], 1.0 / math.sqrt(128))
+            assert np.abs(o[b, j:j + 1] - ref).max() <= parity.ATTN_ABS
+        # the aggregated path after the per-head workspace exists
+        check_pairs(pk, h, w["K"], w["V"], q, [0], batch, H, G, n, 100, check_encode=False)
+    finally:
+        pk.pk_free(h)
+
+
 def test_host_pinned_kv_store(pk):
     """K/V kept in pinned host memory and read through UVA by the attention."""
     w = workloads.llama_layer(1, 20000, H=2, G=4, seed=3, device="cuda")
