@@ -11,7 +11,7 @@ budgets.  The line also carries the metric's 1M point (n = 1048576, 8 KV
 heads, K/V in pinned host memory read through UVA) under "million_token".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload throughput|million|llama|tiny|drift|sweep|longgen] [--no-million]
+                  [--workload throughput|million|llama|tiny|drift|sweep|longgen|heads] [--no-million]
                   [--no-cpu-baseline] [--no-e2e] [--no-dense] [--graph] [--drift-steps T]
 
 For N > 1 launch under torch.distributed.run: every rank runs its own copy of
@@ -49,6 +49,8 @@ WORKLOADS = {
     "sweep": dict(name="ratio_sweep", batch=1, n=0, H=8, G=4, cand=0, kv_host=False,
                   ns=(32768, 131072, 524288, 1048576), betas=(0.02, 0.05, 0.1, 0.2),
                   rhos=(0.05, 0.1, 0.2, 0.35, 0.5), queries=8),
+    # aggregated vs per-query-head retrieval on the throughput shape
+    "heads": dict(name="heads_8x131072", batch=8, n=131072, H=8, G=4, cand=0, kv_host=False, queries=16),
     # sink / local / update-buffer decoding after an 8 x 131072 prefill
     "longgen": dict(name="longgen_8x131072+1024", batch=8, n=131072, H=8, G=4, cand=0, kv_host=False,
                     steps=1024, sink=64, local=512, update=512),
@@ -532,6 +534,10 @@ def main():
         if world > 1:
             raise SystemExit("the drift mode runs on one GPU")
         return run_drift(args, wl, peak)
+    if args.workload == "heads":
+        if world > 1:
+            raise SystemExit("the per-head comparison runs on one GPU")
+        return run_heads(args, wl)
     if args.workload == "longgen":
         if world > 1:
             raise SystemExit("the long-generation mode runs on one GPU")
@@ -674,6 +680,72 @@ def run_drift(args, wl, peaks):
             "recall_at_100_mean": sum(b for _, b in recalls) / max(1, len(recalls)),
             "gpu_launches": None}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------- per-query-head retrieval
+def run_heads(args, wl):
+    """The aggregated query (one search per KV head) against every query
+    head searching on its own: Recall@100 against each query head's exact
+    Top-100 of <k_i, q_g> (fp32), and the retrieval + attention time per
+    step (CUDA events, L2 flushed between steps)."""
+    import torch
+    import kv_cache_top_b200 as pk
+    import workloads
+    dev = torch.device("cuda", 0)
+    B, n, H, G, nq = wl["batch"], wl["n"], wl["H"], wl["G"], wl["queries"]
+    w = workloads.llama_layer(B, n, H=H, G=G, seed=args.seed, device=dev, n_queries=nq)
+    p = pk.pk_default_params(batch=B, n_kv_heads=H, group=G, topk=100, kv_dtype=pk.PK_BF16)
+    h = pk.pk_build_index(w["K"], w["V"], n, p)
+    BH, U = B * H, B * H * G
+    idx_a = torch.empty(BH, 100, dtype=torch.int32, device=dev)
+    idx_h = torch.empty(U, 100, dtype=torch.int32, device=dev)
+    out = torch.empty(B, H * G, 128, dtype=torch.float32, device=dev)
+    rec_a, rec_h = [], []
+    for qi in range(nq):
+        q = w["q"][qi]
+        pk.pk_search(h, q, 100, idx_a)
+        pk.pk_search_heads(h, q, 100, idx_h)
+        ga, gh = idx_a.cpu(), idx_h.cpu()
+        qs = q.float().view(B, H, G, 128)
+        for b in range(B):
+            for hh in range(H):
+                s_ = w["K"][b, hh].float() @ qs[b, hh].T                     # [n][G]
+                ex = torch.topk(s_, 100, dim=0).indices.T.cpu()             # [G][100]
+                for g in range(G):
+                    e = set(ex[g].tolist())
+                    rec_a.append(len(e & set(ga[b * H + hh].tolist())) / 100)
+                    rec_h.append(len(e & set(gh[(b * H + hh) * G + g].tolist())) / 100)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(step, k=200):
+        for i in range(5):
+            step(i)
+        ev = []
+        for i in range(k):
+            flush.zero_()
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            step(i)
+            b_.record(stream)
+            ev.append((a_, b_))
+        torch.cuda.synchronize()
+        return sum(a_.elapsed_time(b_) for a_, b_ in ev) / k
+
+    ms_a = timed(lambda i: (pk.pk_search(h, w["q"][i % nq], 100, idx_a),
+                            pk.pk_attend(h, w["q"][i % nq], idx_a, 100, out)))
+    ms_h = timed(lambda i: (pk.pk_search_heads(h, w["q"][i % nq], 100, idx_h),
+                            pk.pk_attend_heads(h, w["q"][i % nq], idx_h, 100, out)))
+    pk.pk_free(h)
+    print(json.dumps({
+        "metric": "Recall@100 against each query head's exact Top-100, and step time: aggregated vs "
+                  "per-query-head retrieval",
+        "aggregated": {"recall_at_100": sum(rec_a) / len(rec_a), "ms_per_step": ms_a,
+                       "steps_s": 1000.0 / ms_a},
+        "per_head": {"recall_at_100": sum(rec_h) / len(rec_h), "ms_per_step": ms_h, "steps_s": 1000.0 / ms_h},
+        "data": "synthetic", "dtype": "f32",
+        "config": {"workload": wl["name"], "batch": B, "n": n, "kv_heads": H, "q_heads": H * G, "topk": 100,
+                   "queries": nq, "l2": "flushed between steps (outside the events)"}}), flush=True)
 
 
 # ------------------------------------------------------ long generation
