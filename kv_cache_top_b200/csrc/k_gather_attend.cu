@@ -32,7 +32,7 @@ constexpr int kAtThreads = 256;
 constexpr int kAtWarps = kAtThreads / 32;
 constexpr int kAtLoads = kAtRows * 32 / kAtThreads;   // 16-byte loads per thread per tile
 
-__global__ void __launch_bounds__(kAtThreads) k_gather_attend(AttendArgs a)
+__global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
 {
     // the K and V tiles; after the row loop rank 0 reuses them for the
     // cluster's partial accumulators [8][kMaxGroup][kD] (32 KB)
