@@ -12,19 +12,19 @@
 // private multi-stage shared-memory ring with asynchronous 16-byte copies
 // (several stages in flight per warp, no registers held), and four lanes
 // decode a record, each taking one 32-byte group (the nibbles of 4 blocks and
-// their 4 weights, 32 coordinates) with no exchange.  The signed level of a nibble comes
-// from a 16-entry shared table (at most 16 distinct words per request: no
-// bank conflicts), addressed by one byte permute per coordinate; q~ stays in
-// registers.  The kernel is issue-bound, so the layout minimises instructions
-// per record.
+// their 4 weights, 32 coordinates) with no exchange.  The signed level of a
+// nibble comes from a 16-entry shared table (at most 16 distinct words per
+// request: no bank conflicts), addressed by one byte permute per coordinate;
+// q~ stays in registers.  The kernel is issue-bound, so the layout minimises
+// instructions per record.
 //
 // Scores never leave the chip: the CTA turns (score, id) into 64-bit keys
-// ordered by score desc then id asc and radix-selects its Top-k set; a merge
-// kernel (one CTA per pair) selects the final Top-k from the per-slice sets
-// and sorts it with one warp (README: "reranks those candidates with a fused
-// 4-bit approximate inner-product kernel and selects the final Top-k KV
-// indices").  Block barriers are few: each radix pass costs two, and appends
-// to shared lists take one atomic per warp.
+// ordered by score desc then id asc, selects its slice's Top-k set in one
+// counting pass over value-linear bins (radix select as the fallback), and
+// writes it sorted; a merge kernel (one CTA per pair) merges the sorted
+// per-slice lists into the final Top-k with a tree of merge-path steps
+// (README: "reranks those candidates with a fused 4-bit approximate
+// inner-product kernel and selects the final Top-k KV indices").
 #include "pk_internal.cuh"
 
 namespace pk {
