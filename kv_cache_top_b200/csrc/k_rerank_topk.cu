@@ -340,81 +340,6 @@ __device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int coun
     return true;
 }
 
-// One warp sorts v[0..32 E) descending in place: E keys per lane in
-// registers (element e = E lane + i), bitonic network, shuffles for the
-// cross-lane stages -- no shared-memory round trips between stages.
-template <int E>
-__device__ void warp_sort_desc_reg(u64 *v)
-{
-    const int lane = threadIdx.x & 31;
-    constexpr int N = 32 * E;
-    u64 x[E];
-#pragma unroll
-    for (int i = 0; i < E; i++) x[i] = v[E * lane + i];
-#pragma unroll
-    for (int k = 2; k <= N; k <<= 1) {
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            if (j >= E) {
-                const int lx = j / E;
-#pragma unroll
-                for (int i = 0; i < E; i++) {
-                    const int e = E * lane + i;
-                    const u64 o = __shfl_xor_sync(kFull, x[i], lx);
-                    const bool keep_max = ((e & j) == 0) == ((e & k) == 0);
-                    x[i] = keep_max ? (o > x[i] ? o : x[i]) : (o < x[i] ? o : x[i]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < E; i++) {
-                    if ((i & j) == 0) {
-                        const int e = E * lane + i;
-                        const bool desc = (e & k) == 0;
-                        const u64 a = x[i], b = x[i ^ j];
-                        const u64 hi = a > b ? a : b, lo = a > b ? b : a;
-                        x[i] = desc ? hi : lo;
-                        x[i ^ j] = desc ? lo : hi;
-                    }
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < E; i++) v[E * lane + i] = x[i];
-}
-
-// One warp sorts v[0..p2) descending in place (p2 a power of two <= 1024).
-__device__ void warp_sort_desc(u64 *v, int p2)
-{
-    if (p2 <= 32) {
-        warp_sort_desc_reg<1>(v);      // callers pad to >= 32 entries with zeros
-    } else if (p2 == 64) {
-        warp_sort_desc_reg<2>(v);
-    } else if (p2 == 128) {
-        warp_sort_desc_reg<4>(v);
-    } else if (p2 == 256) {
-        warp_sort_desc_reg<8>(v);
-    } else {
-        const int lane = threadIdx.x & 31;
-        for (int kk = 2; kk <= p2; kk <<= 1) {
-            for (int j = kk >> 1; j > 0; j >>= 1) {
-                for (int i = lane; i < p2; i += 32) {
-                    const int ixj = i ^ j;
-                    if (ixj > i) {
-                        const u64 x = v[i], y = v[ixj];
-                        const bool desc = (i & kk) == 0;
-                        if (desc ? (x < y) : (x > y)) {
-                            v[i] = y;
-                            v[ixj] = x;
-                        }
-                    }
-                }
-                __syncwarp();
-            }
-        }
-    }
-}
-
 __device__ __forceinline__ u64 make_key(float est, int32_t idx)
 {
     return ((u64)ord_f32(__fadd_rn(est, 0.0f)) << 32) | (u64)(0xffffffffu - (uint32_t)idx);
