@@ -366,18 +366,32 @@ __device__ __forceinline__ void rank_by_count(const u64 *v, int m, Emit emit)
 // with 8 coordinates of q~.  lo/hi hold 4 x the low/high nibble of every byte,
 // i.e. the byte offsets of the signed levels in the 16-entry table; one byte
 // permute per coordinate then yields the address.
+// (x0, x1) * (y0, y1) + (z0, z1) elementwise, one packed fp32 instruction
+__device__ __forceinline__ float2 fma2(float2 x, float2 y, float2 z)
+{
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(r)
+        : "l"(*reinterpret_cast<unsigned long long *>(&x)), "l"(*reinterpret_cast<unsigned long long *>(&y)),
+          "l"(*reinterpret_cast<unsigned long long *>(&z)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+
+// The even and odd coordinates accumulate in the two lanes of one packed
+// fp32 pair (one packed fma per byte of nibbles), added at the end.
 __device__ __forceinline__ float block_dot(const float *slev, uint32_t nib, const float *q)
 {
     const uint32_t lo = (nib << 2) & 0x3c3c3c3cu, hi = (nib >> 2) & 0x3c3c3c3cu;
     const char *base = reinterpret_cast<const char *>(slev);
-    float d = 0.0f;
+    float2 d = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int i = 0; i < 4; i++) {
         const uint32_t o0 = __byte_perm(lo, 0u, 0x4440u + i), o1 = __byte_perm(hi, 0u, 0x4440u + i);
-        d = fmaf(*reinterpret_cast<const float *>(base + o0), q[2 * i], d);
-        d = fmaf(*reinterpret_cast<const float *>(base + o1), q[2 * i + 1], d);
+        const float2 l = make_float2(*reinterpret_cast<const float *>(base + o0),
+                                     *reinterpret_cast<const float *>(base + o1));
+        d = fma2(l, make_float2(q[2 * i], q[2 * i + 1]), d);
     }
-    return d;
+    return d.x + d.y;
 }
 
 
