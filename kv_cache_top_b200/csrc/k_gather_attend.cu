@@ -15,11 +15,16 @@
 // CTA takes a contiguous share of the selected rows, 32 rows per tile, and
 // issues every 16-byte load of a tile's K and V rows before using any, so a
 // tile costs one round trip over the host link and several SMs pull rows at
-// once.  Each CTA keeps an online softmax (max, sum, weighted V) in fp32, then
-// pushes its partial into CTA rank 0's shared memory with distributed-shared-
-// memory stores (no remote round trip), and rank 0 merges the partials with
-// the log-sum-exp rule.  Ids outside [0, n) are skipped and recorded in the
-// device-check word (no trap).
+// once.  A tile's scores take 8 threads per row, each a partial dot over
+// every 8th 16-byte piece of the row (conflict-free shared-memory reads), and
+// 3 shuffles.  Each CTA keeps an online softmax (max, sum, weighted V) in
+// fp32, then pushes its partial into a region of CTA rank 0's shared memory
+// that nothing else uses, with distributed-shared-memory stores (no remote
+// round trip), and arrives at the cluster barrier; rank 0 merges the
+// partials with the log-sum-exp rule.  The only other cluster barrier phase
+// is arrived at on entry, so the pushes know every CTA of the cluster runs.
+// Ids outside [0, n) are skipped and recorded in the device-check word (no
+// trap).
 #include <cooperative_groups.h>
 
 #include "pk_internal.cuh"
@@ -29,26 +34,37 @@ namespace cg = cooperative_groups;
 namespace pk {
 
 constexpr int kAtThreads = 256;
-constexpr int kAtWarps = kAtThreads / 32;
 constexpr int kAtLoads = kAtRows * 32 / kAtThreads;   // 16-byte loads per thread per tile
+constexpr int kQPad = kD + kD / 8;                    // padded query row (4 floats after every 32)
+
+// query element d of a head in the padded row: the 8 threads of a score row
+// read 16-byte pieces whose banks then never collide
+__device__ __forceinline__ int qpad(int d) { return d + 4 * (d >> 5); }
+
+// split cluster barrier (every thread of every CTA of the cluster takes part)
+__device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+// size of the partials region (dynamic shared memory): [nsplit][G][kD] fp32
+size_t attend_smem(int nsplit, int G) { return (size_t)nsplit * G * kD * sizeof(float); }
 
 __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
 {
-    // the K and V tiles; after the row loop rank 0 reuses them for the
-    // cluster's partial accumulators [8][kMaxGroup][kD] (32 KB)
+    // the K and V tiles
     __shared__ __align__(16) unsigned char s_kv[2 * kAtRows * kD * 4];
     unsigned char *sK = s_kv;
     unsigned char *sV = s_kv + kAtRows * kD * 4;
     __shared__ int32_t s_idx[kAtRows];
-    __shared__ float s_q[kMaxGroup][kD];
+    __shared__ __align__(16) float s_q[kMaxGroup][kQPad];
     __shared__ float s_p[kMaxGroup][kAtRows];
     __shared__ float s_m[kMaxGroup], s_l[kMaxGroup], s_alpha[kMaxGroup];
     // rank 0 only: every CTA's partial (running max, sum, accumulator), pushed
     // here with distributed-shared-memory stores before the cluster barrier
     __shared__ float s_pm[8][kMaxGroup], s_pl[8][kMaxGroup];
-    static_assert(8 * kMaxGroup * kD * 4 <= 2 * kAtRows * kD * 4, "partials fit in the row tiles");
-    float (*s_pacc)[kMaxGroup][kD] = reinterpret_cast<float (*)[kMaxGroup][kD]>(s_kv);
+    extern __shared__ __align__(16) float s_pacc[];            // [nsplit][G][kD]
 
+    cluster_arrive_relaxed();                     // this CTA runs (waited for before the pushes)
     cg::cluster_group cluster = cg::this_cluster();
     const int sp = (int)cluster.block_rank(), bh = blockIdx.y;
     const int nsp = a.nsplit;
@@ -64,7 +80,7 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
     const int r_beg = min(nrows, sp * per), r_end = min(nrows, r_beg + per);
 
     const int64_t qbase = ((int64_t)b_seq * a.H * G + (int64_t)h * G) * kD;
-    for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][i % kD] = ld_as_f32(a.q, qbase + i, a.is_bf16);
+    for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][qpad(i % kD)] = ld_as_f32(a.q, qbase + i, a.is_bf16);
     if (tid < G) {
         s_m[tid] = -INFINITY;
         s_l[tid] = 0.0f;
@@ -127,23 +143,64 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
             }
         }
         __syncthreads();
-        // ---- scores: warp w takes rows w, w+8, ..; lane holds dims 4 lane .. 4 lane + 3
-        for (int r = warp; r < rows; r += kAtWarps) {
-            float kx[4];
-            if (a.is_bf16) {
-                const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(sK + (size_t)r * row_bytes) + 2 * lane;
-                const float2 f0 = __bfloat1622float2(p[0]), f1 = __bfloat1622float2(p[1]);
-                kx[0] = f0.x; kx[1] = f0.y; kx[2] = f1.x; kx[3] = f1.y;
-            } else {
-                const float4 f = reinterpret_cast<const float4 *>(sK + (size_t)r * row_bytes)[lane];
-                kx[0] = f.x; kx[1] = f.y; kx[2] = f.z; kx[3] = f.w;
-            }
-            for (int g = 0; g < G; g++) {
-                float s = kx[0] * s_q[g][4 * lane] + kx[1] * s_q[g][4 * lane + 1] +
-                          kx[2] * s_q[g][4 * lane + 2] + kx[3] * s_q[g][4 * lane + 3];
+        // ---- scores: thread (row tid / 8, part j = tid % 8) dots 16-byte pieces
+        // j, j + 8, .. of the row with the matching query elements
+        {
+            const int r = tid >> 3, j = tid & 7;
+            float sc[kMaxGroup];
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(kFull, s, o);
-                if (lane == 0) s_p[g][r] = (s_idx[r] != -1) ? s * a.scale : -INFINITY;
+            for (int g = 0; g < kMaxGroup; g++) sc[g] = 0.0f;
+            if (r < rows) {
+                const uint4 *krow = reinterpret_cast<const uint4 *>(sK + (size_t)r * row_bytes);
+                if (a.is_bf16) {
+#pragma unroll
+                    for (int c = j; c < kD / 8; c += 8) {            // 8 bf16 per piece
+                        const uint4 kv = krow[c];
+                        const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kv.x));
+                        const float2 k1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kv.y));
+                        const float2 k2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kv.z));
+                        const float2 k3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kv.w));
+                        const int q0 = qpad(8 * c);
+#pragma unroll
+                        for (int g = 0; g < kMaxGroup; g++) {
+                            if (g < G) {
+                                const float4 qa = *reinterpret_cast<const float4 *>(&s_q[g][q0]);
+                                const float4 qb = *reinterpret_cast<const float4 *>(&s_q[g][q0 + 4]);
+                                float t = sc[g];
+                                t = fmaf(k0.x, qa.x, t); t = fmaf(k0.y, qa.y, t);
+                                t = fmaf(k1.x, qa.z, t); t = fmaf(k1.y, qa.w, t);
+                                t = fmaf(k2.x, qb.x, t); t = fmaf(k2.y, qb.y, t);
+                                t = fmaf(k3.x, qb.z, t); t = fmaf(k3.y, qb.w, t);
+                                sc[g] = t;
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int c = j; c < kD / 4; c += 8) {            // 4 fp32 per piece
+                        const float4 kv = reinterpret_cast<const float4 *>(krow)[c];
+                        const int q0 = qpad(4 * c);
+#pragma unroll
+                        for (int g = 0; g < kMaxGroup; g++) {
+                            if (g < G) {
+                                const float4 qa = *reinterpret_cast<const float4 *>(&s_q[g][q0]);
+                                float t = sc[g];
+                                t = fmaf(kv.x, qa.x, t); t = fmaf(kv.y, qa.y, t);
+                                t = fmaf(kv.z, qa.z, t); t = fmaf(kv.w, qa.w, t);
+                                sc[g] = t;
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < kMaxGroup; g++) {
+                if (g < G) {
+                    sc[g] += __shfl_xor_sync(kFull, sc[g], 1);
+                    sc[g] += __shfl_xor_sync(kFull, sc[g], 2);
+                    sc[g] += __shfl_xor_sync(kFull, sc[g], 4);
+                    if (j == 0 && r < rows) s_p[g][r] = (s_idx[r] != -1) ? sc[g] * a.scale : -INFINITY;
+                }
             }
         }
         __syncthreads();
@@ -191,8 +248,8 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
     // ---- push this CTA's partial into rank 0 (remote stores: no round trip)
     float *pm = cluster.map_shared_rank(&s_pm[0][0], 0);
     float *pl = cluster.map_shared_rank(&s_pl[0][0], 0);
-    float *pacc = cluster.map_shared_rank(&s_pacc[0][0][0], 0);
-    cluster.sync();                                   // every CTA is done with its rows (and s_m, s_l)
+    float *pacc = cluster.map_shared_rank(s_pacc, 0);
+    cluster_wait();                                   // every CTA of the cluster has started
     if (tid < G) {
         pm[sp * kMaxGroup + tid] = s_m[tid];
         pl[sp * kMaxGroup + tid] = s_l[tid];
@@ -200,9 +257,10 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
 #pragma unroll
     for (int i = 0; i < kMaxGroup / 2; i++) {
         const int g = gsel + 2 * i;
-        if (g < G) pacc[((size_t)sp * kMaxGroup + g) * kD + d] = acc[i];
+        if (g < G) pacc[((size_t)sp * G + g) * kD + d] = acc[i];
     }
-    cluster.sync();                                   // every partial has landed in rank 0
+    cluster_arrive();
+    cluster_wait();                                   // every partial has landed in rank 0
     if (sp == 0) {
         // log-sum-exp merge of the nsp partials, from local shared memory
 #pragma unroll
@@ -216,7 +274,7 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
                 for (int r = 0; r < nsp; r++) {
                     const float mr = s_pm[r][g];
                     const float f = (mr == -INFINITY) ? 0.0f : expf(mr - M);
-                    num = fmaf(f, s_pacc[r][g][d], num);
+                    num = fmaf(f, s_pacc[((size_t)r * G + g) * kD + d], num);
                     den = fmaf(f, s_pl[r][g], den);
                 }
             }
@@ -227,10 +285,17 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
 
 cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s)
 {
+    static int attr_set = 0;                      // per process: the partials region may pass 48 KB in total
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(k_gather_attend, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)attend_smem(8, kMaxGroup));
+        if (e != cudaSuccess) return e;
+        attr_set = 1;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.nsplit, bh, 1);
     cfg.blockDim = dim3(kAtThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = attend_smem(a.nsplit, a.G);
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
