@@ -7,8 +7,10 @@
 // precomputed, so GPU ranking needs no full-precision keys".
 //
 // Work is split by candidate slices (not key ranges), so every CTA reranks
-// the same number of records wherever the candidates sit.  A CTA stages its
-// candidate ids in shared memory; each warp streams its records into a
+// the same number of records wherever the candidates sit; a CTA has 256 or
+// 128 threads, whichever one-wave split loads the busiest SM with fewer
+// records.  A CTA stages its candidate ids in shared memory (in the slots
+// that later hold the keys); each warp streams its records into a
 // private multi-stage shared-memory ring with asynchronous 16-byte copies
 // (several stages in flight per warp, no registers held), and four lanes
 // decode a record, each taking one 32-byte group (the nibbles of 4 blocks and
@@ -22,14 +24,16 @@
 // ordered by score desc then id asc, selects its slice's Top-k set in one
 // counting pass over value-linear bins (radix select as the fallback), and
 // writes it sorted; a merge kernel (one CTA per pair) merges the sorted
-// per-slice lists into the final Top-k with a tree of merge-path steps
+// per-slice lists into the final Top-k with a tree of pairwise merges
+// (bitonic warp merges in registers for k <= 128, merge-path runs in shared
+// memory otherwise)
 // (README: "reranks those candidates with a fused 4-bit approximate
 // inner-product kernel and selects the final Top-k KV indices").
 #include "pk_internal.cuh"
 
 namespace pk {
 
-constexpr int kRrThreads = 256;
+constexpr int kRrThreads = 256;                  // the merge CTA; a rerank CTA has NT = 256 or 128
 constexpr int kRrWarps = kRrThreads / 32;
 
 typedef unsigned long long u64;
@@ -84,12 +88,13 @@ __device__ __forceinline__ u64 warp_sort32_desc(u64 x)
 // every key in one bin); histogram increments are aggregated per warp over
 // lanes that hit the same bin.  Once the bin holding the k-th key has at most
 // 32 keys, one warp sorts that bin and finishes.  All threads of the block
-// must call it.
+// must call it (NT threads).
+template <int NT>
 __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     u64 lo = ~0ull, hi = 0ull;
-    for (int i = tid; i < count; i += kRrThreads) {
+    for (int i = tid; i < count; i += NT) {
         const u64 x = keys[i];
         lo = x < lo ? x : lo;
         hi = x > hi ? x : hi;
@@ -104,14 +109,14 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
         sm.red[0][warp] = lo;
         sm.red[1][warp] = hi;
     }
-    for (int i = tid; i < 2 * 256; i += kRrThreads) (&sm.hist[0][0])[i] = 0u;
+    for (int i = tid; i < 2 * 256; i += NT) (&sm.hist[0][0])[i] = 0u;
     if (tid == 0) {
         sm.sh[3] = 0;
         sm.bcnt = 0;
     }
     __syncthreads();
 #pragma unroll
-    for (int w = 0; w < kRrWarps; w++) {
+    for (int w = 0; w < (NT / 32); w++) {
         lo = sm.red[0][w] < lo ? sm.red[0][w] : lo;
         hi = sm.red[1][w] > hi ? sm.red[1][w] : hi;
     }
@@ -127,7 +132,7 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
         const int shift = top + 1 - width;
         const uint32_t dmask = (1u << width) - 1u;
         uint32_t *H = sm.hist[pass];
-        for (int base = 0; base < count; base += kRrThreads) {
+        for (int base = 0; base < count; base += NT) {
             const int i = base + tid;
             bool act = false;
             uint32_t bin = 0xffffffffu;
@@ -181,7 +186,7 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
     // go to a side list when the bin is small.
     const bool small = (int)inbin != need;
     u64 mn = ~0ull;
-    for (int base = 0; base < count; base += kRrThreads) {
+    for (int base = 0; base < count; base += NT) {
         const int i = base + tid;
         u64 x = 0;
         bool above = false, inb = false;
@@ -219,31 +224,32 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
     if (lane == 0) sm.red[0][warp] = mn;
     __syncthreads();
 #pragma unroll
-    for (int w = 0; w < kRrWarps; w++) mn = sm.red[0][w] < mn ? sm.red[0][w] : mn;
+    for (int w = 0; w < (NT / 32); w++) mn = sm.red[0][w] < mn ? sm.red[0][w] : mn;
     return mn;
 }
 
-// Keep the k largest of keys[0..count) (k < count <= kMaxSlice; keys
+// Keep the k largest of keys[0..count) (k < count <= kSelPer NT; keys
 // distinct) in sm.tmp[0..k), any order, in one counting pass.  Scores of one
 // query span both signs and a few octaves, so bits of the key spread them
 // poorly; instead bin b(v) = min(255, floor((v - vmin) 256 / (vmax - vmin)))
 // of the score v, which never decreases as the key grows, so every key in a
 // bin above the boundary bin is kept.  The upper tail is sparse, so the bin
 // holding the k-th key usually has a few keys; one warp sorts it.  Keys are
-// held in registers, each warp histograms into its own 256 counters (hist,
-// 8 KB of free scratch), and appends take one atomic per warp.  Returns
+// held in registers, each warp histograms into its own 256 counters (hist:
+// 1 KB of free scratch per warp), and placement is one block scan.  Returns
 // false -- with nothing written to sm.tmp -- when the scores are all equal or
 // the boundary bin holds more than 32 keys that must be split; the caller
 // then runs the radix select.  All threads of the block call it.
+template <int NT>
 __device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int count, int k, uint32_t *hist)
 {
-    constexpr int kPer = kMaxSlice / kRrThreads;
+    constexpr int kPer = kSelPer;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     u64 x[kPer];
     float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll
     for (int u = 0; u < kPer; u++) {
-        const int i = tid + u * kRrThreads;
+        const int i = tid + u * NT;
         x[u] = (i < count) ? keys[i] : 0ull;
         if (i < count) {
             const float v = unord_f32((uint32_t)(x[u] >> 32));
@@ -262,13 +268,13 @@ __device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int coun
     float *red = reinterpret_cast<float *>(&sm.red[0][0]);
     if (lane == 0) {
         red[warp] = vmin;
-        red[kRrWarps + warp] = vmax;
+        red[(NT / 32) + warp] = vmax;
     }
     __syncthreads();
 #pragma unroll
-    for (int w = 0; w < kRrWarps; w++) {
+    for (int w = 0; w < (NT / 32); w++) {
         vmin = fminf(vmin, red[w]);
-        vmax = fmaxf(vmax, red[kRrWarps + w]);
+        vmax = fmaxf(vmax, red[(NT / 32) + w]);
     }
     const float range = vmax - vmin;
     const float scale = 256.0f / range;
@@ -282,18 +288,30 @@ __device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int coun
     };
 #pragma unroll
     for (int u = 0; u < kPer; u++)
-        if (tid + u * kRrThreads < count) atomicAdd(&wh[bin_of(x[u])], 1u);
+        if (tid + u * NT < count) atomicAdd(&wh[bin_of(x[u])], 1u);
     __syncthreads();
-    // thread tid takes bin 255 - tid: keys in higher bins by an exclusive scan
-    uint32_t hv = 0;
+    // thread tid takes the BPT = 256 / NT bins 255 - BPT tid - i (i < BPT),
+    // highest first: keys in higher bins by an exclusive scan of its sum
+    static_assert(NT == 128 || NT == 256, "one or two bins per thread");
+    constexpr int BPT = 256 / NT;
+    uint32_t hb[BPT], hv = 0;
 #pragma unroll
-    for (int w = 0; w < kRrWarps; w++) hv += hist[w * 256 + 255 - tid];
+    for (int i = 0; i < BPT; i++) {
+        hb[i] = 0u;
+#pragma unroll
+        for (int w = 0; w < (NT / 32); w++) hb[i] += hist[w * 256 + 255 - BPT * tid - i];
+        hv += hb[i];
+    }
     uint32_t tot;
-    const uint32_t above = block_excl_scan<kRrThreads>(hv, reinterpret_cast<uint32_t *>(&sm.hist[0][0]), &tot);
-    if (above < (uint32_t)k && above + hv >= (uint32_t)k) {
-        sm.sh[0] = 255 - tid;
-        sm.sh[1] = above;
-        sm.sh[2] = hv;
+    uint32_t above = block_excl_scan<NT>(hv, reinterpret_cast<uint32_t *>(&sm.hist[0][0]), &tot);
+#pragma unroll
+    for (int i = 0; i < BPT; i++) {
+        if (above < (uint32_t)k && above + hb[i] >= (uint32_t)k) {
+            sm.sh[0] = 255 - BPT * tid - i;
+            sm.sh[1] = above;
+            sm.sh[2] = hb[i];
+        }
+        above += hb[i];
     }
     if (tid == 0) {
         sm.sh[3] = 0u;
@@ -314,13 +332,13 @@ __device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int coun
     uint32_t keepm = 0, inbm = 0;
 #pragma unroll
     for (int u = 0; u < kPer; u++) {
-        const bool live = tid + u * kRrThreads < count;
+        const bool live = tid + u * NT < count;
         const int bq = live ? bin_of(x[u]) : -1;
         if (live && (small ? bq > bstar : bq >= bstar)) keepm |= 1u << u;
         if (live && small && bq == bstar) inbm |= 1u << u;
     }
     uint32_t tot2;
-    const uint32_t ex2 = block_excl_scan<kRrThreads>(((uint32_t)__popc(keepm) << 16) | (uint32_t)__popc(inbm),
+    const uint32_t ex2 = block_excl_scan<NT>(((uint32_t)__popc(keepm) << 16) | (uint32_t)__popc(inbm),
                                                      reinterpret_cast<uint32_t *>(&sm.hist[0][0]), &tot2);
     uint32_t pos = ex2 >> 16, bp = ex2 & 0xffffu;
 #pragma unroll
@@ -349,10 +367,10 @@ __device__ __forceinline__ u64 make_key(float est, int32_t idx)
 // #{y in v : y > x}.  Every thread walks the whole list in step (broadcast
 // shared-memory reads), so the pass costs m / blockDim compares per key and
 // no barrier; it sorts and selects at once for small m.
-template <typename Emit>
+template <int NT, typename Emit>
 __device__ __forceinline__ void rank_by_count(const u64 *v, int m, Emit emit)
 {
-    for (int i0 = 0; i0 < m; i0 += kRrThreads) {
+    for (int i0 = 0; i0 < m; i0 += NT) {
         const int i = i0 + (int)threadIdx.x;
         const u64 x = (i < m) ? v[i] : ~0ull;
         int r = 0;
@@ -395,18 +413,87 @@ __device__ __forceinline__ float block_dot(const float *slev, uint32_t nib, cons
 }
 
 
+// Merge of the per-slice Top-k lists of one pair into its final sorted
+// Top-k.  Each list arrives sorted descending (zero = padding; real keys are
+// distinct).  Lists of at most 128 keys merge by a tree of warp merges in
+// registers (warp_merge_tree).  Otherwise, when the lists fit in shared
+// memory, a tree of pairwise merges halves their number per level, each
+// merge keeping its k best.  A level splits every merge's outputs into runs, about one per
+// thread; a run starts at the co-rank of its first output d (merge path: the
+// first d outputs are A[0..i) and B[0..d-i) for the i found by binary
+// search) and merges sequentially from there, so a level costs one barrier
+// whatever the score distribution.
+// Larger inputs run in rounds of radix select that keep the best k seen.
+__device__ __forceinline__ void emit_topk(int32_t *out_idx, float *out_score, int bh, int k, int r, u64 x)
+{
+    const bool live = x != 0ull;
+    out_idx[(size_t)bh * k + r] = live ? (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu)) : -1;
+    if (out_score) out_score[(size_t)bh * k + r] = live ? unord_f32((uint32_t)(x >> 32)) : 0.0f;
+}
+
+// Lists s = 0..ns-1 of k keys at src + s k; returns the buffer holding the
+// merged list (k keys).  src needs ns k keys, dst (ns + 1) / 2 k keys.  All
+// NT threads of the block call it.
+template <int NT>
+__device__ const u64 *merge_tree(u64 *src, u64 *dst, int ns, int k)
+{
+    while (ns > 1) {
+        const int np = (ns + 1) / 2;
+        // about one run of R consecutive outputs per thread
+        const int R = max(1, (np * k + NT - 1) / NT);
+        const int rpm = (k + R - 1) / R;          // runs per merge
+        for (int t = threadIdx.x; t < np * rpm; t += NT) {
+            const int m = t / rpm, d0 = (t - m * rpm) * R, d1 = min(k, d0 + R);
+            const u64 *A = src + (size_t)(2 * m) * k;
+            u64 *out = dst + (size_t)m * k;
+            if (2 * m + 1 >= ns) {
+                for (int d = d0; d < d1; d++) out[d] = A[d];     // odd list out: carried up
+            } else {
+                const u64 *B = A + k;
+                int lo = 0, hi = d0;              // d0 < k: the co-rank i is in [0, d0]
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (A[mid] > B[d0 - 1 - mid]) lo = mid + 1;
+                    else hi = mid;
+                }
+                int i = lo, j = d0 - lo;
+                u64 x = A[i], y = B[j];
+                for (int d = d0; d < d1; d++) {   // sequential merge of the run
+                    if (x > y) {
+                        out[d] = x;
+                        x = (++i < k) ? A[i] : 0ull;
+                    } else {
+                        out[d] = y;
+                        y = (++j < k) ? B[j] : 0ull;
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        u64 *t = src;
+        src = dst;
+        dst = t;
+        ns = np;
+    }
+    return src;
+}
+
 constexpr int kRrStages = 3;                       // per-warp pipeline depth
 constexpr int kRrStep = 16;                        // records per warp stage
 constexpr int kRecPad = 144;                       // shared-memory record stride (conflict-free)
-constexpr size_t kRrRingBytes = (size_t)kRrWarps * kRrStages * kRrStep * kRecPad;
+__host__ __device__ constexpr size_t rr_ring_bytes(int nt) { return (size_t)(nt / 32) * kRrStages * kRrStep * kRecPad; }
 
-__global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
+// NT = 256 (2 CTAs per SM) or 128 (4 CTAs per SM): the host takes the size
+// whose one-wave split of the candidates loads the SMs more evenly.
+template <int NT>
+__global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
 {
+    constexpr int NW = NT / 32;
     extern __shared__ __align__(16) unsigned char s_dyn[];
     __shared__ RrShared sm;
     unsigned char *ring_all = s_dyn;                                   // [warps][stages][16][144]
-    u64 *keys = reinterpret_cast<u64 *>(s_dyn + kRrRingBytes);         // [slice]
-    int32_t *ids = reinterpret_cast<int32_t *>(s_dyn + kRrRingBytes + (size_t)a.slice * sizeof(u64));
+    // [slice]: the candidate ids (low 32 bits) until a record is decoded, then its key
+    u64 *keys = reinterpret_cast<u64 *>(s_dyn + rr_ring_bytes(NT));
     const int bh = blockIdx.y, sl = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int k = a.topk;
@@ -416,7 +503,7 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
     if (tid < 16) sm.slev[tid] = (tid & 8) ? -a.lv.lev[tid & 7] : a.lv.lev[tid & 7];
     pdl_wait();                                   // candidates come from the compaction
     const int32_t *cand = a.cand + (size_t)bh * a.stride + m0;
-    for (int i = tid; i < count; i += kRrThreads) ids[i] = cand[i];
+    for (int i = tid; i < count; i += NT) keys[i] = (u64)(uint32_t)cand[i];
     const int q4 = lane & 3, sub = lane >> 2;          // 32-byte group of the record, record of the round
     float qr[32];
 #pragma unroll
@@ -434,28 +521,30 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
     unsigned char *ring = ring_all + (size_t)warp * kRrStages * kRrStep * kRecPad;
     const int nsteps = (count + kRrStep - 1) / kRrStep;
     auto issue = [&](int step_local, int stage) {
-        const int r0 = (warp + step_local * kRrWarps) * kRrStep;
+        const int r0 = (warp + step_local * NW) * kRrStep;
         if (r0 < count) {
 #pragma unroll
             for (int u = 0; u < 4; u++) {
                 const int piece = lane + 32 * u;
                 const int j = piece >> 3, c = piece & 7;
                 const int r = r0 + j;
-                const int32_t id = ids[r < count ? r : 0];
-                cp_async16(ring + ((size_t)stage * kRrStep + j) * kRecPad + 16 * c,
-                           rec + (size_t)id * kRecBytes + 16 * c);
+                if (r < count) {                      // keys[r] still holds the id: r is decoded later
+                    const int32_t id = (int32_t)(uint32_t)keys[r];
+                    cp_async16(ring + ((size_t)stage * kRrStep + j) * kRecPad + 16 * c,
+                               rec + (size_t)id * kRecBytes + 16 * c);
+                }
             }
         }
         cp_async_commit();                            // always one group per call
     };
-    const int my_steps = (nsteps > warp) ? (nsteps - warp + kRrWarps - 1) / kRrWarps : 0;
+    const int my_steps = (nsteps > warp) ? (nsteps - warp + NW - 1) / NW : 0;
 #pragma unroll
     for (int s = 0; s < kRrStages - 1; s++) issue(s, s);
     for (int t = 0; t < my_steps; t++) {
         cp_async_wait<kRrStages - 2>();               // step t has landed (this lane's pieces)
         __syncwarp();                                 // ... and every lane's
         const int stage = t % kRrStages;
-        const int r0 = (warp + t * kRrWarps) * kRrStep;
+        const int r0 = (warp + t * NW) * kRrStep;
         const unsigned char *st = ring + (size_t)stage * kRrStep * kRecPad;
 #pragma unroll
         for (int u = 0; u < 2; u++) {
@@ -471,7 +560,7 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
             const int r = r0 + j;
             if (q4 == 0 && r < count) {
                 const float est = qnorm * part;
-                keys[r] = make_key(est, ids[r]);
+                keys[r] = make_key(est, (int32_t)(uint32_t)keys[r]);
                 if (dest) dest[r] = est;
             }
         }
@@ -485,66 +574,104 @@ __global__ void __launch_bounds__(kRrThreads, 2) k_rerank_topk(RerankArgs a)
     const int have = min(count, k);
     if (count > k) {
         // the ring is free now: 8 KB of it hold the per-warp histograms
-        if (!block_topk_select_linear(sm, keys, count, k, reinterpret_cast<uint32_t *>(ring_all)))
-            block_topk_select(sm, keys, count, k);
+        if (!block_topk_select_linear<NT>(sm, keys, count, k, reinterpret_cast<uint32_t *>(ring_all)))
+            block_topk_select<NT>(sm, keys, count, k);
     } else {
-        for (int i = tid; i < count; i += kRrThreads) sm.tmp[i] = keys[i];
+        for (int i = tid; i < count; i += NT) sm.tmp[i] = keys[i];
         __syncthreads();
     }
     // the slice's set, sorted descending (zeros pad a slice shorter than k)
     u64 *part = a.partial + ((size_t)bh * a.max_slices + sl) * a.topk_cap;
-    rank_by_count(sm.tmp, have, [&](int r, u64 x) { part[r] = x; });
-    for (int i = have + tid; i < k; i += kRrThreads) part[i] = 0ull;
+    rank_by_count<NT>(sm.tmp, have, [&](int r, u64 x) { part[r] = x; });
+    for (int i = have + tid; i < k; i += NT) part[i] = 0ull;
     pdl_trigger();
 }
 
-// Merge of the per-slice Top-k lists of one pair into its final sorted
-// Top-k.  Each list arrives sorted descending (zero = padding; real keys are
-// distinct).  When the lists fit in shared memory (the usual case) a tree of
-// pairwise merges halves their number per level, each merge keeping its k
-// best: output position d of merge(A, B) comes from the co-rank of d (merge
-// path) -- the first d outputs are A[0..i) and B[0..d-i) for the i found by
-// binary search -- so every output is computed independently in log2(k)
-// steps and a level costs one barrier, whatever the score distribution.
-// Larger inputs run in rounds of radix select that keep the best k seen.
-__device__ __forceinline__ void merge_emit(const MergeArgs &a, int bh, int k, int r, u64 x)
+// keys the merge's dynamic shared memory holds for a list capacity cap
+__host__ __device__ inline int64_t merge_keys(int cap) { return (int64_t)cap + (cap + 1) / 2 + 64 + 1024; }
+
+// One warp: the top 128 of two descending lists of at most 128 keys each
+// (element 32 j + lane in register j; missing keys are 0), descending, into
+// a.  max(A[i], B[127 - i]) over i is the top half of A and B together and is
+// bitonic (a falling sequence against a rising one), so seven half-cleaner
+// stages sort it: strides 64 and 32 inside a lane's registers, 16 .. 1 across
+// lanes by shuffles.
+__device__ __forceinline__ void warp_merge128(u64 (&a)[4], const u64 (&b)[4])
 {
-    const bool live = x != 0ull;
-    a.out_idx[(size_t)bh * k + r] = live ? (int32_t)(0xffffffffu - (uint32_t)(x & 0xffffffffu)) : -1;
-    if (a.out_score) a.out_score[(size_t)bh * k + r] = live ? unord_f32((uint32_t)(x >> 32)) : 0.0f;
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const u64 y = __shfl_sync(kFull, b[3 - j], 31 - lane);
+        a[j] = a[j] > y ? a[j] : y;
+    }
+#pragma unroll
+    for (int s = 2; s >= 1; s >>= 1) {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            if ((j & s) == 0) {
+                const u64 x = a[j], y = a[j + s];
+                a[j] = x > y ? x : y;
+                a[j + s] = x > y ? y : x;
+            }
+        }
+    }
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+        const bool upper = (lane & s) == 0;       // keeps the larger key of the pair
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const u64 y = __shfl_xor_sync(kFull, a[j], s);
+            a[j] = upper ? (a[j] > y ? a[j] : y) : (a[j] < y ? a[j] : y);
+        }
+    }
 }
 
-// Lists s = 0..ns-1 of k keys at src + s k; returns the buffer holding the
-// merged list (k keys).  src needs ns k keys, dst (ns + 1) / 2 k keys.  All
-// threads of the block call it.
-__device__ const u64 *merge_tree(u64 *src, u64 *dst, int ns, int k)
+// Top k (k <= 128) of ns >= 2 descending lists (list s: k keys at
+// src + s stride) by a tree of warp merges: warp w takes merges w, w + 8, ..
+// of a level and fetches its next pair before merging the current one.
+// buf holds ((ns + 1) / 2 + (ns + 3) / 4) x 128 keys; returns the merged list.
+__device__ const u64 *warp_merge_tree(const u64 *src, size_t stride, bool global_src, int ns, int k, u64 *buf)
 {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    u64 *dst = buf, *alt = buf + (size_t)((ns + 1) / 2) * 128;
+    auto fetch = [&](const u64 *list, int len, u64 (&v)[4]) {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int e = 32 * j + lane;
+            v[j] = (list && e < len) ? (global_src ? __ldcg(list + e) : list[e]) : 0ull;
+        }
+    };
     while (ns > 1) {
         const int np = (ns + 1) / 2;
-        const int tasks = np * k;
-        for (int t = threadIdx.x; t < tasks; t += kRrThreads) {
-            const int m = t / k, d = t - m * k;
-            const u64 *A = src + (size_t)(2 * m) * k;
-            u64 out;
-            if (2 * m + 1 >= ns) {
-                out = A[d];                       // odd list out: carried up
-            } else {
-                const u64 *B = A + k;
-                int lo = 0, hi = d;               // d < k: i in [0, d]
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (A[mid] > B[d - 1 - mid]) lo = mid + 1;
-                    else hi = mid;
-                }
-                const u64 x = A[lo], y = B[d - lo];
-                out = y > x ? y : x;
+        u64 a[4], b[4], na[4], nb[4];
+        int m = warp;
+        if (m < np) {
+            fetch(src + (size_t)(2 * m) * stride, k, a);
+            fetch(2 * m + 1 < ns ? src + (size_t)(2 * m + 1) * stride : nullptr, k, b);
+        }
+        while (m < np) {
+            const int mn = m + kRrWarps;
+            if (mn < np) {                        // in flight while this pair merges
+                fetch(src + (size_t)(2 * mn) * stride, k, na);
+                fetch(2 * mn + 1 < ns ? src + (size_t)(2 * mn + 1) * stride : nullptr, k, nb);
             }
-            dst[(size_t)m * k + d] = out;
+            warp_merge128(a, b);
+            u64 *o = dst + (size_t)m * 128;
+#pragma unroll
+            for (int j = 0; j < 4; j++) o[32 * j + lane] = a[j];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                a[j] = na[j];
+                b[j] = nb[j];
+            }
+            m = mn;
         }
         __syncthreads();
-        u64 *t = src;
         src = dst;
-        dst = t;
+        dst = alt;
+        alt = const_cast<u64 *>(src);
+        stride = 128;
+        global_src = false;
         ns = np;
     }
     return src;
@@ -562,20 +689,52 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
     pdl_wait();                                   // per-slice lists come from the rerank
     const int64_t total = (int64_t)a.nslices * k;
     const u64 *plist = a.partial + (size_t)bh * a.max_slices * a.topk_cap;
+    const int ns = a.nslices;
+    if (k <= 128 && (ns == 1 || (int64_t)((ns + 1) / 2 + (ns + 3) / 4) * 128 <= merge_keys(cap))) {
+        // lists of at most 128 keys: warp merges in registers
+        const u64 *res = ns == 1 ? plist : warp_merge_tree(plist, a.topk_cap, true, ns, k, keys);
+        if (tid < 32) {                          // keys in the result: one warp counts
+            int got = 0;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int e = 32 * j + tid;
+                got += __popc(__ballot_sync(kFull, e < k && (ns == 1 ? __ldcg(res + e) : res[e]) != 0ull));
+            }
+            if (tid == 0 && got < k) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
+        }
+        for (int d = tid; d < k; d += kRrThreads)
+            emit_topk(a.out_idx, a.out_score, bh, k, d, ns == 1 ? __ldcg(res + d) : res[d]);
+        __syncthreads();                          // release the attention only once every output is written
+        pdl_trigger();
+        return;
+    }
     if (total <= cap) {
-#pragma unroll 4
-        for (int e = tid; e < (int)total; e += kRrThreads) {
-            const int sl = e / k, r = e - sl * k;
-            keys[e] = plist[(size_t)sl * a.topk_cap + r];
+        constexpr int kLd = 16;                   // loads in flight per thread
+        for (int e0 = 0; e0 < (int)total; e0 += kLd * kRrThreads) {
+            u64 v[kLd];
+#pragma unroll
+            for (int u = 0; u < kLd; u++) {
+                const int e = e0 + u * kRrThreads + tid;
+                v[u] = 0ull;
+                if (e < (int)total) {
+                    const int sl = e / k, r = e - sl * k;
+                    v[u] = plist[(size_t)sl * a.topk_cap + r];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kLd; u++) {
+                const int e = e0 + u * kRrThreads + tid;
+                if (e < (int)total) keys[e] = v[u];
+            }
         }
         __syncthreads();
-        const u64 *res = merge_tree(keys, keys + cap, a.nslices, k);
+        const u64 *res = merge_tree<kRrThreads>(keys, keys + cap, a.nslices, k);
         if (tid == 0 && res[k - 1] == 0ull) {
             int got = 0;
             while (got < k && res[got] != 0ull) got++;
             devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
         }
-        for (int d = tid; d < k; d += kRrThreads) merge_emit(a, bh, k, d, res[d]);
+        for (int d = tid; d < k; d += kRrThreads) emit_topk(a.out_idx, a.out_score, bh, k, d, res[d]);
         pdl_trigger();
         return;
     }
@@ -607,7 +766,7 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
         __syncthreads();
         cnt = (int)sm.cnt;
         if (cnt > k) {
-            tau = block_topk_select(sm, keys, cnt, k);
+            tau = block_topk_select<kRrThreads>(sm, keys, cnt, k);
             for (int i = tid; i < k; i += kRrThreads) keys[i] = sm.tmp[i];
             cnt = k;
             __syncthreads();
@@ -615,14 +774,14 @@ __global__ void __launch_bounds__(kRrThreads) k_topk_merge(MergeArgs a)
     }
     const int got = min(cnt, k);
     if (got != k && tid == 0) devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, got);
-    rank_by_count(keys, got, [&](int r, u64 x) { merge_emit(a, bh, k, r, x); });
-    for (int i = got + tid; i < k; i += kRrThreads) merge_emit(a, bh, k, i, 0ull);
+    rank_by_count<kRrThreads>(keys, got, [&](int r, u64 x) { emit_topk(a.out_idx, a.out_score, bh, k, r, x); });
+    for (int i = got + tid; i < k; i += kRrThreads) emit_topk(a.out_idx, a.out_score, bh, k, i, 0ull);
     pdl_trigger();
 }
 
 // dynamic shared memory of the merge: cap keys for the lists, (cap + 1) / 2 + k
 // for the first level of the merge tree
-size_t merge_smem(int cap) { return ((size_t)cap + (cap + 1) / 2 + 64 + 1024) * sizeof(u64); }
+size_t merge_smem(int cap) { return (size_t)merge_keys(cap) * sizeof(u64); }
 
 cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s)
 {
@@ -637,19 +796,26 @@ cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s)
     return launch_pdl(k_topk_merge, dim3(bh), dim3(kRrThreads), smem, s, a);
 }
 
-size_t rerank_smem(int slice) { return kRrRingBytes + (size_t)slice * (sizeof(u64) + sizeof(int32_t)); }
+size_t rerank_smem(int slice, int nt) { return rr_ring_bytes(nt) + (size_t)slice * sizeof(u64); }
+
+template <int NT>
+cudaError_t launch_rerank_nt(const RerankArgs &a, int bh, cudaStream_t s)
+{
+    static int attr_max = 0;
+    const size_t smem = rerank_smem(a.slice, NT);
+    if ((int)smem > attr_max) {
+        const int most = (int)rerank_smem(kSelPer * NT, NT);
+        cudaError_t e = cudaFuncSetAttribute(k_rerank_topk<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+        if (e != cudaSuccess) return e;
+        attr_max = most;
+    }
+    return launch_pdl(k_rerank_topk<NT>, dim3(a.nslices, bh), dim3(NT), smem, s, a);
+}
 
 cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s)
 {
-    static int attr_max = 0;
-    const size_t smem = rerank_smem(a.slice);
-    if ((int)smem > attr_max) {
-        cudaError_t e = cudaFuncSetAttribute(k_rerank_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)rerank_smem(kMaxSlice));
-        if (e != cudaSuccess) return e;
-        attr_max = (int)rerank_smem(kMaxSlice);
-    }
-    return launch_pdl(k_rerank_topk, dim3(a.nslices, bh), dim3(kRrThreads), smem, s, a);
+    if (a.slice > kSelPer * a.nt) return cudaErrorInvalidValue;
+    return a.nt == 128 ? launch_rerank_nt<128>(a, bh, s) : launch_rerank_nt<256>(a, bh, s);
 }
 
 }  // namespace pk

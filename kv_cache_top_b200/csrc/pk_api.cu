@@ -138,19 +138,32 @@ void chunking(const pk_index *ix, const Work &w, int64_t n, int32_t *nchunks, in
     *nchunks = (int32_t)ceil_div(n, ch);
 }
 
-// rerank work split: slices of the candidate list, ~3 CTAs per SM in total
+// rerank work split: slices of each unit's candidate list.  A CTA of nt
+// threads holds at most kSelPer x nt candidates, and 512 / nt CTAs fit on an
+// SM.  Per CTA size: at most one wave unless the slice cap forces more; then
+// the size whose busiest SM gets fewer records (ties: 256, fewer lists to
+// merge).
 int32_t slice_lo(const pk_index *ix) { return std::max<int32_t>(256, 2 * ix->topk_cap); }
 
-void slicing(const pk_index *ix, const Work &w, int64_t C, int32_t *slice, int32_t *nslices)
+void slicing(const pk_index *ix, const Work &w, int64_t C, int32_t *slice, int32_t *nslices, int32_t *nt)
 {
-    // at most one wave (2 resident CTAs per SM) unless the slice-size cap forces more
-    int64_t ns = std::max<int64_t>(1, (2 * (int64_t)ix->num_sms) / w.units);
-    ns = std::max<int64_t>(ns, ceil_div(C, kMaxSlice));
-    int64_t sl = ceil_div(ceil_div(C, ns), 64) * 64;
-    sl = std::max<int64_t>(sl, slice_lo(ix));
-    sl = std::min<int64_t>(sl, kMaxSlice);
-    *slice = (int32_t)sl;
-    *nslices = (int32_t)ceil_div(C, sl);
+    int64_t best_load = -1;
+    for (int t : {256, 128}) {
+        const int64_t slots = (512 / t) * (int64_t)ix->num_sms, cap = (int64_t)kSelPer * t;
+        int64_t ns = std::max<int64_t>(1, slots / w.units);
+        ns = std::max<int64_t>(ns, ceil_div(C, cap));
+        int64_t sl = ceil_div(ceil_div(C, ns), 16) * 16;
+        sl = std::max<int64_t>(sl, slice_lo(ix));
+        sl = std::min<int64_t>(sl, cap);
+        const int64_t nsl = ceil_div(C, sl);
+        const int64_t load = ceil_div(nsl * w.units, (int64_t)ix->num_sms) * sl;   // records on the busiest SM
+        if (best_load < 0 || load < best_load) {
+            best_load = load;
+            *slice = (int32_t)sl;
+            *nslices = (int32_t)nsl;
+            *nt = t;
+        }
+    }
 }
 
 // attention work split: one cluster of up to 8 CTAs per pair, ~2 CTAs per SM
@@ -190,9 +203,9 @@ cudaError_t work_alloc(pk_index *ix, Work &w, int32_t units, int64_t n_cap, cuda
                                               ceil_div(n_cap, kMaxChunk) + 1);
     {   // largest slice count any C <= n_cap can need
         const int64_t lo = slice_lo(ix);
-        const int64_t by_target = std::max<int64_t>(1, (2 * (int64_t)ix->num_sms) / units);
+        const int64_t by_target = std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / units);
         w.max_slices = (int32_t)std::max<int64_t>(std::min<int64_t>(ceil_div(n_cap, lo), by_target),
-                                                  ceil_div(n_cap, kMaxSlice)) + 1;
+                                                  ceil_div(n_cap, kSelPer * 128)) + 1;
     }
     const size_t U = units, NC = ix->stride, MC = w.max_chunks, MS = w.max_slices;
     cudaError_t e = cudaSuccess;
@@ -411,7 +424,7 @@ pk_status search_impl(pk_index *ix, Work &w, int32_t kvg, const void *q, int32_t
     ra.qnorm = w.qnorm;
     ra.stride = ix->stride;
     ra.C = C;
-    slicing(ix, w, C, &ra.slice, &ra.nslices);
+    slicing(ix, w, C, &ra.slice, &ra.nslices, &ra.nt);
     if (ra.nslices > w.max_slices) return PK_ERR_CAPACITY;
     ra.max_slices = w.max_slices;
     ra.topk = topk;

@@ -21,7 +21,8 @@ constexpr int kCum = kBins + 1;  // suffix-count entries per chunk (98, last = 0
 constexpr int kRecBytes = 128;   // 4-bit summary record per key
 constexpr int kMaxTopk = 1024;
 constexpr int kMaxGroup = 8;
-constexpr int kMaxSlice = 4096;  // candidates per rerank CTA (upper bound)
+constexpr int kSelPer = 16;      // candidates per rerank thread (upper bound): a slice has <= kSelPer x CTA size
+constexpr int kMaxSlice = kSelPer * 256;  // candidates per rerank CTA (upper bound)
 constexpr int kAtRows = 32;      // selected rows per attention CTA (upper bound)
 constexpr int kMergeCap = 16384; // partial keys one merge CTA holds at once
 constexpr unsigned kFull = 0xffffffffu;
@@ -108,6 +109,7 @@ struct RerankArgs {
     int64_t stride, C;
     int32_t kvg;             // query units per index pair
     int32_t slice, nslices, max_slices, topk, topk_cap;
+    int32_t nt;              // threads per CTA: 256 or 128
     unsigned long long *partial;   // [BH][max_slices][topk_cap]  per-slice Top-k sets
     Levels lv;
     float *dbg_est;          // [BH][C] or null
@@ -286,7 +288,7 @@ cudaError_t launch_compact(const CompactArgs &a, int nchunks, int bh, cudaStream
 cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s);
-size_t rerank_smem(int slice);
+size_t rerank_smem(int slice, int nt);
 
 // Launch with programmatic stream serialisation (the kernel calls pdl_wait()
 // before reading what earlier kernels of the stream wrote).

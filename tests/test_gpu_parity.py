@@ -123,6 +123,7 @@ def test_llama_shaped_layer_config(pk):
     (3001, 0, 1, 1, 1, 3),        # topk = 1
     (70001, 0, 100, 1, 1, 4),     # many compaction windows, odd n
     (9000, 200, 200, 3, 1, 8),    # C == topk, G = 8
+    (40000, 0, 256, 1, 2, 1),     # topk > 128 over several slices: shared-memory merge tree
 ])
 def test_edge_and_ragged_sizes(pk, n, cand, topk, batch, H, G):
     w = workloads.llama_layer(batch, n, H=H, G=G, seed=n, device="cuda")
@@ -417,6 +418,26 @@ def test_search_rejects_bad_arguments(pk):
         assert e.value.status == 1
     finally:
         pk.pk_free(h)
+
+
+def test_many_pairs_small_rerank_ctas(pk):
+    """8 sequences x 8 KV heads (64 pairs), n = 40960, C = 4096: the rerank
+    splits each pair's candidates over 128-thread CTAs (9 slices of 464; the
+    256-thread split, 4 slices of 1024 on 256 CTAs, would load the busiest SM
+    with 2048 records against 1856), so the merge combines 9 lists.  Four
+    pairs checked element by element."""
+    batch, n, H, G = 8, 40960, 8, 4
+    w = workloads.llama_layer(batch, n, H=H, G=G, seed=12, device="cuda", n_queries=1)
+    h = build(pk, w["K"], w["V"], n, batch, H, G, cand_budget=4096)
+    try:
+        idx = check_pairs(pk, h, w["K"], w["V"], w["q"][0], [0, 21, 42, 63], batch, H, G, n, 100,
+                          cand_budget=4096)
+        for p in range(batch * H):
+            assert len(set(idx[p].tolist())) == 100
+    finally:
+        pk.pk_free(h)
+        del w
+        torch.cuda.empty_cache()
 
 
 # ------------------------------------------------- full-size workloads
