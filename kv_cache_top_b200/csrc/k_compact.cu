@@ -7,7 +7,9 @@
 // S = s* keys it keeps; here each CTA loads its whole chunk of S at once (up
 // to 8 x 16 bytes per thread, each thread a contiguous run of keys), turns
 // every 16 bytes into 16-bit masks of "S > s*" and "S = s*", and places the
-// candidates with one block-wide scan: no per-key branches.
+// candidates with one block-wide scan: no per-key branches.  The ids are
+// staged in shared memory in output order and stored by consecutive threads
+// (chunks with more than kCpStage candidates store them from each thread).
 //
 // Byte-parallel compares: scores are <= 96 < 128, so for a byte s,
 // s > t  <=>  bit 7 of s + (127 - t) is set, and s >= t <=> bit 7 of
@@ -19,6 +21,7 @@ namespace pk {
 
 constexpr int kCpThreads = 256;
 constexpr int kCpMaxU = 8;    // 16-byte groups per thread: chunk <= 32768 keys
+constexpr int kCpStage = 4096;   // candidates of a chunk staged in shared memory for coalesced stores
 
 // bit-7 flags of the 4 bytes -> 4-bit mask (bit i = byte i)
 __device__ __forceinline__ uint32_t gather4(uint32_t flags) { return (flags * 0x00204081u) >> 28; }
@@ -41,6 +44,7 @@ __device__ __forceinline__ void masks16(uint4 v, uint32_t add_gt, uint32_t add_g
 __global__ void __launch_bounds__(kCpThreads) k_compact(CompactArgs a)
 {
     __shared__ uint32_t s_ws[kCpThreads / 32 + 1];
+    __shared__ int32_t s_ids[kCpStage];
     const int bh = blockIdx.y, chunk = blockIdx.x;
     const int tid = threadIdx.x;
     const int64_t lo = (int64_t)chunk * a.chunk;
@@ -82,6 +86,9 @@ __global__ void __launch_bounds__(kCpThreads) k_compact(CompactArgs a)
     int32_t *out = a.cand + (size_t)bh * a.stride + slot0;
     int32_t *dbg = a.dbg_cand ? a.dbg_cand + (size_t)bh * a.C + slot0 : nullptr;
     const int64_t room = a.C - (int64_t)slot0;
+    // the chunk's candidates: every S > s* key and its first `quota` ties
+    const uint32_t n_out = (tot >> 16) + min(tot & 0xffffu, quota);
+    const bool stage = n_out <= (uint32_t)kCpStage;   // else each thread stores its own ids
     uint32_t slot = gtb + min(eqb, quota);
 #pragma unroll
     for (int u = 0; u < kCpMaxU; u++) {
@@ -95,7 +102,9 @@ __global__ void __launch_bounds__(kCpThreads) k_compact(CompactArgs a)
         const int32_t k0 = (int32_t)(t0 + 16 * u);
         while (m) {
             const int bit = __ffs(m) - 1;
-            if ((int64_t)slot < room) {
+            if (stage) {
+                s_ids[slot] = k0 + bit;
+            } else if ((int64_t)slot < room) {
                 out[slot] = k0 + bit;
                 if (dbg) dbg[slot] = k0 + bit;
             }
@@ -105,6 +114,14 @@ __global__ void __launch_bounds__(kCpThreads) k_compact(CompactArgs a)
     }
     if (tid == kCpThreads - 1 && (int64_t)slot > room)
         devchk(a.dev_err, nullptr, DEVCHK_CAND_COUNT, (long long)slot0);
+    if (stage) {                                  // consecutive threads store consecutive slots
+        __syncthreads();
+        const uint32_t lim = room <= 0 ? 0u : ((int64_t)n_out < room ? n_out : (uint32_t)room);
+        for (uint32_t i = tid; i < lim; i += kCpThreads) {
+            out[i] = s_ids[i];
+            if (dbg) dbg[i] = s_ids[i];
+        }
+    }
     pdl_trigger();
 }
 
