@@ -80,12 +80,15 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
     const int r_beg = min(nrows, sp * per), r_end = min(nrows, r_beg + per);
 
     const int64_t qbase = ((int64_t)b_seq * a.H * G + (int64_t)h * G) * kD;
-    for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][qpad(i % kD)] = ld_as_f32(a.q, qbase + i, a.is_bf16);
     if (tid < G) {
         s_m[tid] = -INFINITY;
         s_l[tid] = 0.0f;
     }
     pdl_wait();                                   // the selected ids may come from the search
+    // the first tile's selected ids and the query heads load together (one round trip)
+    const int rr0 = r_beg + tid;
+    const int32_t id0 = (tid < kAtRows && rr0 < r_end && rr0 < a.topk) ? a.idx[(size_t)bh * a.topk + rr0] : 0;
+    for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][qpad(i % kD)] = ld_as_f32(a.q, qbase + i, a.is_bf16);
     const size_t kp = (size_t)index_pair(bh, a.kvg);     // the index pair holding this unit's rows
     const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + kp * a.stride * row_bytes;
     const unsigned char *Vb = reinterpret_cast<const unsigned char *>(a.V) + kp * a.stride * row_bytes;
@@ -105,7 +108,7 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
         if (tid < rows) {
             const int rr = t0 + tid;
             if (rr < a.topk) {
-                const int32_t id = a.idx[(size_t)bh * a.topk + rr];
+                const int32_t id = t0 == r_beg ? id0 : a.idx[(size_t)bh * a.topk + rr];
                 const bool ok = id >= 0 && (int64_t)id < a.n;
                 if (!ok) devchk(a.dev_err, a.dev_err_detail, DEVCHK_BAD_INDEX, id);
                 s_idx[tid] = ok ? id : -1;

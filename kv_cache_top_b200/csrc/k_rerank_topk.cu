@@ -503,7 +503,14 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
     if (tid < 16) sm.slev[tid] = (tid & 8) ? -a.lv.lev[tid & 7] : a.lv.lev[tid & 7];
     pdl_wait();                                   // candidates come from the compaction
     const int32_t *cand = a.cand + (size_t)bh * a.stride + m0;
-    for (int i = tid; i < count; i += NT) keys[i] = (u64)(uint32_t)cand[i];
+    {   // count <= kSelPer NT: every id load of the thread in flight at once
+        int32_t cv[kSelPer];
+#pragma unroll
+        for (int u = 0; u < kSelPer; u++) cv[u] = (tid + u * NT < count) ? cand[tid + u * NT] : 0;
+#pragma unroll
+        for (int u = 0; u < kSelPer; u++)
+            if (tid + u * NT < count) keys[tid + u * NT] = (u64)(uint32_t)cv[u];
+    }
     const int q4 = lane & 3, sub = lane >> 2;          // 32-byte group of the record, record of the round
     float qr[32];
 #pragma unroll
