@@ -229,7 +229,8 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
 }
 
 // Keep the k largest of keys[0..count) (k < count <= kSelPer NT; keys
-// distinct) in sm.tmp[0..k), any order, in one counting pass.  Scores of one
+// distinct) in sm.tmp[0..k), any order, in one counting pass; [vmin, vmax]
+// is the range of the keys' scores (the caller tracks it).  Scores of one
 // query span both signs and a few octaves, so bits of the key spread them
 // poorly; instead bin b(v) = min(255, floor((v - vmin) 256 / (vmax - vmin)))
 // of the score v, which never decreases as the key grows, so every key in a
@@ -241,41 +242,21 @@ __device__ u64 block_topk_select(RrShared &sm, const u64 *keys, int count, int k
 // the boundary bin holds more than 32 keys that must be split; the caller
 // then runs the radix select.  All threads of the block call it.
 template <int NT>
-__device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int count, int k, uint32_t *hist)
+__device__ bool block_topk_select_linear(RrShared &sm, const u64 *keys, int count, int k, uint32_t *hist,
+                                         float vmin, float vmax)
 {
     constexpr int kPer = kSelPer;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     u64 x[kPer];
-    float vmin = INFINITY, vmax = -INFINITY;
 #pragma unroll
     for (int u = 0; u < kPer; u++) {
         const int i = tid + u * NT;
         x[u] = (i < count) ? keys[i] : 0ull;
-        if (i < count) {
-            const float v = unord_f32((uint32_t)(x[u] >> 32));
-            vmin = fminf(vmin, v);
-            vmax = fmaxf(vmax, v);
-        }
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        vmin = fminf(vmin, __shfl_xor_sync(kFull, vmin, o));
-        vmax = fmaxf(vmax, __shfl_xor_sync(kFull, vmax, o));
-    }
-    uint32_t *wh = hist + warp * 256;
+    uint32_t *wh = hist + warp * 256;             // this warp's own counters
 #pragma unroll
     for (int i = 0; i < 8; i++) wh[lane + 32 * i] = 0u;
-    float *red = reinterpret_cast<float *>(&sm.red[0][0]);
-    if (lane == 0) {
-        red[warp] = vmin;
-        red[(NT / 32) + warp] = vmax;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < (NT / 32); w++) {
-        vmin = fminf(vmin, red[w]);
-        vmax = fmaxf(vmax, red[(NT / 32) + w]);
-    }
+    __syncwarp();
     const float range = vmax - vmin;
     const float scale = 256.0f / range;
     if (!(range > 0.0f) || !(range < INFINITY) || !(scale < INFINITY)) {
@@ -516,6 +497,7 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
 #pragma unroll
     for (int i = 0; i < 32; i++) qr[i] = a.qt[(size_t)bh * kD + 32 * q4 + i];
     const float qnorm = a.qnorm[bh];
+    float vlo = INFINITY, vhi = -INFINITY;        // range of this lane's scores (the select's bins)
     const uint8_t *rec = a.rec + (size_t)index_pair(bh, a.kvg) * a.stride * kRecBytes;
     float *dest = a.dbg_est ? a.dbg_est + (size_t)bh * a.C + m0 : nullptr;
     __syncthreads();
@@ -567,6 +549,9 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
             const int r = r0 + j;
             if (q4 == 0 && r < count) {
                 const float est = qnorm * part;
+                const float v = __fadd_rn(est, 0.0f);     // the score the key orders by
+                vlo = fminf(vlo, v);
+                vhi = fmaxf(vhi, v);
                 keys[r] = make_key(est, (int32_t)(uint32_t)keys[r]);
                 if (dest) dest[r] = est;
             }
@@ -575,13 +560,28 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
         issue(t + kRrStages - 1, (t + kRrStages - 1) % kRrStages);
     }
     cp_async_wait<0>();
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        vlo = fminf(vlo, __shfl_xor_sync(kFull, vlo, o));
+        vhi = fmaxf(vhi, __shfl_xor_sync(kFull, vhi, o));
+    }
+    float *red = reinterpret_cast<float *>(&sm.red[0][0]);
+    if (lane == 0) {
+        red[warp] = vlo;
+        red[NW + warp] = vhi;
+    }
     __syncthreads();
+#pragma unroll
+    for (int w = 0; w < NW; w++) {
+        vlo = fminf(vlo, red[w]);
+        vhi = fmaxf(vhi, red[NW + w]);
+    }
 
     // ---- Top-k set of the slice (unordered) and its smallest key
     const int have = min(count, k);
     if (count > k) {
-        // the ring is free now: 8 KB of it hold the per-warp histograms
-        if (!block_topk_select_linear<NT>(sm, keys, count, k, reinterpret_cast<uint32_t *>(ring_all)))
+        // the ring is free now: NW KB of it hold the per-warp histograms
+        if (!block_topk_select_linear<NT>(sm, keys, count, k, reinterpret_cast<uint32_t *>(ring_all), vlo, vhi))
             block_topk_select<NT>(sm, keys, count, k);
     } else {
         for (int i = tid; i < count; i += NT) sm.tmp[i] = keys[i];
