@@ -50,7 +50,7 @@ __device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], u
     return s;
 }
 
-__global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
+__global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
 {
     const int bh = blockIdx.y, chunk = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -82,20 +82,27 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
     // and iterations that lie wholly inside the chunk skip the per-key checks.
     const uint32_t ucnt = (uint32_t)cnt;
     uint32_t *hw = s_hist[warp];
-    for (uint32_t base = (uint32_t)warp * 32 * kScanUnroll + lane; base < ucnt + lane;
-         base += (uint32_t)NW * 32 * kScanUnroll) {
-        const bool full = base - lane + 32 * kScanUnroll <= ucnt;
-        uint4 c[kScanUnroll];
-        if (full) {
+    // the next iteration's codes load while this one is scored (registers
+    // double-buffered), so a warp always has a load in flight
+    const uint32_t step = (uint32_t)NW * 32 * kScanUnroll;
+    auto load = [&](uint32_t b, uint4 (&c)[kScanUnroll]) {
+        if (b - lane + 32 * kScanUnroll <= ucnt) {
 #pragma unroll
-            for (int u = 0; u < kScanUnroll; u++) c[u] = __ldcs(codes + base + u * 32);
+            for (int u = 0; u < kScanUnroll; u++) c[u] = __ldcs(codes + b + u * 32);
         } else {
 #pragma unroll
             for (int u = 0; u < kScanUnroll; u++) {
-                const uint32_t i = base + u * 32;
+                const uint32_t i = b + u * 32;
                 c[u] = (i < ucnt) ? __ldcs(codes + i) : make_uint4(0, 0, 0, 0);
             }
         }
+    };
+    uint4 c[kScanUnroll], cn[kScanUnroll];
+    uint32_t base = (uint32_t)warp * 32 * kScanUnroll + lane;
+    if (base < ucnt + lane) load(base, c);
+    for (; base < ucnt + lane; base += step) {
+        const bool full = base - lane + 32 * kScanUnroll <= ucnt;
+        if (base + step < ucnt + lane) load(base + step, cn);
         uint32_t sc[kScanUnroll];
 #pragma unroll
         for (int u = 0; u < kScanUnroll; u++) sc[u] = collision_score(tab, c[u]);
@@ -120,6 +127,8 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan(ScanArgs a)
                 }
             }
         }
+#pragma unroll
+        for (int u = 0; u < kScanUnroll; u++) c[u] = cn[u];
     }
     __syncthreads();
 
