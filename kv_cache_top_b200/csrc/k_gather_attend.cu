@@ -49,7 +49,7 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // size of the partials region (dynamic shared memory): [nsplit][G][kD] fp32
 size_t attend_smem(int nsplit, int G) { return (size_t)nsplit * G * kD * sizeof(float); }
 
-__global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
+__global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
 {
     // the K and V tiles
     __shared__ __align__(16) unsigned char s_kv[2 * kAtRows * kD * 4];
@@ -218,14 +218,14 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
             const float m_new = fmaxf(m_old, mx);
             float sum = 0.0f;
             for (int r = lane; r < rows; r += 32) {
-                const float p = (m_new == -INFINITY) ? 0.0f : expf(s_p[g][r] - m_new);
+                const float p = (m_new == -INFINITY) ? 0.0f : __expf(s_p[g][r] - m_new);
                 s_p[g][r] = p;
                 sum += p;
             }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
             if (lane == 0) {
-                const float alpha = (m_old == -INFINITY) ? 0.0f : expf(m_old - m_new);
+                const float alpha = (m_old == -INFINITY) ? 0.0f : __expf(m_old - m_new);
                 s_alpha[g] = alpha;
                 s_l[g] = s_l[g] * alpha + sum;
                 s_m[g] = m_new;
@@ -233,19 +233,18 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
         }
         __syncthreads();
         // ---- P V: thread owns dim d of heads gsel, gsel + 2, ...
+        // (one V element per row, used by every head this thread owns)
 #pragma unroll
-        for (int i = 0; i < kMaxGroup / 2; i++) {
-            const int g = gsel + 2 * i;
-            if (g < G) {
-                float v = acc[i] * s_alpha[g];
-                for (int r = 0; r < rows; r++) {
-                    const float vv = a.is_bf16
-                        ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sV + (size_t)r * row_bytes)[d])
-                        : reinterpret_cast<const float *>(sV + (size_t)r * row_bytes)[d];
-                    v = fmaf(s_p[g][r], vv, v);
-                }
-                acc[i] = v;
-            }
+        for (int i = 0; i < kMaxGroup / 2; i++)
+            if (gsel + 2 * i < G) acc[i] *= s_alpha[gsel + 2 * i];
+#pragma unroll 4
+        for (int r = 0; r < rows; r++) {
+            const float vv = a.is_bf16
+                ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sV + (size_t)r * row_bytes)[d])
+                : reinterpret_cast<const float *>(sV + (size_t)r * row_bytes)[d];
+#pragma unroll
+            for (int i = 0; i < kMaxGroup / 2; i++)
+                if (gsel + 2 * i < G) acc[i] = fmaf(s_p[gsel + 2 * i][r], vv, acc[i]);
         }
     }
     // ---- push this CTA's partial into rank 0 (remote stores: no round trip)
@@ -265,23 +264,32 @@ __global__ void __launch_bounds__(kAtThreads, 4) k_gather_attend(AttendArgs a)
     cluster_arrive();
     cluster_wait();                                   // every partial has landed in rank 0
     if (sp == 0) {
-        // log-sum-exp merge of the nsp partials, from local shared memory
+        // log-sum-exp merge of the nsp partials, from local shared memory: the
+        // weight e^(m_r - M) / sum_r' e^(m_r' - M) l_r' of partial r and head g
+        // once per (r, g), then one weighted sum per output
+        __shared__ float s_w[8][kMaxGroup];
+        if (tid < G) {
+            const int g = tid;
+            float M = -INFINITY;
+            for (int r = 0; r < nsp; r++) M = fmaxf(M, s_pm[r][g]);
+            float den = 0.0f;
+            for (int r = 0; r < nsp; r++) {
+                const float mr = s_pm[r][g];
+                const float f = (M == -INFINITY || mr == -INFINITY) ? 0.0f : __expf(mr - M);
+                s_w[r][g] = f;
+                den = fmaf(f, s_pl[r][g], den);
+            }
+            const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+            for (int r = 0; r < nsp; r++) s_w[r][g] *= inv;
+        }
+        __syncthreads();
 #pragma unroll
         for (int i = 0; i < kMaxGroup / 2; i++) {
             const int g = gsel + 2 * i;
             if (g >= G) continue;
-            float M = -INFINITY;
-            for (int r = 0; r < nsp; r++) M = fmaxf(M, s_pm[r][g]);
-            float num = 0.0f, den = 0.0f;
-            if (M != -INFINITY) {
-                for (int r = 0; r < nsp; r++) {
-                    const float mr = s_pm[r][g];
-                    const float f = (mr == -INFINITY) ? 0.0f : expf(mr - M);
-                    num = fmaf(f, s_pacc[((size_t)r * G + g) * kD + d], num);
-                    den = fmaf(f, s_pl[r][g], den);
-                }
-            }
-            a.out[qbase + (int64_t)g * kD + d] = (den > 0.0f) ? num / den : 0.0f;
+            float num = 0.0f;
+            for (int r = 0; r < nsp; r++) num = fmaf(s_w[r][g], s_pacc[((size_t)r * G + g) * kD + d], num);
+            a.out[qbase + (int64_t)g * kD + d] = num;
         }
     }
 }
