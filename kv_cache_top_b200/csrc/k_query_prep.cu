@@ -11,25 +11,29 @@
 //     better-ranked buckets (from the occupancy table), and a bucket inside
 //     the top-rho fraction (P(c) < R = ceil(rho n)) gets bonus 6 - floor(6P/R).
 //
-// Grid (8, pairs): a CTA of 256 threads takes 2 blocks, one 128-thread half
-// per block.  The kernel is a latency chain, so its steps are laid out for a
-// short critical path with little repeated work: every global load is issued
-// up front (no load waits on another), warp 0 aggregates and rotates the
-// query once and shares it through shared memory, each half ranks the 256
-// centres of its block by a bitonic sort holding 2 keys per thread (shuffles
-// inside a warp; shared memory for the 3 stages that cross warps), a scan
-// over the half turns bucket sizes in rank order into P(c), and one warp per
-// half packs the bonus table 4 bits per centre in the layout the collision
-// scan keeps in registers -- lane l's word holds the bonus of centre 32 t + l
-// in the 4 bits starting at bit (4 t + r(l)) mod 32, r(l) = (l >> 3) & 3.
+// Grid (2, pairs): a CTA of 8 warps takes 8 blocks, one warp per block, so
+// a block's ranking needs no block barrier.  Warp 0 aggregates and rotates
+// the query once per CTA and shares it through shared memory.  Flipping all 8
+// signs of a centre negates its score exactly (fp32 addition is symmetric
+// under negation), so the 128 centres with bit 7 clear are sorted -- 4 keys
+// per lane, in registers and shuffles -- and the other 128 are their mirror
+// images in reverse order: the 256 keys then form an ascending run followed
+// by a descending one, and one 8-stage bitonic merge ranks them all.  A warp
+// scan turns bucket sizes in rank order into P(c), and the warp packs the
+// bonus table 4 bits per centre in the layout the collision scan keeps in
+// registers -- lane l's word holds the bonus of centre 32 t + l in the 4 bits
+// starting at bit (4 t + r(l)) mod 32, r(l) = (l >> 3) & 3.
 #include "pk_internal.cuh"
 
 namespace pk {
 
+constexpr int kQpWarps = 8;                   // blocks per CTA, one warp each
+constexpr int kQpThreads = 32 * kQpWarps;
+
 constexpr int kQpHalf = 128;                  // threads per block of centres
 constexpr int kQpBlocks = 2;                  // blocks per CTA
-constexpr int kQpThreads = kQpHalf * kQpBlocks;
-constexpr int kQpWarps = kQpThreads / 32;
+constexpr int kQwThreads = kQpHalf * kQpBlocks;
+constexpr int kQwWarps = kQwThreads / 32;
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -56,9 +60,187 @@ __device__ __forceinline__ uint32_t tier_bonus(uint32_t P, unsigned long long R)
            (uint32_t)(p6 >= 4 * R) - (uint32_t)(p6 >= 5 * R);
 }
 
+typedef unsigned long long u64;
+
+// sort key of a centre: ascending key order = rank order (score desc, id asc)
+__device__ __forceinline__ u64 centre_key(float L, uint32_t c)
+{
+    return ((u64)(~ord_f32(__fadd_rn(L, 0.0f))) << 8) | c;   // +0 folds -0: equal scores tie
+}
+
+// the key of the mirror centre c ^ 0xff, whose score is exactly -L
+__device__ __forceinline__ u64 mirror_key(u64 key)
+{
+    const float L = unord_f32(~(uint32_t)(key >> 8));
+    return centre_key(-L, (uint32_t)(key & 0xffu) ^ 0xffu);
+}
+
+__device__ __forceinline__ void cmp_swap(u64 &lo, u64 &hi, bool up)
+{
+    const u64 a = lo < hi ? lo : hi, b = lo < hi ? hi : lo;
+    lo = up ? a : b;
+    hi = up ? b : a;
+}
+
 __global__ void __launch_bounds__(kQpThreads) k_query_prep(PrepArgs a)
 {
-    typedef unsigned long long u64;
+    const int bh = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = kQpWarps * blockIdx.x + warp;              // this warp's block
+    const int b_seq = bh / a.H, h = bh - b_seq * a.H;
+    __shared__ __align__(16) uint32_t s_occ[kQpWarps][kNC];
+    __shared__ float s_x[kD];
+    __shared__ uint8_t s_bonus[kQpWarps][kNC];
+
+    if (blockIdx.x == 0) {   // reset the per-call counters of the collision scan and the rerank
+        for (int i = tid; i < kBins; i += kQpThreads) a.head_hist[(size_t)bh * kBins + i] = 0u;
+        if (tid < 2) a.tickets[(size_t)bh * 2 + tid] = 0u;
+    }
+    // global loads first: 8 bucket sizes per lane; warp 0 the G query heads
+    const uint4 *occ = reinterpret_cast<const uint4 *>(a.occ + ((size_t)index_pair(bh, a.kvg) * kB + b) * kNC);
+    const uint4 o0 = occ[2 * lane], o1 = occ[2 * lane + 1];
+    if (warp == 0) {
+        float qv[4][kMaxGroup];
+        const int64_t base = ((int64_t)b_seq * a.H * a.G + (int64_t)h * a.G) * kD;
+        if (a.is_bf16)
+            load_heads(qv, reinterpret_cast<const __nv_bfloat16 *>(a.q) + base, a.G, lane);
+        else
+            load_heads(qv, reinterpret_cast<const float *>(a.q) + base, a.G, lane);
+        float x[4];
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+            float acc = qv[r][0];
+#pragma unroll
+            for (int g = 1; g < kMaxGroup; g++)
+                if (g < a.G) acc = __fadd_rn(acc, qv[r][g]);
+            x[r] = acc;
+        }
+        const float nrm = warp_rotate128(x, a.rot, lane);
+#pragma unroll
+        for (int r = 0; r < 4; r++) s_x[lane + 32 * r] = x[r];
+        if (blockIdx.x == 0) {
+#pragma unroll
+            for (int r = 0; r < 4; r++) {
+                a.qt[(size_t)bh * kD + lane + 32 * r] = x[r];
+                if (a.dbg_qt) a.dbg_qt[(size_t)bh * kD + lane + 32 * r] = x[r];
+            }
+            if (lane == 0) {
+                a.qnorm[bh] = nrm;
+                if (a.dbg_qnorm) a.dbg_qnorm[bh] = nrm;
+            }
+        }
+    }
+    reinterpret_cast<uint4 *>(s_occ[warp])[2 * lane] = o0;
+    reinterpret_cast<uint4 *>(s_occ[warp])[2 * lane + 1] = o1;
+    __syncthreads();
+    float xq[kM];
+#pragma unroll
+    for (int j = 0; j < kM; j++) xq[j] = s_x[kM * b + j];
+
+    // the 128 centres with bit 7 clear, element e = 4 lane + i holding centre e;
+    // L(c) = sum_j +-q~_j (minus where bit j of c is set), summed in j order
+    u64 v[8];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint32_t c = 4 * lane + i;
+        float L = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kM; j++) L = __fadd_rn(L, ((c >> j) & 1) ? -xq[j] : xq[j]);
+        v[i] = centre_key(L, c);
+    }
+    // bitonic sort of the 128 keys, ascending: strides 1, 2 inside a lane,
+    // 4 .. 64 across lanes (lane ^ stride / 4)
+#pragma unroll
+    for (int k = 2; k <= 128; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j < 4) {
+#pragma unroll
+                for (int i = 0; i < 4; i++)
+                    if ((i & j) == 0) cmp_swap(v[i], v[i | j], ((4 * lane + i) & k) == 0);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const u64 o = __shfl_xor_sync(kFull, v[i], j >> 2);
+                    const int e = 4 * lane + i;
+                    const bool take_min = ((e & j) == 0) == ((e & k) == 0);
+                    v[i] = take_min ? (o < v[i] ? o : v[i]) : (o > v[i] ? o : v[i]);
+                }
+            }
+        }
+    }
+    // positions 128 + 4 lane + i: the mirror of position 4 lane + i, so the
+    // second half descends; an 8-stage bitonic merge sorts all 256
+#pragma unroll
+    for (int i = 0; i < 4; i++) v[4 + i] = mirror_key(v[i]);
+#pragma unroll
+    for (int i = 0; i < 4; i++) cmp_swap(v[i], v[4 + i], true);           // stride 128
+#pragma unroll
+    for (int j = 64; j >= 4; j >>= 1) {                                       // across lanes
+        const bool lower = ((4 * lane) & j) == 0;                             // keeps the smaller key
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const u64 o = __shfl_xor_sync(kFull, v[i], j >> 2);
+            v[i] = lower ? (o < v[i] ? o : v[i]) : (o > v[i] ? o : v[i]);
+        }
+    }
+#pragma unroll
+    for (int hh = 0; hh < 8; hh += 4) {                                      // strides 2, 1
+        cmp_swap(v[hh + 0], v[hh + 2], true);
+        cmp_swap(v[hh + 1], v[hh + 3], true);
+        cmp_swap(v[hh + 0], v[hh + 1], true);
+        cmp_swap(v[hh + 2], v[hh + 3], true);
+    }
+
+    // P(c): bucket sizes of the better-ranked centres (rank p = 4 lane + i,
+    // then 128 + 4 lane + i), by a lane prefix and a warp scan per half
+    uint32_t n[8], pre[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) n[i] = s_occ[warp][v[i] & 0xffu];
+    uint32_t half_base = 0;
+#pragma unroll
+    for (int hh = 0; hh < 8; hh += 4) {
+        uint32_t run = 0;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            pre[hh + i] = run;
+            run += n[hh + i];
+        }
+        uint32_t incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - run + half_base;
+#pragma unroll
+        for (int i = 0; i < 4; i++) pre[hh + i] += excl;
+        half_base += __shfl_sync(kFull, incl, 31);
+    }
+    const unsigned long long R = (unsigned long long)a.R;
+    uint8_t *db = a.dbg_bonus ? a.dbg_bonus + ((size_t)bh * kB + b) * kNC : nullptr;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        const uint32_t c = (uint32_t)(v[i] & 0xffu);
+        const uint8_t bon = (uint8_t)tier_bonus(pre[i], R);
+        s_bonus[warp][c] = bon;
+        if (db) db[c] = bon;
+    }
+    __syncwarp();
+    uint32_t word = 0;
+#pragma unroll
+    for (int tt = 0; tt < 8; tt++) word |= (uint32_t)s_bonus[warp][32 * tt + lane] << (4 * tt);
+    const uint32_t rl = (uint32_t)(lane >> 3) & 3u;
+    a.bonus_packed[((size_t)bh * kB + b) * 32 + lane] = __funnelshift_l(word, word, rl);
+}
+
+// The same preparation with 4 warps per block (2 blocks per 256-thread CTA,
+// grid (8, pairs)): each 128-thread half ranks its block's 256 centres by a
+// bitonic sort holding 2 keys per thread (shuffles inside a warp, shared
+// memory for the 3 stages that cross warps).  Shorter per block than the warp
+// version, so it is taken when there are few pairs and the SMs have room.
+__global__ void __launch_bounds__(kQwThreads) k_query_prep_wide(PrepArgs a)
+{
     const int bh = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int half = tid / kQpHalf, t = tid % kQpHalf;      // t: thread within the half
@@ -67,11 +249,11 @@ __global__ void __launch_bounds__(kQpThreads) k_query_prep(PrepArgs a)
     __shared__ uint32_t s_occ[kQpBlocks][kNC];
     __shared__ u64 s_key[2][kQpBlocks][kNC];
     __shared__ float s_x[kD];
-    __shared__ uint32_t s_ws[kQpWarps];
+    __shared__ uint32_t s_ws[kQwWarps];
     __shared__ uint8_t s_bonus[kQpBlocks][kNC];
 
     if (blockIdx.x == 0) {   // reset the per-call counters of the collision scan and the rerank
-        for (int i = tid; i < kBins; i += kQpThreads) a.head_hist[(size_t)bh * kBins + i] = 0u;
+        for (int i = tid; i < kBins; i += kQwThreads) a.head_hist[(size_t)bh * kBins + i] = 0u;
         if (tid < 2) a.tickets[(size_t)bh * 2 + tid] = 0u;
     }
     // global loads: 2 bucket sizes per thread; warp 0 the G query heads
@@ -194,7 +376,11 @@ __global__ void __launch_bounds__(kQpThreads) k_query_prep(PrepArgs a)
 
 cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s)
 {
-    k_query_prep<<<dim3(kB / kQpBlocks, a.bh), kQpThreads, 0, s>>>(a);
+    static_assert(kB % kQpWarps == 0 && kB % kQpBlocks == 0, "whole blocks per CTA");
+    if (a.wide)
+        k_query_prep_wide<<<dim3(kB / kQpBlocks, a.bh), kQwThreads, 0, s>>>(a);
+    else
+        k_query_prep<<<dim3(kB / kQpWarps, a.bh), kQpThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -354,6 +354,8 @@ pk_status search_impl(pk_index *ix, Work &w, int32_t kvg, const void *q, int32_t
     pa.kvg = kvg;
     pa.is_bf16 = ix->p.kv_dtype == PK_BF16;
     pa.bh = w.units;
+    // one warp per block unless the 4-warp layout still fits about two CTAs per SM
+    pa.wide = (int64_t)w.units * (kB / 2) <= 2 * (int64_t)ix->num_sms;
     pa.R = R;
     pa.occ = ix->occ;
     pa.rot = ix->rot;

@@ -59,6 +59,7 @@ struct PrepArgs {
     int32_t H, G, is_bf16, bh;
     int64_t R;               // collision budget ceil(rho n)
     int32_t kvg;             // query units per index pair (1, or G for per-head search)
+    int32_t wide;            // 1: 4 warps per block (few pairs); 0: one warp per block
     const uint32_t *occ;
     RotConst rot;
     float *qt;               // [BH][D]
