@@ -442,6 +442,24 @@ def test_many_pairs_small_rerank_ctas(pk):
         torch.cuda.empty_cache()
 
 
+def test_compaction_large_chunks_every_key_a_candidate(pk):
+    """40 pairs of n = 70000 with C = n: 14 chunks of ~5000 keys per pair, so
+    a chunk holds more candidates than the compaction stages in shared memory
+    and its threads store their ids directly.  Three pairs checked element by
+    element."""
+    batch, n, H, G = 40, 70000, 1, 1
+    w = workloads.llama_layer(batch, n, H=H, G=G, seed=77, device="cuda", n_queries=1)
+    h = build(pk, w["K"], w["V"], n, batch, H, G, cand_budget=n)
+    try:
+        assert pk.pk_get_info(h).nchunks <= 16
+        check_pairs(pk, h, w["K"], w["V"], w["q"][0], [0, 17, 39], batch, H, G, n, 100, cand_budget=n,
+                    check_encode=False)
+    finally:
+        pk.pk_free(h)
+        del w
+        torch.cuda.empty_cache()
+
+
 # ------------------------------------------------- full-size workloads
 def test_throughput_batch_full_size_sampled(pk):
     """8 sequences x n = 131072, 8 KV heads, 32 query heads, bf16, ratio-table
