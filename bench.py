@@ -198,6 +198,17 @@ def profiled_traffic(kernel: str, workload: str):
     return float(m.group(1))
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (for the CPU-baseline lines)."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 # -------------------------------------------------------- algorithmic bytes
 def alg_bytes(kernel: str, wl: dict, C: int, topk: int = 100):
     """Bytes a launch must move at minimum (per launch, all pairs)."""
@@ -449,7 +460,7 @@ def cpu_baseline(wl, seed, w, dev, pairs_wanted=4, queries=32):
             tot += time.perf_counter() - t0
             cnt += 1
     per_pair = tot / cnt
-    return {"value": 1.0 / (per_pair * bh), "unit": "steps/s", "cores": 1, "kind": "oracle",
+    return {"value": 1.0 / (per_pair * bh), "unit": "steps/s", "cores": 1, "kind": "oracle", "cpu": cpu_model(),
             "sample": "%d of %d (sequence, KV head) pairs x %d queries each (%.1f s of timed "
                       "search+attend, index build untimed); one step = %d pair-searches" %
                       (len(pairs), bh, queries, tot, bh),
@@ -500,7 +511,7 @@ def cpu_baseline_parallel(wl, seed, queries=64, max_workers=32):
         res = list(ex.map(_oracle_worker, jobs, timeout=900))
     done = sum(r[0] for r in res)
     tmax = max(r[1] for r in res)
-    return {"value": done / tmax / bh, "unit": "steps/s", "cores": P, "kind": "oracle",
+    return {"value": done / tmax / bh, "unit": "steps/s", "cores": P, "kind": "oracle", "cpu": cpu_model(),
             "sample": "%d processes, one (sequence, KV head) pair each, %d queries each, timed together "
                       "(%.1f s; index build untimed); one step = %d pair-searches" % (P, queries, tmax, bh)}
 
@@ -898,7 +909,7 @@ def run_reference(args, rank, world):
             "data": "synthetic",
             "config": {"workload": wl["name"], "batch": batch, "n": n, "kv_heads": H, "q_heads": H * G,
                        "head_dim": 128, "topk": 100},
-            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle", "cpu": cpu_model(),
                              "sample": "each timed step = one of %d sampled pairs (search + attend); "
                                        "value = 1 / (mean pair time x %d pairs)" % (npairs, bh)},
             "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
