@@ -22,7 +22,9 @@
 // scan turns bucket sizes in rank order into P(c), and the warp packs the
 // bonus table 4 bits per centre in the layout the collision scan keeps in
 // registers -- lane l's word holds the bonus of centre 32 t + l in the 4 bits
-// starting at bit (4 t + r(l)) mod 32, r(l) = (l >> 3) & 3.
+// starting at bit (4 t + r(l)) mod 32, r(l) = (l >> 3) & 3.  With few pairs
+// the SMs have room for more parallelism per block, and k_query_prep_wide
+// (4 warps per block) runs instead; the host chooses.
 #include "pk_internal.cuh"
 
 namespace pk {
@@ -30,6 +32,7 @@ namespace pk {
 constexpr int kQpWarps = 8;                   // blocks per CTA, one warp each
 constexpr int kQpThreads = 32 * kQpWarps;
 
+// the 4-warp layout (k_query_prep_wide)
 constexpr int kQpHalf = 128;                  // threads per block of centres
 constexpr int kQpBlocks = 2;                  // blocks per CTA
 constexpr int kQwThreads = kQpHalf * kQpBlocks;
