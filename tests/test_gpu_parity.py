@@ -126,6 +126,7 @@ def test_llama_shaped_layer_config(pk):
     (40000, 0, 256, 1, 2, 1),     # topk > 128 over several slices: shared-memory merge tree
     (60000, 0, 1024, 1, 2, 2),    # the largest topk: 1024-key selects and merges
     (70001, 70001, 100, 1, 2, 1), # every key a candidate (C = n)
+    (400000, 0, 200, 1, 1, 1),    # 100 slices x 200 keys > the merge's 16384: rounds of radix select
 ])
 def test_edge_and_ragged_sizes(pk, n, cand, topk, batch, H, G):
     w = workloads.llama_layer(batch, n, H=H, G=G, seed=n, device="cuda")
