@@ -28,6 +28,7 @@
 #include <cooperative_groups.h>
 
 #include "pk_internal.cuh"
+#include "pk_launch.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -296,13 +297,9 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
 
 cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s)
 {
-    static int attr_set = 0;                      // per process: the partials region may pass 48 KB in total
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(k_gather_attend, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)attend_smem(8, kMaxGroup));
-        if (e != cudaSuccess) return e;
-        attr_set = 1;
-    }
+    static std::atomic<int> smem_set[kMaxDevices];   // the partials region may pass 48 KB in total
+    const cudaError_t e = dyn_smem_limit(k_gather_attend, (int)attend_smem(8, kMaxGroup), smem_set);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.nsplit, bh, 1);
     cfg.blockDim = dim3(kAtThreads, 1, 1);

@@ -30,6 +30,7 @@
 // (README: "reranks those candidates with a fused 4-bit approximate
 // inner-product kernel and selects the final Top-k KV indices").
 #include "pk_internal.cuh"
+#include "pk_launch.cuh"
 #include "pk_merge.cuh"
 
 namespace pk {
@@ -698,14 +699,10 @@ size_t merge_smem(int cap) { return (size_t)merge_keys(cap) * sizeof(u64); }
 
 cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s)
 {
-    static int attr_max = 0;
+    static std::atomic<int> smem_set[kMaxDevices];
     const size_t smem = merge_smem(a.cap);
-    if ((int)smem > attr_max) {
-        cudaError_t e = cudaFuncSetAttribute(k_topk_merge, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)merge_smem(kMergeCap));
-        if (e != cudaSuccess) return e;
-        attr_max = (int)merge_smem(kMergeCap);
-    }
+    const cudaError_t e = dyn_smem_limit(k_topk_merge, (int)merge_smem(kMergeCap), smem_set);
+    if (e != cudaSuccess) return e;
     return launch_pdl(k_topk_merge, dim3(bh), dim3(kRrThreads), smem, s, a);
 }
 
@@ -714,14 +711,10 @@ size_t rerank_smem(int slice, int nt) { return rr_ring_bytes(nt) + (size_t)slice
 template <int NT>
 cudaError_t launch_rerank_nt(const RerankArgs &a, int bh, cudaStream_t s)
 {
-    static int attr_max = 0;
+    static std::atomic<int> smem_set[kMaxDevices];
     const size_t smem = rerank_smem(a.slice, NT);
-    if ((int)smem > attr_max) {
-        const int most = (int)rerank_smem(kSelPer * NT, NT);
-        cudaError_t e = cudaFuncSetAttribute(k_rerank_topk<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-        if (e != cudaSuccess) return e;
-        attr_max = most;
-    }
+    const cudaError_t e = dyn_smem_limit(k_rerank_topk<NT>, (int)rerank_smem(kSelPer * NT, NT), smem_set);
+    if (e != cudaSuccess) return e;
     return launch_pdl(k_rerank_topk<NT>, dim3(a.nslices, bh), dim3(NT), smem, s, a);
 }
 
