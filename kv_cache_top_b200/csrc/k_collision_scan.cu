@@ -8,10 +8,12 @@
 // last CTA of a pair to finish (ticket counter, no spin-wait) finds the
 // threshold s* = max{s : #{S >= s} >= C}, and for every chunk the first slot of
 // its candidates and how many of its S = s* keys it keeps (lower ids first),
-// so the rerank kernel can compact candidates in ascending id order without
+// so the compaction kernel can place candidates in ascending id order without
 // any further global synchronisation.
 //
-// Hot loop: 16 B of codes per key read with 128-bit streaming loads; the 16
+// Hot loop: 16 B of codes per key read with 128-bit streaming loads,
+// double-buffered in registers (the next iteration's codes are in flight
+// while the current ones are scored); the 16
 // bonus tables (4 bits x 256 centres = one 32-bit register per lane per
 // block) live in registers and are read with warp shuffles, which have no
 // bank conflicts whatever the codes are.  Lane l's word of block b holds the
