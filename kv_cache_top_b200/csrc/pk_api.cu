@@ -76,7 +76,8 @@ pk_status cuda_status(cudaError_t e)
     return PK_ERR_CUDA;
 }
 
-// A pointer the GPU can read: device memory or page-locked host memory.
+// A pointer the GPU can read: device memory of the current device, or
+// page-locked / managed host memory.
 bool device_accessible(const void *ptr)
 {
     if (!ptr) return false;
@@ -85,8 +86,13 @@ bool device_accessible(const void *ptr)
         cudaGetLastError();
         return false;
     }
-    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeHost ||
-           at.type == cudaMemoryTypeManaged;
+    if (at.type == cudaMemoryTypeDevice) {
+        // device memory of another GPU is not read through here: the kernels
+        // launch on the current device
+        int dev = -1;
+        return cudaGetDevice(&dev) == cudaSuccess && at.device == dev;
+    }
+    return at.type == cudaMemoryTypeHost || at.type == cudaMemoryTypeManaged;
 }
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }

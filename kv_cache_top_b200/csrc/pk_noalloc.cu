@@ -182,6 +182,7 @@ pk_status na_scratch(NaScratch **out)
     return PK_OK;
 }
 
+// Device memory of the current device, or page-locked / managed host memory.
 bool na_device_accessible(const void *ptr)
 {
     cudaPointerAttributes at;
@@ -189,8 +190,13 @@ bool na_device_accessible(const void *ptr)
         cudaGetLastError();
         return false;
     }
-    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeHost ||
-           at.type == cudaMemoryTypeManaged;
+    if (at.type == cudaMemoryTypeDevice) {
+        // device memory of another GPU is not read through here: the kernels
+        // launch on the current device
+        int dev = -1;
+        return cudaGetDevice(&dev) == cudaSuccess && at.device == dev;
+    }
+    return at.type == cudaMemoryTypeHost || at.type == cudaMemoryTypeManaged;
 }
 
 }  // namespace

@@ -69,3 +69,23 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(pk):
     with pytest.raises(pk.PkError) as e:
         pk.pk_select_candidates_noalloc(S, 16, 17, cand)
     assert e.value.status == 1
+
+
+@pytest.mark.parametrize("n,C,hi", [
+    (4194304, 300000, 256),   # the largest row (256 chunks), byte scores over the whole 0..255 range
+    (1000003, 1000003, 256),  # C == n: every key
+    (1000003, 123457, 4),     # four distinct scores: the threshold's ties span many chunks
+    (65537, 1, 97),           # one candidate, ragged last chunk
+])
+def test_noalloc_synthetic_rows(pk, n, C, hi):
+    """Synthetic score rows (not produced by a scan): the candidate set is the
+    Top-C by (score desc, id asc) in ascending id order, on two calls in a row."""
+    g = torch.Generator(device="cuda").manual_seed(n + C)
+    S = torch.randint(0, hi, (n,), generator=g, device="cuda", dtype=torch.int32).to(torch.uint8)
+    s = S.cpu().numpy().astype(np.int64)
+    ref = np.sort(np.lexsort((np.arange(n), -s))[:C]).astype(np.int32)
+    for _ in range(2):
+        cand = torch.full((C,), -1, dtype=torch.int32, device="cuda")
+        pk.pk_select_candidates_noalloc(S, n, C, cand)
+        torch.cuda.synchronize()
+        assert np.array_equal(cand.cpu().numpy(), ref)
