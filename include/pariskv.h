@@ -13,11 +13,11 @@
  *                   bit + 3-bit Lloyd-Max magnitude index per coordinate, one
  *                   fp32 weight per block) on the GPU; copy K/V into
  *                   index-owned storage in HBM or pinned host memory.
- *                   [readme] "Prefill: build compact retrieval metadata";
- *                   [slides] Eqs. (5)-(10).
+ *                   [readme] pipeline step 1 (prefill builds the compact
+ *                   retrieval metadata); [slides] Eqs. (5)-(10).
  *   pk_append       index newly decoded keys with the same fixed codebook
- *                   ([slides] "new decode keys can be indexed without
- *                   retraining centroids").
+ *                   ([slides] Sec. 4.1.2: the codebook is fixed, so new
+ *                   keys are encoded without retraining centroids).
  *   pk_search       per (sequence, KV head): GQA-aggregate and rotate the
  *                   query, rank the sign-pattern buckets of every block, give
  *                   buckets inside the top-rho fraction one of six tier
@@ -29,8 +29,8 @@
  *   pk_attend       exact softmax attention of every query head over the
  *                   selected full-precision K/V rows, read from HBM or, for
  *                   host-resident K/V, over the host link through UVA
- *                   ([slides] Sec. 3 Eqs. (1)-(3); [readme] "Attention: fetch
- *                   only selected KV pairs").
+ *                   ([slides] Sec. 3 Eqs. (1)-(3); [readme] pipeline step 3:
+ *                   only the selected K/V pairs are fetched).
  *
  * Conventions for every call:
  *   - D (head_dim) must be 128 and m (sub_dim) must be 8 (B = 16 blocks of
@@ -172,8 +172,8 @@ pk_status pk_attend(pk_index *index, const void *q, const int32_t *sel_idx, int3
 
 /* Exact attention over the selected rows together with rows kept densely on
  * the GPU outside the index -- the sink tokens and the recent local window --
- * under one softmax (README, step 3: attention "over sink tokens, local
- * tokens, and retrieved tokens"; slides, Fig. 5: sink and local tokens stay
+ * under one softmax (README, pipeline step 3: the sink, local and retrieved
+ * tokens are attended together; slides, Fig. 5: sink and local tokens stay
  * on the GPU for dense attention while the retrieval region is searched).
  *   q, sel_idx, topk, out  as for pk_attend, except that topk may be 0
  *            (dense rows only; sel_idx may then be NULL).

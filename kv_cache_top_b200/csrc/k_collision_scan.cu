@@ -1,10 +1,10 @@
 // k_collision_scan.cu -- multi-tier collision counting and the integer Top-C
 // threshold.
 //
-// S_i = sum_b bonus_b[code_{i,b}]  (ParisKV slides, "Stage I uses multi-tier
-// collision votes to prune keys", App. B.2.1 Eq. 15), an integer in [0, 96].
-// "Small integer scores allow histogram and prefix-scan selection instead of a
-// full sort" (same frame): each CTA histograms the S of its chunk, and the
+// S_i = sum_b bonus_b[code_{i,b}]  (ParisKV slides, Sec. 4.2.2 and App. B.2.1
+// Eq. 15), an integer in [0, 96].  Because S takes so few values, the Top-C
+// by S needs no sort: a histogram and a prefix scan fix the threshold (same
+// section).  Each CTA histograms the S of its chunk, and the
 // last CTA of a pair to finish (ticket counter, no spin-wait) finds the
 // threshold s* = max{s : #{S >= s} >= C}, and for every chunk the first slot of
 // its candidates and how many of its S = s* keys it keeps (lower ids first),

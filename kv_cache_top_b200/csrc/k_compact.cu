@@ -1,7 +1,8 @@
 // k_compact.cu -- the candidate set of each pair, in ascending key order.
 //
-// Candidates (ParisKV slides, Sec. 4.2.2 "choose the top-beta keys by S_i"
-// and Sec. 4.3 "rerank C = ceil(beta n)"): every key with S > s*, then the
+// Candidates (ParisKV slides, Sec. 4.2.2: the keys with the largest collision
+// scores S_i; Sec. 4.3: a budget of C = ceil(beta n) of them are reranked):
+// every key with S > s*, then the
 // lowest-id keys with S = s* until C are taken.  The collision scan already
 // fixed, per chunk of keys, the first output slot and how many of the chunk's
 // S = s* keys it keeps; here each CTA loads its whole chunk of S at once (up

@@ -1,8 +1,8 @@
 // k_encode.cu -- key encoding for pk_build_index / pk_append.
 //
-// Per key (ParisKV slides, "Normalization and rotation enable a fixed
-// codebook", Eqs. 5-6, and "Stage II estimates the raw attention score from
-// 4-bit codes", Eqs. 7-10):
+// Per key (ParisKV slides, Sec. 4.1.1-4.1.2 Eqs. 5-6: normalise and rotate so
+// that one fixed codebook serves every key; Eqs. 7-10: the 4-bit summary that
+// Stage II scores):
 //   k~ = R k/||k||; per block b of m = 8 coordinates:
 //   r_b = ||k~_b||, u_b = k~_b / r_b,
 //   code_b = sign pattern of u_b (bit j set iff u_j < 0)    -> PolarANN centre id

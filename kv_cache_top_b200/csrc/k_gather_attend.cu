@@ -1,15 +1,13 @@
 // k_gather_attend.cu -- gather of the selected K/V rows and exact attention.
 //
 // o_g = sum_r softmax_r(scale <q_g, K[sel_r]>) V[sel_r] for every query head
-// g of the KV head (ParisKV slides, "The target is high-score KV indices at
-// each decode step", Sec. 3 Eqs. 1-3: "recompute softmax and value
-// aggregation using the selected full-precision KV").  Optionally the rows
-// kept densely on the GPU outside the index -- the sink and recent local
-// tokens -- join the same softmax (README, step 3: attention "over sink
-// tokens, local tokens, and retrieved tokens"; slides, Fig. 5 layout).  The K/V rows are read
-// where the index keeps them: HBM, or pinned host memory through UVA (README,
-// "Attention: fetch only selected KV pairs ... from pinned CPU memory via
-// UVA").
+// g of the KV head (ParisKV slides, Sec. 3 Eqs. 1-3: softmax and the value sum
+// are computed again over the selected rows, in full precision).  Optionally
+// the rows kept densely on the GPU outside the index -- the sink and recent
+// local tokens -- join the same softmax (README, pipeline step 3; slides,
+// Fig. 5 layout).  The K/V rows are read where the index keeps them: HBM, or
+// pinned host memory through UVA (README, pipeline step 3: only the selected
+// rows cross from host memory, read through UVA).
 //
 // One thread-block cluster per pair (grid x = cluster x = splits <= 8): each
 // CTA takes a contiguous share of the selected rows, 32 rows per tile, and

@@ -2,9 +2,9 @@
 //
 // (1) GQA aggregation q_agg = ((q_0 + q_1) + ..) + q_{G-1} in fp32, then the
 //     canonical normalise + SRHT rotate (ParisKV slides, Eq. 5).
-// (2) Stage I bucket tiers (slides, "Stage I uses multi-tier collision votes
-//     to prune keys", Sec. 4.2.2 / App. B.2.1 Eq. 15; README "activates the
-//     nearest direction centroids in each subspace"): in block b every
+// (2) Stage I bucket tiers (slides, Sec. 4.2.2 / App. B.2.1 Eq. 15; README,
+//     pipeline step 2: per subspace, the centroids nearest the query's
+//     direction are the active ones): in block b every
 //     sign-pattern centre c gets the score L_b(c) = sum_j +-q~_{b,j} (minus
 //     where bit j of c is set; the 1/sqrt(m) factor does not change the order),
 //     the 256 centres are ranked by (L desc, c asc), P(c) = number of keys in

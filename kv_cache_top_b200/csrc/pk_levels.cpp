@@ -1,11 +1,11 @@
 // pk_levels.cpp -- Lloyd-Max magnitude levels of the ParisKV 4-bit summary.
 //
-// ParisKV slides, "The codebook is data-independent; the quantizer uses a
-// prior" (Prop. 4.1, App. B.1): under a Haar rotation (u_b)_j^2 follows
+// ParisKV slides, Prop. 4.1 and App. B.1 (the codebook does not depend on the
+// data; the quantiser is fitted to a prior): under a Haar rotation (u_b)_j^2 follows
 // Beta(1/2, (m-1)/2), so y = |u_j| has density proportional to
 // (1 - y^2)^((m-3)/2) on [0, 1], and offline Lloyd-Max quantisation gives the
-// shared 3-bit magnitude levels (README: "Lloyd-Max magnitude levels for
-// 4-bit reranking").
+// shared 3-bit magnitude levels (README, repository contents: a Lloyd-Max
+// level file used by the 4-bit rerank).
 //
 // The cell integrals have closed forms: with y = sin(theta),
 //   F0(Y) = int_0^Y (1-y^2)^((m-3)/2) dy = int_0^asin(Y) cos^(m-2)(theta) d theta

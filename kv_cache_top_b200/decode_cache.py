@@ -1,7 +1,7 @@
 """Sink / local / update-buffer layout for long decoding.
 
 ParisKV keeps recent tokens dense while older tokens are indexed and
-offloaded (README, "Long-generation support": a sink/local/update-buffer
+offloaded (README, section on long generation: a sink/local/update-buffer
 layout; slides, Fig. 5: sink and recent local tokens stay on the GPU for
 dense attention, new tokens enter an update buffer, and a full buffer
 triggers encoding and offload of the oldest local tokens; attention runs over

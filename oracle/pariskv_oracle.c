@@ -12,8 +12,8 @@
 #include <string.h>
 
 /* ===================================================================== */
-/* SRHT signs.  The pages say only that R is "a shared orthogonal transform */
-/* (implemented with SRHT)" (slides, Sec. 4.1.1, Eq. 5).  Reading: the      */
+/* SRHT signs.  The pages state only that one orthogonal transform, an     */
+/* SRHT, is shared by all keys (slides, Sec. 4.1.1, Eq. 5).  Reading: the   */
 /* square SRHT H_D diag(s) / sqrt(D) with a seeded +-1 diagonal.  The       */
 /* diagonal is drawn from splitmix64 (Vigna), counter-based per coordinate. */
 /* ===================================================================== */
@@ -38,7 +38,7 @@ void or_srht_signs(uint64_t seed, int D, int8_t *signs)
 /* vector, (u_b)_j^2 ~ Beta(1/2, (m-1)/2).  Then y = |(u_b)_j| has density  */
 /*   f(y) = 2 (1 - y^2)^((m-3)/2) / B(1/2, (m-1)/2),  0 <= y <= 1.           */
 /* The 3-bit magnitude levels are the Lloyd-Max quantiser of f (slides,     */
-/* same frame; readme, "regenerate the default 8-level magnitude codebook"). */
+/* same section; the readme ships a script that rebuilds the 8 levels).    */
 /* Reading: the exact-density fixed point, found by adaptive Simpson        */
 /* quadrature in fp64 and Lloyd's centroid / midpoint iteration.            */
 /* ===================================================================== */
@@ -181,7 +181,7 @@ static float tree_sum(float *v, int len)
 
 /* ===================================================================== */
 /* Key encoding.  Block split D = B m (slides, Sec. 4.1.2 and the notation */
-/* frame: "use D = Bm").  Per block (slides, Eqs. 6-10):                   */
+/* errata, which fix D as B times m).  Per block (slides, Eqs. 6-10):       */
 /*   r_b = ||k~_b||, u_b = k~_b / r_b                                       */
 /*   c_b = argmax_{w in {+-1/sqrt m}^m} <u_b, w>  = sign pattern of u_b     */
 /*         (bit j set iff u_j < 0; u_j = 0 counts as +, lowest id on ties)  */
@@ -248,8 +248,8 @@ void or_encode_keys(const float *K, int64_t n, int D, int m, const int8_t *signs
 }
 
 /* ===================================================================== */
-/* Stage I (slides, Sec. 4.2.2 and App. B.2.1 Eq. 15; readme, "activates   */
-/* the nearest direction centroids in each subspace and counts collisions"):*/
+/* Stage I (slides, Sec. 4.2.2 and App. B.2.1 Eq. 15; readme, pipeline     */
+/* step 2: per subspace the centroids nearest the query vote for keys):     */
 /*   per block, keep the top-rho fraction of keys ranked by the score of    */
 /*   their assigned centre; split it into six percentile tiers with bonuses */
 /*   6..1;  S_i = sum_b 1{i in T_b(rho)} w_{l(i,b)}.                        */
@@ -324,7 +324,7 @@ void or_collision(const uint16_t *codes, int64_t n, int D, int m, const uint8_t 
     }
 }
 
-/* Top-C of S (slides, Sec. 4.2.2: "choose the top-beta keys by S_i"; Sec. */
+/* Top-C of S (slides, Sec. 4.2.2: the keys with the largest S_i; Sec.    */
 /* 4.3: C = ceil(beta n)).  Tie rule: higher S, then lower index.           */
 typedef struct { int s; int32_t i; } sidx_t;
 
@@ -452,7 +452,8 @@ void or_attend(const float *q, int G, int D, const float *K, const float *V,
 }
 
 /* ===================================================================== */
-/* Adaptive ratio table (readme, "candidate and collision ratios" table):  */
+/* Adaptive ratio table (readme, the table of candidate / collision ratio  */
+/* by retrieval-zone length):                                               */
 /*   < 5K: 0.50/0.50;  5K-10K: 0.25/0.30;  10K-30K: 0.20/0.25;             */
 /*   >= 30K: 0.10/0.20.   Reading: K = 1000, half-open ranges.             */
 /* ===================================================================== */

@@ -217,7 +217,8 @@ def test_occupancy_counts(enc_random):
 
 def test_encoding_is_append_consistent():
     """Encoding keys one at a time equals encoding them together; new keys
-    need no retraining (slides, "The codebook is data-independent")."""
+    need no retraining (slides, Prop. 4.1: the codebook does not depend on
+    the data)."""
     rng = np.random.default_rng(3)
     K = rng.standard_normal((200, D)).astype(np.float32)
     full = oracle.encode_keys(K, _signs())
