@@ -1,10 +1,10 @@
 // k_collision_scan.cu -- multi-tier collision counting and the integer Top-C
 // threshold.
 //
-// S_i = sum_b bonus_b[code_{i,b}]  (ParisKV slides, Sec. 4.2.2 and App. B.2.1
-// Eq. 15), an integer in [0, 96].  Because S takes so few values, the Top-C
-// by S needs no sort: a histogram and a prefix scan fix the threshold (same
-// section).  Each CTA histograms the S of its chunk, and the
+// S_i = sum_b bonus_b[code_{i,b}]  (ParisKV slides, "Stage I uses multi-tier
+// collision votes to prune keys", App. B.2.1 Eq. 15), an integer in [0, 96].
+// "Small integer scores allow histogram and prefix-scan selection instead of a
+// full sort" (same frame): each CTA histograms the S of its chunk, and the
 // last CTA of a pair to finish (ticket counter, no spin-wait) finds the
 // threshold s* = max{s : #{S >= s} >= C}, and for every chunk the first slot of
 // its candidates and how many of its S = s* keys it keeps (lower ids first),
@@ -32,22 +32,31 @@ constexpr int kScanThreads = 256;
 constexpr int kScanUnroll = 4;
 constexpr int kHistPad = 104;
 
-__device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], uint4 c)
+// Code byte 3 of every 32-bit code word (blocks 3, 7, 11 and 15) is looked up
+// in a byte table in shared memory instead of the register tables: one shift
+// and an LDS.U8 (at most two distinct words per bank: a 256-byte table spans
+// 64 words), against a shuffle, two shifts, a rotate and half an add and a
+// mask on the register path.  The split moves work from the integer ALU
+// pipe, which bounds the all-register scan, to the load/store pipe; moving
+// two or three bytes per word instead measured slower (bank conflicts and
+// register spills at 4 CTAs per SM).
+__device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], const uint8_t *btab, uint4 c)
 {
     uint32_t s = 0;
     const uint32_t wds[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int q = 0; q < 4; q++) {
         const uint32_t w = wds[q];
+        // bytes 0..2: register tables by shuffles
         const uint32_t v0 = __shfl_sync(kFull, tab[4 * q + 0], (int)w);
         const uint32_t v1 = __shfl_sync(kFull, tab[4 * q + 1], (int)(w >> 8));
         const uint32_t v2 = __shfl_sync(kFull, tab[4 * q + 2], (int)(w >> 16));
-        const uint32_t v3 = __shfl_sync(kFull, tab[4 * q + 3], (int)(w >> 24));
         const uint32_t x0 = __funnelshift_r(v0, v0, w >> 3);
         const uint32_t x1 = __funnelshift_r(v1, v1, w >> 11);
         const uint32_t x2 = __funnelshift_r(v2, v2, w >> 19);
-        const uint32_t x3 = __funnelshift_r(v3, v3, w >> 27);
-        s += ((x0 + x1) & 0xfu) + ((x2 + x3) & 0xfu);
+        // byte 3: the block's byte table in shared memory
+        const uint32_t l3 = btab[256 * (4 * q + 3) + (w >> 24)];
+        s += ((x0 + x1) & 0xfu) + (x2 & 0xfu) + l3;
     }
     return s;
 }
@@ -61,6 +70,7 @@ __global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
     __shared__ uint32_t s_cum[kHistPad];
     __shared__ uint32_t s_ws[NW + 1];
     __shared__ int s_last;
+    __shared__ __align__(16) uint8_t s_btab[kB][kNC];   // bonus of (block, centre) for blocks 3, 7, 11, 15
 
     for (int i = tid; i < NW * kHistPad; i += kScanThreads) (&s_hist[0][0])[i] = 0u;
 
@@ -69,6 +79,18 @@ __global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
     const uint32_t *bp = a.bonus_packed + (size_t)bh * kB * 32;
 #pragma unroll
     for (int b = 0; b < kB; b++) tab[b] = bp[b * 32 + lane];
+    {   // byte tables of blocks 3, 7, 11, 15 (warps 3 and 7 build them): lane
+        // l's word of block b holds the bonus of centre 32 t + l in bits 4 t..
+        // after undoing its rotation by r(l)
+        const uint32_t rl = (uint32_t)(lane >> 3) & 3u;
+#pragma unroll
+        for (int b = 0; b < kB; b++) {
+            if ((b & 3) != 3 || (b & (NW - 1)) != warp) continue;
+            const uint32_t plain = __funnelshift_r(tab[b], tab[b], rl);
+#pragma unroll
+            for (int t = 0; t < 8; t++) s_btab[b][32 * t + lane] = (uint8_t)((plain >> (4 * t)) & 0xfu);
+        }
+    }
     __syncthreads();
 
     const int64_t lo = (int64_t)chunk * a.chunk;
@@ -107,7 +129,7 @@ __global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
         if (base + step < ucnt + lane) load(base + step, cn);
         uint32_t sc[kScanUnroll];
 #pragma unroll
-        for (int u = 0; u < kScanUnroll; u++) sc[u] = collision_score(tab, c[u]);
+        for (int u = 0; u < kScanUnroll; u++) sc[u] = collision_score(tab, &s_btab[0][0], c[u]);
         if (full) {
 #pragma unroll
             for (int u = 0; u < kScanUnroll; u++) {

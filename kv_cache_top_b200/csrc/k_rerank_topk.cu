@@ -1,10 +1,10 @@
 // k_rerank_topk.cu -- 4-bit RSQ-IP rerank of the candidates and the Top-k.
 //
-// Estimate (ParisKV slides, "Stage II estimates the raw attention score from
-// 4-bit codes", Eqs. 7-10):
+// Estimate (ParisKV slides, Sec. 4.2.3 Eqs. 7-10):
 //     <k_i, q>^ = ||q|| sum_b w_{i,b} sum_j sigma_{i,b,j} l_{t_{i,b,j}} q~_{b,j}
-// read from the key's 128-byte summary record; "key-only factors are
-// precomputed, so GPU ranking needs no full-precision keys".
+// read from the key's 128-byte summary record: every factor that depends on
+// the key alone is stored at encode time, so scoring a candidate touches no
+// full-precision key.
 //
 // Work is split by candidate slices (not key ranges), so every CTA reranks
 // the same number of records wherever the candidates sit; a CTA has 256 or
@@ -27,8 +27,8 @@
 // per-slice lists into the final Top-k with a tree of pairwise merges
 // (bitonic warp merges in registers for k <= 128, merge-path runs in shared
 // memory otherwise)
-// (README: "reranks those candidates with a fused 4-bit approximate
-// inner-product kernel and selects the final Top-k KV indices").
+// (README, pipeline step 2: one fused kernel scores the candidates with the
+// 4-bit inner-product estimate and picks the final Top-k ids).
 #include "pk_internal.cuh"
 #include "pk_launch.cuh"
 #include "pk_merge.cuh"
@@ -38,16 +38,26 @@ namespace pk {
 constexpr int kRrThreads = 256;                  // the merge CTA; a rerank CTA has NT = 256 or 128
 constexpr int kRrWarps = kRrThreads / 32;
 
+// Signed level x query coordinate, one 16-entry table per coordinate j:
+//     tab[tab_index(j, c)] = sigma(c) l_{c & 7} q~_j,   sigma(c) = -1 iff c & 8,
+// placed so that coordinates j and j + 64 (read at once by the two halves of a
+// warp) sit in opposite halves of the 32 banks: entry (j, c) is word
+// 32 (j & 63) + 16 (j >> 6) + c.
+__host__ __device__ constexpr int tab_index(int j, int c) { return 32 * (j & 63) + 16 * (j >> 6) + c; }
+
 struct RrShared {
-    u64 tmp[kMaxTopk];
+    union {
+        u64 tmp[kMaxTopk];        // the select's kept keys (after the decode)
+        float tab[kD * 16];       // the decode's lookup tables
+    };
     uint32_t hist[2][256];
     u64 red[2][kRrWarps];
     uint32_t sh[4];
     uint32_t cnt;
     uint32_t bcnt;
-    float slev[16];
     int last;
 };
+static_assert(sizeof(u64) * kMaxTopk == sizeof(float) * kD * 16, "tab and tmp share storage");
 
 // Warp-aggregated append: every lane with `want` gets a distinct slot of
 // *ctr (one shared-memory atomic per warp instead of one per lane).
@@ -361,36 +371,25 @@ __device__ __forceinline__ void rank_by_count(const u64 *v, int m, Emit emit)
     }
 }
 
-// dot of one block's 8 nibbles (one u32: byte i holds coordinates 2i, 2i+1)
-// with 8 coordinates of q~.  lo/hi hold 4 x the low/high nibble of every byte,
-// i.e. the byte offsets of the signed levels in the 16-entry table; one byte
-// permute per coordinate then yields the address.
-// (x0, x1) * (y0, y1) + (z0, z1) elementwise, one packed fp32 instruction
-__device__ __forceinline__ float2 fma2(float2 x, float2 y, float2 z)
+// <v_b, q~_b> of one block from its 8 nibbles (one u32: byte i holds
+// coordinates 2i and 2i + 1 in its low and high nibble).  lo / hi hold, per
+// byte, 64 h + 4 x the low / high nibble (h = this lane's half of the warp),
+// i.e. the byte offset of the entry inside the two-table slot of a coordinate
+// pair; one byte permute per coordinate yields the address, and the 8 table
+// entries are summed in a fixed order.  `tb` points at the slot of the
+// block's first coordinate (tab + 32 x 8 bb words for block bb of the half).
+__device__ __forceinline__ float block_dot(const float *tb, uint32_t nib, uint32_t hmask)
 {
-    unsigned long long r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;"
-        : "=l"(r)
-        : "l"(*reinterpret_cast<unsigned long long *>(&x)), "l"(*reinterpret_cast<unsigned long long *>(&y)),
-          "l"(*reinterpret_cast<unsigned long long *>(&z)));
-    return *reinterpret_cast<float2 *>(&r);
-}
-
-// The even and odd coordinates accumulate in the two lanes of one packed
-// fp32 pair (one packed fma per byte of nibbles), added at the end.
-__device__ __forceinline__ float block_dot(const float *slev, uint32_t nib, const float *q)
-{
-    const uint32_t lo = (nib << 2) & 0x3c3c3c3cu, hi = (nib >> 2) & 0x3c3c3c3cu;
-    const char *base = reinterpret_cast<const char *>(slev);
-    float2 d = make_float2(0.0f, 0.0f);
+    const uint32_t lo = ((nib << 2) & 0x3c3c3c3cu) | hmask, hi = ((nib >> 2) & 0x3c3c3c3cu) | hmask;
+    const char *base = reinterpret_cast<const char *>(tb);
+    float x[8];
 #pragma unroll
     for (int i = 0; i < 4; i++) {
         const uint32_t o0 = __byte_perm(lo, 0u, 0x4440u + i), o1 = __byte_perm(hi, 0u, 0x4440u + i);
-        const float2 l = make_float2(*reinterpret_cast<const float *>(base + o0),
-                                     *reinterpret_cast<const float *>(base + o1));
-        d = fma2(l, make_float2(q[2 * i], q[2 * i + 1]), d);
+        x[2 * i] = *reinterpret_cast<const float *>(base + 128 * (2 * i) + o0);
+        x[2 * i + 1] = *reinterpret_cast<const float *>(base + 128 * (2 * i + 1) + o1);
     }
-    return d.x + d.y;
+    return ((x[0] + x[1]) + (x[2] + x[3])) + ((x[4] + x[5]) + (x[6] + x[7]));
 }
 
 
@@ -453,10 +452,21 @@ __device__ const u64 *merge_tree(u64 *src, u64 *dst, int ns, int k)
     return src;
 }
 
-constexpr int kRrStages = 3;                       // per-warp pipeline depth
+// Per-warp ring of record stages.  The gather is latency-bound (random
+// 128-byte records), so the ring is as deep as shared memory allows at the
+// CTA's occupancy: 4 stages at 256 threads (2 CTAs per SM), 3 at 128 (4 per
+// SM); stages - 1 of them are in flight while one is decoded.
+__host__ __device__ constexpr int rr_stages(int nt) { return nt == 256 ? 4 : 3; }
 constexpr int kRrStep = 16;                        // records per warp stage
-constexpr int kRecPad = 144;                       // shared-memory record stride (conflict-free)
-__host__ __device__ constexpr size_t rr_ring_bytes(int nt) { return (size_t)(nt / 32) * kRrStages * kRrStep * kRecPad; }
+constexpr int kRecSlot = 128;                      // shared-memory record slot, no padding
+__host__ __device__ constexpr size_t rr_ring_bytes(int nt)
+{
+    return (size_t)(nt / 32) * rr_stages(nt) * kRrStep * kRecSlot;
+}
+// Byte offset of 16-byte chunk c of slot j in a stage: chunks are XOR-swizzled
+// by the slot index, so 8 lanes reading (or writing) chunk c of 8 consecutive
+// slots, or 8 chunks of one slot, hit 8 different 16-byte bank groups.
+__device__ __forceinline__ int slot_off(int j, int c) { return j * kRecSlot + 16 * (c ^ (j & 7)); }
 
 // NT = 256 (2 CTAs per SM) or 128 (4 CTAs per SM): the host takes the size
 // whose one-wave split of the candidates loads the SMs more evenly.
@@ -475,7 +485,6 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
     const int64_t m0 = (int64_t)sl * a.slice;
     const int count = (int)min((int64_t)a.slice, a.C - m0);
 
-    if (tid < 16) sm.slev[tid] = (tid & 8) ? -a.lv.lev[tid & 7] : a.lv.lev[tid & 7];
     pdl_wait();                                   // candidates come from the compaction
     const int32_t *cand = a.cand + (size_t)bh * a.stride + m0;
     {   // count <= kSelPer NT: every id load of the thread in flight at once
@@ -486,10 +495,21 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
         for (int u = 0; u < kSelPer; u++)
             if (tid + u * NT < count) keys[tid + u * NT] = (u64)(uint32_t)cv[u];
     }
-    const int q4 = lane & 3, sub = lane >> 2;          // 32-byte group of the record, record of the round
-    float qr[32];
+    {   // the lookup tables: entry e of tab holds (j, c) with c = e & 15,
+        // j = 64 ((e >> 4) & 1) + (e >> 5); one fp32 product each
+        const float *qt = a.qt + (size_t)bh * kD;
 #pragma unroll
-    for (int i = 0; i < 32; i++) qr[i] = a.qt[(size_t)bh * kD + 32 * q4 + i];
+        for (int u = 0; u < (kD * 16) / NT; u++) {
+            const int e = tid + u * NT, c = e & 15, j = 64 * ((e >> 4) & 1) + (e >> 5);
+            const float l = a.lv.lev[c & 7];
+            sm.tab[e] = __fmul_rn((c & 8) ? -l : l, qt[j]);
+        }
+    }
+    const int rr = lane & 15, half = lane >> 4;        // record of the step, half of it (8 blocks)
+    const uint32_t hmask = half ? 0x40404040u : 0u;    // this half's tables: +64 bytes in each slot
+    // this lane's four 16-byte chunks (nibbles, weights, nibbles, weights) of its record slot
+    const int off0 = slot_off(rr, 4 * half), off1 = slot_off(rr, 4 * half + 1);
+    const int off2 = slot_off(rr, 4 * half + 2), off3 = slot_off(rr, 4 * half + 3);
     const float qnorm = a.qnorm[bh];
     float vlo = INFINITY, vhi = -INFINITY;        // range of this lane's scores (the select's bins)
     const uint8_t *rec = a.rec + (size_t)index_pair(bh, a.kvg) * a.stride * kRecBytes;
@@ -501,7 +521,8 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
     // stages: the copies of the next stages are in flight while one stage is
     // decoded.  Copies are coalesced: lane l moves 16-byte pieces l, l+32,
     // l+64, l+96 of the step's 2 KB.
-    unsigned char *ring = ring_all + (size_t)warp * kRrStages * kRrStep * kRecPad;
+    constexpr int kRrStages = rr_stages(NT);
+    unsigned char *ring = ring_all + (size_t)warp * kRrStages * kRrStep * kRecSlot;
     const int nsteps = (count + kRrStep - 1) / kRrStep;
     auto issue = [&](int step_local, int stage) {
         const int r0 = (warp + step_local * NW) * kRrStep;
@@ -513,7 +534,7 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
                 const int r = r0 + j;
                 if (r < count) {                      // keys[r] still holds the id: r is decoded later
                     const int32_t id = (int32_t)(uint32_t)keys[r];
-                    cp_async16(ring + ((size_t)stage * kRrStep + j) * kRecPad + 16 * c,
+                    cp_async16(ring + (size_t)stage * kRrStep * kRecSlot + slot_off(j, c),
                                rec + (size_t)id * kRecBytes + 16 * c);
                 }
             }
@@ -528,20 +549,24 @@ __global__ void __launch_bounds__(NT, 512 / NT) k_rerank_topk(RerankArgs a)
         __syncwarp();                                 // ... and every lane's
         const int stage = t % kRrStages;
         const int r0 = (warp + t * NW) * kRrStep;
-        const unsigned char *st = ring + (size_t)stage * kRrStep * kRecPad;
-#pragma unroll
-        for (int u = 0; u < 2; u++) {
-            const int j = 8 * u + sub;
-            const uint4 *p = reinterpret_cast<const uint4 *>(st + (size_t)j * kRecPad + 32 * q4);
-            const uint4 nv = p[0], wv = p[1];
-            float part = __uint_as_float(wv.x) * block_dot(sm.slev, nv.x, qr);
-            part = fmaf(__uint_as_float(wv.y), block_dot(sm.slev, nv.y, qr + 8), part);
-            part = fmaf(__uint_as_float(wv.z), block_dot(sm.slev, nv.z, qr + 16), part);
-            part = fmaf(__uint_as_float(wv.w), block_dot(sm.slev, nv.w, qr + 24), part);
-            part += __shfl_xor_sync(kFull, part, 1);
-            part += __shfl_xor_sync(kFull, part, 2);
-            const int r = r0 + j;
-            if (q4 == 0 && r < count) {
+        const unsigned char *st = ring + (size_t)stage * kRrStep * kRecSlot;
+        {
+            // lanes rr and rr + 16 take the two halves (8 blocks each) of record rr
+            const uint4 n0 = *reinterpret_cast<const uint4 *>(st + off0);
+            const uint4 w0 = *reinterpret_cast<const uint4 *>(st + off1);
+            const uint4 n1 = *reinterpret_cast<const uint4 *>(st + off2);
+            const uint4 w1 = *reinterpret_cast<const uint4 *>(st + off3);
+            float part = __fmul_rn(__uint_as_float(w0.x), block_dot(sm.tab + 256 * 0, n0.x, hmask));
+            part = fmaf(__uint_as_float(w0.y), block_dot(sm.tab + 256 * 1, n0.y, hmask), part);
+            part = fmaf(__uint_as_float(w0.z), block_dot(sm.tab + 256 * 2, n0.z, hmask), part);
+            part = fmaf(__uint_as_float(w0.w), block_dot(sm.tab + 256 * 3, n0.w, hmask), part);
+            part = fmaf(__uint_as_float(w1.x), block_dot(sm.tab + 256 * 4, n1.x, hmask), part);
+            part = fmaf(__uint_as_float(w1.y), block_dot(sm.tab + 256 * 5, n1.y, hmask), part);
+            part = fmaf(__uint_as_float(w1.z), block_dot(sm.tab + 256 * 6, n1.z, hmask), part);
+            part = fmaf(__uint_as_float(w1.w), block_dot(sm.tab + 256 * 7, n1.w, hmask), part);
+            part += __shfl_xor_sync(kFull, part, 16);
+            const int r = r0 + rr;
+            if (half == 0 && r < count) {
                 const float est = qnorm * part;
                 const float v = __fadd_rn(est, 0.0f);     // the score the key orders by
                 vlo = fminf(vlo, v);
