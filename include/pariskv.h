@@ -109,6 +109,7 @@ typedef struct {
     int64_t kv_bytes;         /* full K/V store (device or pinned host)        */
     int32_t kv_location;
     int32_t num_sms;
+    int64_t n_staged;         /* keys staged by pk_append_stage, not yet published */
 } pk_info;
 
 /* Optional intermediate outputs of pk_search_debug (device pointers; any may
@@ -147,6 +148,35 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
  * PK_ERR_CAPACITY when n + n_new > n_cap (nothing is written). */
 pk_status pk_append(pk_index *index, const void *k_new, const void *v_new, int64_t n_new,
                     void *stream);
+
+/* Asynchronous re-indexing in two calls ([readme] section on long
+ * generation: older tokens are indexed and offloaded in the background;
+ * [slides] Fig. 5: a full update buffer is encoded and offloaded in one
+ * batch).
+ *
+ * pk_append_stage encodes n_new keys per pair into the rows after the keys
+ * already present or staged, copies their K/V rows into the store, and counts
+ * their occupancy in a side table.  Searches and attention do not see staged
+ * keys: they use n and the published occupancy only.  So the call may run on
+ * a stream of its own, concurrently with pk_search / pk_attend on the decode
+ * stream; the caller must not change the source rows until the staging work
+ * is done (it is, for any stream, once that stream has passed
+ * pk_append_publish).
+ *   k_new, v_new  row 0 of pair 0 of a [BH][src_stride][D] kv_dtype array
+ *                 (device or mapped host); rows 0..n_new-1 of each pair are
+ *                 taken, so a window of a larger per-pair buffer can be staged
+ *                 in place.  src_stride 0 means n_new.
+ * PK_ERR_CAPACITY when n + staged + n_new > n_cap (nothing is written).
+ * Two stage calls must not overlap on the GPU (use one staging stream).
+ *
+ * pk_append_publish makes every staged key visible to work enqueued on
+ * `stream` after it: the stream waits (on the GPU) for the staging work, the
+ * side counts are added into the occupancy table, and n grows by the staged
+ * count.  Nothing to publish is not an error.  pk_append returns
+ * PK_ERR_INVALID_ARG while keys are staged. */
+pk_status pk_append_stage(pk_index *index, const void *k_new, const void *v_new, int64_t n_new,
+                          int64_t src_stride, void *stream);
+pk_status pk_append_publish(pk_index *index, void *stream);
 
 /* Retrieve the Top-k keys of every pair for one decode step.
  *   q          [batch][H*G][D] kv_dtype; query head j belongs to KV head j/G.

@@ -38,8 +38,8 @@ __all__ = [
     "pk_attend", "pk_free", "pk_status_str", "pk_last_device_error", "pk_get_info",
     "pk_export_index", "pk_magnitude_levels", "pk_resolve", "pk_trace_enable", "pk_trace_read",
     "pk_select_candidates_noalloc", "pk_attend_dense", "pk_search_heads", "pk_attend_heads",
-    "pk_params", "pk_info", "pk_debug_out", "PK_F32", "PK_BF16", "PK_KV_DEVICE",
-    "PK_KV_HOST_PINNED", "KERNELS", "lib",
+    "pk_append_stage", "pk_append_publish", "pk_params", "pk_info", "pk_debug_out", "PK_F32",
+    "PK_BF16", "PK_KV_DEVICE", "PK_KV_HOST_PINNED", "KERNELS", "lib",
 ]
 
 
@@ -95,6 +95,18 @@ def pk_build_index(K, V, n: int, params: pk_params, stream=None) -> C.c_void_p:
 
 def pk_append(index, k_new, v_new, n_new: int, stream=None):
     _check(_L().pk_append(index, _ptr(k_new), _ptr(v_new), int(n_new), _stream(stream)), "pk_append")
+
+
+def pk_append_stage(index, k_new, v_new, n_new: int, src_stride: int = 0, stream=None):
+    """Encode n_new rows per pair of k_new/v_new ([BH][src_stride][D]) into the
+    index without making them visible to search (see pk_append_publish)."""
+    _check(_L().pk_append_stage(index, _ptr(k_new), _ptr(v_new), int(n_new), int(src_stride), _stream(stream)),
+           "pk_append_stage")
+
+
+def pk_append_publish(index, stream=None):
+    """Make the staged keys visible to work enqueued on `stream` after this call."""
+    _check(_L().pk_append_publish(index, _stream(stream)), "pk_append_publish")
 
 
 def pk_search(index, q, topk: int, out_idx, out_score=None, stream=None):

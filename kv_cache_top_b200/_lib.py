@@ -16,6 +16,7 @@ EXPORTS = (
     "pk_attend", "pk_free", "pk_status_str", "pk_last_device_error", "pk_get_info",
     "pk_export_index", "pk_magnitude_levels", "pk_resolve", "pk_trace_enable", "pk_trace_read",
     "pk_select_candidates_noalloc", "pk_attend_dense", "pk_search_heads", "pk_attend_heads",
+    "pk_append_stage", "pk_append_publish",
 )
 
 PK_OK, PK_ERR_INVALID_ARG, PK_ERR_CAPACITY, PK_ERR_OOM, PK_ERR_CUDA, PK_ERR_TIMEOUT, \
@@ -41,7 +42,7 @@ class pk_info(C.Structure):
         ("n", C.c_int64), ("n_cap", C.c_int64), ("bh", C.c_int32), ("nchunks", C.c_int32),
         ("chunk", C.c_int64), ("cand", C.c_int64), ("coll", C.c_int64),
         ("index_bytes", C.c_int64), ("kv_bytes", C.c_int64), ("kv_location", C.c_int32),
-        ("num_sms", C.c_int32),
+        ("num_sms", C.c_int32), ("n_staged", C.c_int64),
     ]
 
 
@@ -66,6 +67,10 @@ def load() -> C.CDLL:
     lib.pk_build_index.argtypes = [P, P, I64, C.POINTER(pk_params), P, C.POINTER(P)]
     lib.pk_append.restype = st
     lib.pk_append.argtypes = [P, P, P, I64, P]
+    lib.pk_append_stage.restype = st
+    lib.pk_append_stage.argtypes = [P, P, P, I64, I64, P]
+    lib.pk_append_publish.restype = st
+    lib.pk_append_publish.argtypes = [P, P]
     lib.pk_search.restype = st
     lib.pk_search.argtypes = [P, P, I32, P, P, P]
     lib.pk_search_debug.restype = st

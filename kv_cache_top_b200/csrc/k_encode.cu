@@ -12,7 +12,9 @@
 // codes, indices and weights are bit-exact across implementations.
 //
 // One warp per key: lane l holds coordinates l + 32 r (r = 0..3), so register
-// r holds blocks 4r..4r+3, one block per aligned 8-lane group.
+// r holds blocks 4r..4r+3, one block per aligned 8-lane group.  Large batches
+// (the prefill, a batched re-indexing) count their occupancy per CTA in
+// shared memory; a few keys count straight into the table.
 //
 // Record layout (128 B per key, 16-byte aligned):
 //   for g = 0..3:  [16 B: blocks 4g..4g+3, one u32 each, nibble j = coordinate
@@ -22,60 +24,107 @@
 
 namespace pk {
 
-__global__ void __launch_bounds__(256) k_encode(EncodeArgs a)
+constexpr int kEncWarps = 8;
+constexpr int kEncKeysShared = 1024;   // keys per CTA when the occupancy counts go through shared memory
+
+// Encode one key (a warp): writes its codes and record; each of the 16
+// (block, code) counts goes to count(b, code).
+template <typename Count>
+__device__ __forceinline__ void encode_key(const EncodeArgs &a, int64_t bh, int64_t i, int lane, Count count)
+{
+    const int64_t pos = a.pos0 + i;
+    float x[4];
+#pragma unroll
+    for (int r = 0; r < 4; r++) x[r] = ld_as_f32(a.K, (bh * a.k_stride + i) * kD + lane + 32 * r, a.is_bf16);
+    const float nk = warp_rotate128(x, a.rot, lane);
+
+    uint8_t *codes = a.codes + ((size_t)bh * a.n_cap + pos) * kB;
+    uint8_t *rec = a.rec + ((size_t)bh * a.n_cap + pos) * kRecBytes;
+    const int g = lane >> 3;       // block within the register group
+    const int j = lane & 7;        // coordinate within the block
+#pragma unroll
+    for (int r = 0; r < 4; r++) {
+        const float xv = x[r];
+        float sq = __fmul_rn(xv, xv);
+        sq = __fadd_rn(sq, __shfl_xor_sync(kFull, sq, 4));   // tree h = 4, 2, 1
+        sq = __fadd_rn(sq, __shfl_xor_sync(kFull, sq, 2));
+        sq = __fadd_rn(sq, __shfl_xor_sync(kFull, sq, 1));
+        const float rb = __fsqrt_rn(sq);
+        // rb is uniform over the 8-lane group; a zero block keeps u = 0,
+        // t = 0, w = 0.  No branch around the shuffles below.
+        const bool live = rb != 0.0f;
+        const float u = live ? __fdiv_rn(xv, rb) : 0.0f;
+        const bool neg = u < 0.0f;
+        const float au = fabsf(u);
+        int t = 0;
+#pragma unroll
+        for (int q = 0; q < kL - 1; q++) t += (au > a.lv.thr[q]) ? 1 : 0;
+        float p = __fmul_rn(a.lv.lev[t], au);
+        p = __fadd_rn(p, __shfl_xor_sync(kFull, p, 4));
+        p = __fadd_rn(p, __shfl_xor_sync(kFull, p, 2));
+        p = __fadd_rn(p, __shfl_xor_sync(kFull, p, 1));
+        const float w = live ? __fdiv_rn(__fmul_rn(nk, rb), p) : 0.0f;
+        const uint32_t bal = __ballot_sync(kFull, neg);
+        uint32_t word = (uint32_t)(((neg ? 8 : 0) | t) << (4 * j));
+        word |= __shfl_xor_sync(kFull, word, 4);
+        word |= __shfl_xor_sync(kFull, word, 2);
+        word |= __shfl_xor_sync(kFull, word, 1);
+        if (j == 0) {
+            const int b = 4 * r + g;
+            const uint32_t code = (bal >> (8 * g)) & 0xffu;
+            codes[b] = (uint8_t)code;
+            reinterpret_cast<uint32_t *>(rec + 32 * r)[g] = word;
+            reinterpret_cast<float *>(rec + 32 * r + 16)[g] = w;
+            count(b, code);
+        }
+    }
+}
+
+// Few keys: one warp per key over all pairs, counts straight to global memory.
+__global__ void __launch_bounds__(32 * kEncWarps) k_encode(EncodeArgs a)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t warps = (int64_t)gridDim.x * kEncWarps;
     const int64_t total = (int64_t)a.bh * a.n_new;
-    for (int64_t e = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); e < total;
-         e += warps) {
+    for (int64_t e = (int64_t)blockIdx.x * kEncWarps + (threadIdx.x >> 5); e < total; e += warps) {
         const int64_t bh = e / a.n_new;
-        const int64_t i = e - bh * a.n_new;
-        const int64_t pos = a.pos0 + i;
-        float x[4];
-#pragma unroll
-        for (int r = 0; r < 4; r++) x[r] = ld_as_f32(a.K, e * kD + lane + 32 * r, a.is_bf16);
-        const float nk = warp_rotate128(x, a.rot, lane);
+        encode_key(a, bh, e - bh * a.n_new, lane, [&](int b, uint32_t code) {
+            atomicAdd(&a.occ[((size_t)bh * kB + b) * kNC + code], 1u);
+        });
+    }
+}
 
-        uint8_t *codes = a.codes + ((size_t)bh * a.n_cap + pos) * kB;
-        uint8_t *rec = a.rec + ((size_t)bh * a.n_cap + pos) * kRecBytes;
-        const int g = lane >> 3;       // block within the register group
-        const int j = lane & 7;        // coordinate within the block
-#pragma unroll
-        for (int r = 0; r < 4; r++) {
-            const float xv = x[r];
-            float sq = __fmul_rn(xv, xv);
-            sq = __fadd_rn(sq, __shfl_xor_sync(kFull, sq, 4));   // tree h = 4, 2, 1
-            sq = __fadd_rn(sq, __shfl_xor_sync(kFull, sq, 2));
-            sq = __fadd_rn(sq, __shfl_xor_sync(kFull, sq, 1));
-            const float rb = __fsqrt_rn(sq);
-            // rb is uniform over the 8-lane group; a zero block keeps u = 0,
-            // t = 0, w = 0.  No branch around the shuffles below.
-            const bool live = rb != 0.0f;
-            const float u = live ? __fdiv_rn(xv, rb) : 0.0f;
-            const bool neg = u < 0.0f;
-            const float au = fabsf(u);
-            int t = 0;
-#pragma unroll
-            for (int q = 0; q < kL - 1; q++) t += (au > a.lv.thr[q]) ? 1 : 0;
-            float p = __fmul_rn(a.lv.lev[t], au);
-            p = __fadd_rn(p, __shfl_xor_sync(kFull, p, 4));
-            p = __fadd_rn(p, __shfl_xor_sync(kFull, p, 2));
-            p = __fadd_rn(p, __shfl_xor_sync(kFull, p, 1));
-            const float w = live ? __fdiv_rn(__fmul_rn(nk, rb), p) : 0.0f;
-            const uint32_t bal = __ballot_sync(kFull, neg);
-            uint32_t word = (uint32_t)(((neg ? 8 : 0) | t) << (4 * j));
-            word |= __shfl_xor_sync(kFull, word, 4);
-            word |= __shfl_xor_sync(kFull, word, 2);
-            word |= __shfl_xor_sync(kFull, word, 1);
-            if (j == 0) {
-                const int b = 4 * r + g;
-                const uint32_t code = (bal >> (8 * g)) & 0xffu;
-                codes[b] = (uint8_t)code;
-                reinterpret_cast<uint32_t *>(rec + 32 * r)[g] = word;
-                reinterpret_cast<float *>(rec + 32 * r + 16)[g] = w;
-                atomicAdd(&a.occ[((size_t)bh * kB + b) * kNC + code], 1u);
-            }
+// Many keys: CTA (x, pair) encodes keys x kEncKeysShared .. of one pair and
+// counts them in shared memory; the non-zero counts are added to the pair's
+// table once per CTA (at most 4096 global atomics instead of 16 per key).
+__global__ void __launch_bounds__(32 * kEncWarps) k_encode_shared(EncodeArgs a)
+{
+    __shared__ uint32_t s_occ[kB * kNC];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t bh = blockIdx.y;
+    for (int i = threadIdx.x; i < kB * kNC; i += 32 * kEncWarps) s_occ[i] = 0u;
+    __syncthreads();
+    const int64_t k0 = (int64_t)blockIdx.x * kEncKeysShared;
+    const int64_t k1 = min(a.n_new, k0 + kEncKeysShared);
+    for (int64_t i = k0 + warp; i < k1; i += kEncWarps)
+        encode_key(a, bh, i, lane, [&](int b, uint32_t code) { atomicAdd(&s_occ[b * kNC + code], 1u); });
+    __syncthreads();
+    uint32_t *occ = a.occ + (size_t)bh * kB * kNC;
+    for (int i = threadIdx.x; i < kB * kNC; i += 32 * kEncWarps) {
+        const uint32_t v = s_occ[i];
+        if (v) atomicAdd(&occ[i], v);
+    }
+}
+
+// Publishing staged keys: their counts join the table, and the side table is
+// left at zero for the next staging.
+__global__ void __launch_bounds__(256) k_occ_merge(uint32_t *occ, uint32_t *add, int64_t count)
+{
+    for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < count; i += (int64_t)gridDim.x * 256) {
+        const uint32_t v = add[i];
+        if (v) {
+            occ[i] += v;
+            add[i] = 0u;
         }
     }
 }
@@ -83,13 +132,28 @@ __global__ void __launch_bounds__(256) k_encode(EncodeArgs a)
 }  // namespace pk
 
 namespace pk {
+cudaError_t launch_occ_merge(uint32_t *occ, uint32_t *add, int64_t count, cudaStream_t s)
+{
+    const int64_t blocks = (count + 255) / 256;
+    k_occ_merge<<<(unsigned)(blocks < 1184 ? blocks : 1184), 256, 0, s>>>(occ, add, count);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s)
 {
     const int64_t keys = (int64_t)a.bh * a.n_new;
     if (keys <= 0) return cudaSuccess;
-    const int64_t blocks = (keys + 7) / 8;                 // 8 warps per CTA, one key each
-    const int grid = (int)(blocks < 65535 * 16 ? blocks : 65535 * 16);
-    k_encode<<<grid, 256, 0, s>>>(a);
+    // the shared-memory counts pay off from a few thousand keys per pair; a
+    // smaller batch (a decode-time re-indexing) takes one warp per key across
+    // all pairs, so its whole batch encodes in parallel
+    if (a.n_new >= 4 * kEncKeysShared && a.bh <= 65535) {
+        const int64_t gx = (a.n_new + kEncKeysShared - 1) / kEncKeysShared;
+        k_encode_shared<<<dim3((unsigned)gx, (unsigned)a.bh), 32 * kEncWarps, 0, s>>>(a);
+    } else {
+        const int64_t blocks = (keys + kEncWarps - 1) / kEncWarps;   // one key per warp
+        const int grid = (int)(blocks < 65535 * 16 ? blocks : 65535 * 16);
+        k_encode<<<grid, 32 * kEncWarps, 0, s>>>(a);
+    }
     return cudaGetLastError();
 }
 }  // namespace pk

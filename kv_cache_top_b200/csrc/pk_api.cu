@@ -49,6 +49,12 @@ struct pk_index {
     // K/V store (device, or mapped pinned host)
     void *K = nullptr, *V = nullptr;
     bool kv_host = false;
+    // staged appends: n_staged keys encoded at rows n .. n + n_staged - 1,
+    // their occupancy counts in occ_stage [BH][16][256] (zero when nothing is
+    // staged), not yet visible to search; stage_ev marks the staging work
+    int64_t n_staged = 0;
+    uint32_t *occ_stage = nullptr;
+    cudaEvent_t stage_ev = nullptr;
     // search workspaces (device): w for the aggregated query, wh for
     // per-query-head search (made on first use)
     Work w, wh;
@@ -254,6 +260,8 @@ void free_all(pk_index *ix)
 
     cudaFree(ix->dev_err);
     cudaFree(ix->dev_err_detail);
+    cudaFree(ix->occ_stage);
+    if (ix->stage_ev) cudaEventDestroy(ix->stage_ev);
     for (cudaEvent_t e : ix->ev_pool) cudaEventDestroy(e);
 }
 
@@ -303,10 +311,14 @@ pk_status check_params(const pk_params *p)
     return PK_OK;
 }
 
-pk_status encode_range(pk_index *ix, const void *Kin, int64_t n_new, int64_t pos0, cudaStream_t s)
+// Encode rows 0..n_new-1 of every pair of Kin ([BH][k_stride][D]) at
+// positions pos0.. and add their occupancy counts to occ.
+pk_status encode_range(pk_index *ix, const void *Kin, int64_t k_stride, int64_t n_new, int64_t pos0,
+                       uint32_t *occ, cudaStream_t s)
 {
     EncodeArgs a{};
     a.K = Kin;
+    a.k_stride = k_stride;
     a.n_new = n_new;
     a.pos0 = pos0;
     a.n_cap = ix->stride;
@@ -314,7 +326,7 @@ pk_status encode_range(pk_index *ix, const void *Kin, int64_t n_new, int64_t pos
     a.is_bf16 = ix->p.kv_dtype == PK_BF16;
     a.codes = ix->codes;
     a.rec = ix->rec;
-    a.occ = ix->occ;
+    a.occ = occ;
     a.rot = ix->rot;
     a.lv = ix->lv;
     trace_begin(ix, PK_K_ENCODE, s);
@@ -323,13 +335,14 @@ pk_status encode_range(pk_index *ix, const void *Kin, int64_t n_new, int64_t pos
     return cuda_status(e);
 }
 
-// copy [BH][n_new][D] rows into the store at positions pos0.. of each pair
-pk_status copy_rows(pk_index *ix, void *store, const void *src, int64_t n_new, int64_t pos0,
-                    cudaStream_t s)
+// copy rows 0..n_new-1 of every pair of src ([BH][src_stride][D]) into the
+// store at positions pos0.. of each pair
+pk_status copy_rows(pk_index *ix, void *store, const void *src, int64_t src_stride, int64_t n_new,
+                    int64_t pos0, cudaStream_t s)
 {
     const size_t row = (size_t)kD * ix->es;
     cudaError_t e = cudaMemcpy2DAsync((char *)store + (size_t)pos0 * row, (size_t)ix->stride * row,
-                                      src, (size_t)n_new * row, (size_t)n_new * row, (size_t)ix->bh,
+                                      src, (size_t)src_stride * row, (size_t)n_new * row, (size_t)ix->bh,
                                       cudaMemcpyDefault, s);
     return cuda_status(e);
 }
@@ -641,9 +654,9 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(cudaMemsetAsync(ix->occ, 0, BH * kB * kNC * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->dev_err, 0, sizeof(int32_t), s));
     chk(cudaMemsetAsync(ix->dev_err_detail, 0, sizeof(long long), s));
-    if (e == cudaSuccess) st = copy_rows(ix, ix->K, K, n, 0, s);
-    if (e == cudaSuccess && st == PK_OK) st = copy_rows(ix, ix->V, V, n, 0, s);
-    if (e == cudaSuccess && st == PK_OK) st = encode_range(ix, K, n, 0, s);
+    if (e == cudaSuccess) st = copy_rows(ix, ix->K, K, n, n, 0, s);
+    if (e == cudaSuccess && st == PK_OK) st = copy_rows(ix, ix->V, V, n, n, 0, s);
+    if (e == cudaSuccess && st == PK_OK) st = encode_range(ix, K, n, n, 0, ix->occ, s);
     if (e != cudaSuccess || st != PK_OK) {
         cudaStreamSynchronize(s);
         free_all(ix);
@@ -658,15 +671,60 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
 pk_status pk_append(pk_index *ix, const void *k_new, const void *v_new, int64_t n_new, void *stream)
 {
     if (!ix || !k_new || !v_new || n_new < 1) return PK_ERR_INVALID_ARG;
+    if (ix->n_staged) return PK_ERR_INVALID_ARG;       // publish staged keys first
     if (ix->n + n_new > ix->p.n_cap) return PK_ERR_CAPACITY;
     if (!device_accessible(k_new) || !device_accessible(v_new)) return PK_ERR_INVALID_ARG;
     if (!aligned(k_new, ix->es) || !aligned(v_new, ix->es)) return PK_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
-    pk_status st = copy_rows(ix, ix->K, k_new, n_new, ix->n, s);
-    if (st == PK_OK) st = copy_rows(ix, ix->V, v_new, n_new, ix->n, s);
-    if (st == PK_OK) st = encode_range(ix, k_new, n_new, ix->n, s);
+    pk_status st = copy_rows(ix, ix->K, k_new, n_new, n_new, ix->n, s);
+    if (st == PK_OK) st = copy_rows(ix, ix->V, v_new, n_new, n_new, ix->n, s);
+    if (st == PK_OK) st = encode_range(ix, k_new, n_new, n_new, ix->n, ix->occ, s);
     if (st == PK_OK) ix->n += n_new;
     return st;
+}
+
+pk_status pk_append_stage(pk_index *ix, const void *k_new, const void *v_new, int64_t n_new, int64_t src_stride,
+                          void *stream)
+{
+    if (!ix || !k_new || !v_new || n_new < 1) return PK_ERR_INVALID_ARG;
+    if (src_stride == 0) src_stride = n_new;
+    if (src_stride < n_new) return PK_ERR_INVALID_ARG;
+    if (ix->n + ix->n_staged + n_new > ix->p.n_cap) return PK_ERR_CAPACITY;
+    if (!device_accessible(k_new) || !device_accessible(v_new)) return PK_ERR_INVALID_ARG;
+    if (!aligned(k_new, ix->es) || !aligned(v_new, ix->es)) return PK_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t occ_words = (size_t)ix->bh * kB * kNC;
+    if (!ix->occ_stage) {
+        cudaError_t e = dalloc(&ix->occ_stage, occ_words);
+        if (e == cudaSuccess) e = cudaMemsetAsync(ix->occ_stage, 0, occ_words * sizeof(uint32_t), s);
+        if (e == cudaSuccess && !ix->stage_ev) e = cudaEventCreateWithFlags(&ix->stage_ev, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            cudaFree(ix->occ_stage);
+            ix->occ_stage = nullptr;
+            return cuda_status(e);
+        }
+    }
+    const int64_t pos0 = ix->n + ix->n_staged;
+    pk_status st = copy_rows(ix, ix->K, k_new, src_stride, n_new, pos0, s);
+    if (st == PK_OK) st = copy_rows(ix, ix->V, v_new, src_stride, n_new, pos0, s);
+    if (st == PK_OK) st = encode_range(ix, k_new, src_stride, n_new, pos0, ix->occ_stage, s);
+    if (st == PK_OK) st = cuda_status(cudaEventRecord(ix->stage_ev, s));
+    if (st == PK_OK) ix->n_staged += n_new;
+    return st;
+}
+
+pk_status pk_append_publish(pk_index *ix, void *stream)
+{
+    if (!ix) return PK_ERR_INVALID_ARG;
+    if (!ix->n_staged) return PK_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaStreamWaitEvent(s, ix->stage_ev, 0);
+    if (e == cudaSuccess) e = launch_occ_merge(ix->occ, ix->occ_stage, (int64_t)ix->bh * kB * kNC, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    ix->n += ix->n_staged;
+    ix->n_staged = 0;
+    return PK_OK;
 }
 
 pk_status pk_search(pk_index *ix, const void *q, int32_t topk, int32_t *out_idx, float *out_score,
@@ -746,6 +804,7 @@ pk_status pk_get_info(const pk_index *ix, pk_info *info)
     if (!ix || !info) return PK_ERR_INVALID_ARG;
     std::memset(info, 0, sizeof(*info));
     info->n = ix->n;
+    info->n_staged = ix->n_staged;
     info->n_cap = ix->p.n_cap;
     info->bh = ix->bh;
     chunking(ix, ix->w, ix->n, &info->nchunks, &info->chunk);

@@ -41,7 +41,8 @@ struct Levels {
 };
 
 struct EncodeArgs {
-    const void *K;           // [BH][n_new][D] kv dtype
+    const void *K;           // [BH][k_stride][D] kv dtype: rows 0..n_new-1 of each pair
+    int64_t k_stride;        // rows between pairs of the input (>= n_new)
     int64_t n_new;
     int64_t pos0;            // first position written
     int64_t n_cap;
@@ -49,7 +50,7 @@ struct EncodeArgs {
     int32_t is_bf16;
     uint8_t *codes;          // [BH][n_cap][16]
     uint8_t *rec;            // [BH][n_cap][128]
-    uint32_t *occ;           // [BH][16][256]
+    uint32_t *occ;           // [BH][16][256]  counts are added here
     RotConst rot;
     Levels lv;
 };
@@ -283,6 +284,8 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *ws, ui
 namespace pk {
 // kernel launchers (one per kernel translation unit)
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
+// occ[i] += add[i], add[i] = 0 for i < count
+cudaError_t launch_occ_merge(uint32_t *occ, uint32_t *add, int64_t count, cudaStream_t s);
 cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s);
 cudaError_t launch_collision_scan(const ScanArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_compact(const CompactArgs &a, int nchunks, int bh, cudaStream_t s);

@@ -23,13 +23,26 @@ would make it longer, its oldest `update` tokens are encoded into the index
 with one pk_append, and the zone grows by `update`.  Where the pages leave
 the boundary rule open, this is the reading: re-indexing moves exactly
 `update` tokens at a time and never lets the tail drop below `local`.
+
+With async_reindex=True the batch is indexed off the decode stream (the
+pages index and offload older tokens in the background): when the tail is
+full, the oldest `update` tail tokens are staged with pk_append_stage on a
+side stream, in `stage_pieces` pieces over as many consecutive steps, read
+in place from the dense buffer, while the decode stream keeps attending them
+densely.  The side stream also copies the tail rows that stay into a second
+dense buffer, and new tokens go to both buffers meanwhile.  `publish_lag`
+steps after the last piece, pk_append_publish makes the batch part of the
+index on the decode stream (which waits for the side stream on the GPU, not
+on the host) and the buffers swap.  The tail then holds up to
+`local + update + stage_pieces - 1 + publish_lag` tokens.
 """
 from __future__ import annotations
 
 import torch
 
-from . import (PK_BF16, PK_F32, PK_KV_DEVICE, PK_KV_HOST_PINNED, pk_append, pk_attend_dense,
-               pk_build_index, pk_default_params, pk_free, pk_get_info, pk_search)
+from . import (PK_BF16, PK_F32, PK_KV_DEVICE, PK_KV_HOST_PINNED, pk_append, pk_append_publish,
+               pk_append_stage, pk_attend_dense, pk_build_index, pk_default_params, pk_free, pk_get_info,
+               pk_search)
 
 
 class DecodeCache:
@@ -40,7 +53,8 @@ class DecodeCache:
     must hold at least `topk` tokens."""
 
     def __init__(self, K, V, *, group: int, sink: int = 64, local: int = 512, update: int = 512,
-                 max_len: int, topk: int = 100, offload: bool = False, **params):
+                 max_len: int, topk: int = 100, offload: bool = False, async_reindex: bool = False,
+                 publish_lag: int = 1, stage_pieces: int = 4, **params):
         assert K.dim() == 4 and K.shape == V.shape and K.shape[-1] == 128
         self.batch, self.H, T0, D = K.shape
         self.G, self.sink, self.local, self.update, self.topk = group, sink, local, update, topk
@@ -53,13 +67,24 @@ class DecodeCache:
                               kv_dtype=PK_BF16 if K.dtype == torch.bfloat16 else PK_F32,
                               kv_location=PK_KV_HOST_PINNED if offload else PK_KV_DEVICE, **params)
         self.index = pk_build_index(K[:, :, sink:z].contiguous(), V[:, :, sink:z].contiguous(), z - sink, p)
-        cap = sink + local + update
+        self.async_reindex = async_reindex
+        self.publish_lag = max(1, int(publish_lag))
+        self.pieces = max(1, min(int(stage_pieces), update))
+        cap = sink + local + update + ((self.pieces - 1 + self.publish_lag) if async_reindex else 0)
+        self.cap = cap
         self.dK = torch.zeros(self.batch, self.H, cap, D, dtype=K.dtype, device=K.device)
         self.dV = torch.zeros_like(self.dK)
         self.dK[:, :, :sink] = K[:, :, :sink]
         self.dV[:, :, :sink] = V[:, :, :sink]
         self.dK[:, :, sink:sink + local] = K[:, :, z:]
         self.dV[:, :, sink:sink + local] = V[:, :, z:]
+        if async_reindex:
+            # the second dense buffer (the sink rows never change) and the staging stream
+            self.dK2 = self.dK.clone()
+            self.dV2 = self.dV.clone()
+            self.side = torch.cuda.Stream(device=K.device)
+            self.staged_for = -1                          # steps since staging began, -1: none
+            self.staged = 0                               # tokens of the batch staged so far
         self.tail = local                                 # dense tail length
         self.T = T0
         self.zone_end = z
@@ -82,18 +107,57 @@ class DecodeCache:
         self.zone_end += u
         self.reindexed += 1
 
+    def _stage_piece(self):
+        """Stage the next piece of the oldest `update` tail tokens on the side
+        stream, in place; with the first piece, copy the tail rows that stay
+        into the second buffer."""
+        s, u = self.sink, self.update
+        self.side.wait_stream(torch.cuda.current_stream())   # rows written on the decode stream
+        with torch.cuda.stream(self.side):
+            if self.staged == 0:
+                rest = self.tail - u
+                self.dK2[:, :, s:s + rest].copy_(self.dK[:, :, s + u:s + self.tail])
+                self.dV2[:, :, s:s + rest].copy_(self.dV[:, :, s + u:s + self.tail])
+        c = (u * (self.staged_for + 1)) // self.pieces - self.staged
+        r0 = s + self.staged
+        pk_append_stage(self.index, self.dK[:, :, r0:], self.dV[:, :, r0:], c, self.cap, stream=self.side)
+        self.staged += c
+
+    def _publish(self):
+        """Make the staged tokens part of the index and drop them from the tail."""
+        pk_append_publish(self.index)                     # the decode stream waits for the staging
+        self.dK, self.dK2 = self.dK2, self.dK
+        self.dV, self.dV2 = self.dV2, self.dV
+        self.tail -= self.update
+        self.zone_end += self.update
+        self.reindexed += 1
+        self.staged_for = -1
+        self.staged = 0
+
     def step(self, q, k_new, v_new):
         """One decode step: add the new token k_new, v_new [batch][H][1][D] to
         the dense tail (re-indexing first when the buffer is full), retrieve
         the zone's Top-k for q [batch][H*G][D], and attend over sink + tail +
         retrieved rows.  Returns the attention output [batch][H*G][D] fp32
         (a buffer reused by the next step).  Everything runs on torch's current
-        stream, in order."""
-        if self.tail == self.local + self.update:
+        stream, in order, except the asynchronous staging."""
+        if self.async_reindex:
+            if self.staged_for < 0 and self.tail >= self.local + self.update:
+                self.staged_for = 0                       # a batch begins
+            elif self.staged_for >= 0:
+                self.staged_for += 1
+            if self.staged_for >= 0 and self.staged_for >= self.pieces - 1 + self.publish_lag:
+                self._publish()
+            elif self.staged_for >= 0 and self.staged_for < self.pieces:
+                self._stage_piece()
+        elif self.tail == self.local + self.update:
             self._reindex()
         r = self.sink + self.tail
         self.dK[:, :, r:r + 1] = k_new
         self.dV[:, :, r:r + 1] = v_new
+        if self.async_reindex and self.staged_for >= 0:   # also into the buffer that takes over
+            self.dK2[:, :, r - self.update:r - self.update + 1] = k_new
+            self.dV2[:, :, r - self.update:r - self.update + 1] = v_new
         self.tail += 1
         self.T += 1
         pk_search(self.index, q, self.topk, self.idx)
@@ -102,6 +166,8 @@ class DecodeCache:
 
     def close(self):
         if self.index is not None:
+            if self.async_reindex:
+                self.side.synchronize()               # no staging work in flight
             pk_free(self.index)
             self.index = None
 

@@ -317,32 +317,34 @@ def test_attend_with_dense_rows(pk, kind, topk, dlen, kv_location):
         pk.pk_free(h)
 
 
-@pytest.mark.parametrize("offload", [False, True])
-def test_decode_cache_sink_local_update(pk, offload):
+@pytest.mark.parametrize("offload,async_reindex", [(False, False), (True, False), (False, True), (True, True)])
+def test_decode_cache_sink_local_update(pk, offload, async_reindex):
     """The sink/local/update-buffer layout over 160 decode steps (sink 16,
     local 64, update 32; re-indexing every 32 steps): the retrieval zone
     grows by whole update buffers, the dense tail stays within
-    (local, local + update], the Top-k over the zone matches the oracle's
-    search of the zone, and the output is the oracle's attention over sink +
-    tail + retrieved rows."""
+    (local, local + update] (up to 4 steps more while a batch is staged
+    asynchronously, in 4 pieces),
+    the Top-k over the zone matches the oracle's search of the zone, and the
+    output is the oracle's attention over sink + tail + retrieved rows."""
     from kv_cache_top_b200.decode_cache import DecodeCache
     T0, steps, H, G = 4096, 160, 2, 2
     sink, local, update = 16, 64, 32
     w = workloads.llama_layer(1, T0 + steps, H=H, G=G, seed=77, device="cuda", n_queries=steps)
     K, V = w["K"], w["V"]
     cache = DecodeCache(K[:, :, :T0].contiguous(), V[:, :, :T0].contiguous(), group=G, sink=sink, local=local,
-                        update=update, max_len=T0 + steps, offload=offload)
+                        update=update, max_len=T0 + steps, offload=offload, async_reindex=async_reindex)
+    lag = 4 if async_reindex else 0          # 4 staging pieces, published one step after the last
     try:
         for t in range(steps):
             out = cache.step(w["q"][t], K[:, :, T0 + t:T0 + t + 1].contiguous(),
                              V[:, :, T0 + t:T0 + t + 1].contiguous())
-            if t not in (0, 31, 32, 100, steps - 1):
+            if t not in (0, 31, 32, 33, 100, 129, steps - 1):
                 continue
             torch.cuda.synchronize()
             T = T0 + t + 1
             z0, z1 = cache.zone
             assert z0 == sink and (z1 - (T0 - local)) % update == 0
-            assert cache.info().n == z1 - z0 and cache.tail == T - z1 and local < cache.tail <= local + update
+            assert cache.info().n == z1 - z0 and cache.tail == T - z1 and local < cache.tail <= local + update + lag
             idx2 = torch.empty_like(cache.idx)
             sc2 = torch.empty(H, 100, dtype=torch.float32, device="cuda")
             pk.pk_search(cache.index, w["q"][t], 100, idx2, sc2)
@@ -427,6 +429,43 @@ def test_attend_out_of_range_ids_are_skipped_and_recorded(pk):
                                    1.0 / math.sqrt(128))
         assert np.abs(out[0].cpu().numpy() - ref).max() <= parity.ATTN_ABS
         assert pk.pk_last_device_error(h)[0] == 0
+    finally:
+        pk.pk_free(h)
+
+
+def test_append_stage_publish(pk):
+    """Staged keys stay invisible to search until published; after publishing,
+    the index equals one built over all keys at once (strided source rows,
+    two staging calls, the staging on a side stream)."""
+    w = workloads.llama_layer(2, 9000, H=2, G=2, seed=19, device="cuda")
+    K, V = w["K"], w["V"]
+    n0 = 8000
+    h = build(pk, K[:, :, :n0].contiguous(), V[:, :, :n0].contiguous(), n0, 2, 2, 2, n_cap=9000)
+    try:
+        BH = 4
+        idx0 = torch.empty(BH, 100, dtype=torch.int32, device="cuda")
+        pk.pk_search(h, w["q"][0], 100, idx0)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        # rows n0 .. n0+599 and n0+600 .. 8999 taken in place from the [batch][H][9000][D] arrays
+        pk.pk_append_stage(h, K[:, :, n0:], V[:, :, n0:], 600, 9000, stream=side)
+        pk.pk_append_stage(h, K[:, :, n0 + 600:], V[:, :, n0 + 600:], 400, 9000, stream=side)
+        info = pk.pk_get_info(h)
+        assert info.n == n0 and info.n_staged == 1000
+        with pytest.raises(pk.PkError) as e:        # pk_append while keys are staged
+            pk.pk_append(h, K[:, :, :1].contiguous(), V[:, :, :1].contiguous(), 1)
+        assert e.value.status == 1
+        idx1 = torch.empty_like(idx0)
+        pk.pk_search(h, w["q"][0], 100, idx1)       # the decode stream: staged keys not visible
+        torch.cuda.synchronize()
+        assert torch.equal(idx0, idx1)
+        pk.pk_append_publish(h)
+        pk.pk_append_publish(h)                     # nothing left to publish
+        assert pk.pk_get_info(h).n == 9000 and pk.pk_get_info(h).n_staged == 0
+        check_pairs(pk, h, K, V, w["q"][0], list(range(BH)), 2, 2, 2, 9000, 100)
+        with pytest.raises(pk.PkError) as e:        # past n_cap
+            pk.pk_append_stage(h, K[:, :, :1], V[:, :, :1], 1, 9000)
+        assert e.value.status == 2
     finally:
         pk.pk_free(h)
 
