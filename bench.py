@@ -743,17 +743,32 @@ def run_heads(args, wl):
         torch.cuda.synchronize()
         return sum(a_.elapsed_time(b_) for a_, b_ in ev) / k
 
-    ms_a = timed(lambda i: (pk.pk_search(h, w["q"][i % nq], 100, idx_a),
-                            pk.pk_attend(h, w["q"][i % nq], idx_a, 100, out)))
-    ms_h = timed(lambda i: (pk.pk_search_heads(h, w["q"][i % nq], 100, idx_h),
-                            pk.pk_attend_heads(h, w["q"][i % nq], idx_h, 100, out)))
+    step_a = lambda i: (pk.pk_search(h, w["q"][i % nq], 100, idx_a),
+                        pk.pk_attend(h, w["q"][i % nq], idx_a, 100, out))
+    step_h = lambda i: (pk.pk_search_heads(h, w["q"][i % nq], 100, idx_h),
+                        pk.pk_attend_heads(h, w["q"][i % nq], idx_h, 100, out))
+    ms_a = timed(step_a)
+    ms_h = timed(step_h)
+
+    def kernels(step, k=50):          # per-kernel event times (traced pass)
+        pk.pk_trace_enable(h, True)
+        pk.pk_trace_read(h)
+        for i in range(k):
+            flush.zero_()
+            step(i)
+        kern = pk.pk_trace_read(h)
+        pk.pk_trace_enable(h, False)
+        return {name: round(ms / nl * 1000.0, 2) for name, (nl, ms) in kern.items() if nl}
+
+    kern_a, kern_h = kernels(step_a), kernels(step_h)
     pk.pk_free(h)
     print(json.dumps({
         "metric": "Recall@100 against each query head's exact Top-100, and step time: aggregated vs "
                   "per-query-head retrieval",
         "aggregated": {"recall_at_100": sum(rec_a) / len(rec_a), "ms_per_step": ms_a,
-                       "steps_s": 1000.0 / ms_a},
-        "per_head": {"recall_at_100": sum(rec_h) / len(rec_h), "ms_per_step": ms_h, "steps_s": 1000.0 / ms_h},
+                       "steps_s": 1000.0 / ms_a, "kernel_us": kern_a},
+        "per_head": {"recall_at_100": sum(rec_h) / len(rec_h), "ms_per_step": ms_h, "steps_s": 1000.0 / ms_h,
+                     "kernel_us": kern_h},
         "data": "synthetic", "dtype": "f32",
         "config": {"workload": wl["name"], "batch": B, "n": n, "kv_heads": H, "q_heads": H * G, "topk": 100,
                    "queries": nq, "l2": "flushed between steps (outside the events)"}}), flush=True)

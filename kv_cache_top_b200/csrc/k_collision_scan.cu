@@ -25,6 +25,7 @@
 // of the code word per code.  Two extracted bonuses (each <= 6) are added
 // before one mask, since their sum still fits in the low nibble.
 #include "pk_internal.cuh"
+#include "pk_launch.cuh"
 
 namespace pk {
 
@@ -59,6 +60,79 @@ __device__ __forceinline__ uint32_t collision_score(const uint32_t (&tab)[kB], c
         s += ((x0 + x1) & 0xfu) + (x2 & 0xfu) + l3;
     }
     return s;
+}
+
+// Chunk `chunk` of unit `unit`: thread tid < kBins holds hv = #{S = tid} in
+// the chunk.  Writes the chunk's suffix counts #{S >= s}, s = 0..97, and adds
+// the counts into the unit's histogram.  All kScanThreads threads call it.
+__device__ __forceinline__ void chunk_suffix(const ScanArgs &a, int unit, int chunk, uint32_t hv, uint32_t *s_cum,
+                                             uint32_t *s_ws)
+{
+    const int tid = threadIdx.x;
+    if (tid < kHistPad) s_cum[tid] = (tid < kBins) ? hv : 0u;
+    __syncthreads();
+    // suffix sum by a reversed exclusive scan over the threads
+    const int s = kScanThreads - 1 - tid;   // thread tid handles bin s (descending)
+    const uint32_t v = (s < kBins) ? s_cum[s] : 0u;
+    uint32_t tot;
+    const uint32_t ex = block_excl_scan<kScanThreads>(v, s_ws, &tot);
+    if (s < kCum) a.chunk_cum[((size_t)unit * a.max_chunks + chunk) * kCum + s] = ex + v;
+    if (tid < kBins && hv) atomicAdd(&a.head_hist[(size_t)unit * kBins + tid], hv);
+}
+
+// The last CTA of a unit to finish its chunk: the threshold s* = largest s
+// with #{S >= s} >= C, and for every chunk the first slot of its candidates
+// and how many of its S = s* keys it keeps (lower ids first).  All threads
+// call it; s_int and s_u32 are one shared word each.
+__device__ __forceinline__ void unit_threshold(const ScanArgs &a, int unit, uint32_t *s_ws, int *s_int, uint32_t *s_u32)
+{
+    const int tid = threadIdx.x;
+    uint32_t H = 0;
+    if (tid < kBins) H = __ldcg(&a.head_hist[(size_t)unit * kBins + tid]);
+    if (a.dbg_hist && tid < kBins) a.dbg_hist[(size_t)unit * kBins + tid] = H;
+    int64_t cumH;
+    {
+        const int s = kScanThreads - 1 - tid;
+        const uint32_t v = (s < kBins) ? __ldcg(&a.head_hist[(size_t)unit * kBins + s]) : 0u;
+        uint32_t tot;
+        const uint32_t ex = block_excl_scan<kScanThreads>(v, s_ws, &tot);
+        cumH = (int64_t)(ex + v);           // #{S >= s} for s = 255 - tid
+        // s* = largest s with #{S >= s} >= C  (cum is non-increasing in s)
+        const int pred = (s < kCum) && (cumH >= a.C);
+        const int nsat = __syncthreads_count(pred);
+        if (tid == 0) *s_int = nsat - 1;
+    }
+    __syncthreads();
+    const int sstar = *s_int;
+    if (tid == 0) {
+        a.sstar[unit] = sstar;
+        if (a.dbg_sstar) a.dbg_sstar[unit] = sstar;
+    }
+    // gt_total = #{S > s*}, ties to take t = C - gt_total (1 <= t <= #{S = s*})
+    if (kScanThreads - 1 - tid == sstar + 1) *s_u32 = (uint32_t)cumH;   // s* + 1 <= 97
+    __syncthreads();
+    const int64_t ties = a.C - (int64_t)*s_u32;
+    uint32_t carry_eq = 0, carry_slot = 0;
+    for (int j0 = 0; j0 < a.nchunks; j0 += kScanThreads) {
+        const int j = j0 + tid;
+        uint32_t gt = 0, eq = 0;
+        if (j < a.nchunks) {
+            const uint32_t *cj = a.chunk_cum + ((size_t)unit * a.max_chunks + j) * kCum;
+            const uint32_t c0 = __ldcg(cj + sstar), c1 = __ldcg(cj + sstar + 1);
+            gt = c1;
+            eq = c0 - c1;
+        }
+        uint32_t tot_eq;
+        const uint32_t ex_eq = carry_eq + block_excl_scan<kScanThreads>(eq, s_ws, &tot_eq);
+        const int64_t room = ties - (int64_t)ex_eq;
+        const uint32_t quota = room <= 0 ? 0u : (room >= (int64_t)eq ? eq : (uint32_t)room);
+        uint32_t tot_slot;
+        const uint32_t ex_slot = carry_slot + block_excl_scan<kScanThreads>(gt + quota, s_ws, &tot_slot);
+        if (j < a.nchunks) a.chunk_info[(size_t)unit * a.max_chunks + j] = make_uint2(ex_slot, quota);
+        carry_eq += tot_eq;
+        carry_slot += tot_slot;
+    }
+    __syncthreads();                          // s_ws, s_int, s_u32 free for the next unit
 }
 
 __global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
@@ -156,23 +230,13 @@ __global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
     }
     __syncthreads();
 
-    // chunk histogram -> suffix counts cum[s] = #{S >= s}, s = 0..97
+    // chunk histogram -> suffix counts
     uint32_t hv = 0;
     if (tid < kBins) {
 #pragma unroll
         for (int w = 0; w < NW; w++) hv += s_hist[w][tid];
     }
-    if (tid < kHistPad) s_cum[tid] = (tid < kBins) ? hv : 0u;
-    __syncthreads();
-    // suffix sum by a reversed exclusive scan over 256 threads
-    {
-        const int s = kScanThreads - 1 - tid;   // thread tid handles bin s (descending)
-        const uint32_t v = (s < kBins) ? s_cum[s] : 0u;
-        uint32_t tot;
-        const uint32_t ex = block_excl_scan<kScanThreads>(v, s_ws, &tot);
-        if (s < kCum) a.chunk_cum[((size_t)bh * a.max_chunks + chunk) * kCum + s] = ex + v;
-    }
-    if (tid < kBins && hv) atomicAdd(&a.head_hist[(size_t)bh * kBins + tid], hv);
+    chunk_suffix(a, bh, chunk, hv, s_cum, s_ws);
 
     __threadfence();
     __syncthreads();
@@ -181,55 +245,112 @@ __global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-
     // ---- last CTA of this pair: threshold and per-chunk candidate slots
-    uint32_t H = 0;
-    if (tid < kBins) H = __ldcg(&a.head_hist[(size_t)bh * kBins + tid]);
-    if (a.dbg_hist && tid < kBins) a.dbg_hist[(size_t)bh * kBins + tid] = H;
-    int64_t cumH;
-    {
-        const int s = kScanThreads - 1 - tid;
-        const uint32_t v = (s < kBins) ? __ldcg(&a.head_hist[(size_t)bh * kBins + s]) : 0u;
-        uint32_t tot;
-        const uint32_t ex = block_excl_scan<kScanThreads>(v, s_ws, &tot);
-        cumH = (int64_t)(ex + v);           // #{S >= s} for s = 255 - tid
-        // s* = largest s with #{S >= s} >= C  (cum is non-increasing in s)
-        const int pred = (s < kCum) && (cumH >= a.C);
-        const int nsat = __syncthreads_count(pred);
-        if (tid == 0) s_last = nsat - 1;    // reuse as s*
-    }
-    __syncthreads();
-    const int sstar = s_last;
-    if (tid == 0) {
-        a.sstar[bh] = sstar;
-        if (a.dbg_sstar) a.dbg_sstar[bh] = sstar;
-        a.tickets[(size_t)bh * 2 + 0] = 0u;
-    }
-    // gt_total = #{S > s*}, ties to take t = C - gt_total (1 <= t <= #{S = s*})
     __shared__ uint32_t s_gt_total;
-    if (kScanThreads - 1 - tid == sstar + 1) s_gt_total = (uint32_t)cumH;   // s* + 1 <= 97
-    __syncthreads();
-    const int64_t ties = a.C - (int64_t)s_gt_total;
-    uint32_t carry_eq = 0, carry_slot = 0;
-    for (int j0 = 0; j0 < a.nchunks; j0 += kScanThreads) {
-        const int j = j0 + tid;
-        uint32_t gt = 0, eq = 0;
-        if (j < a.nchunks) {
-            const uint32_t *cj = a.chunk_cum + ((size_t)bh * a.max_chunks + j) * kCum;
-            const uint32_t c0 = __ldcg(cj + sstar), c1 = __ldcg(cj + sstar + 1);
-            gt = c1;
-            eq = c0 - c1;
-        }
-        uint32_t tot_eq;
-        const uint32_t ex_eq = carry_eq + block_excl_scan<kScanThreads>(eq, s_ws, &tot_eq);
-        const int64_t room = ties - (int64_t)ex_eq;
-        const uint32_t quota = room <= 0 ? 0u : (room >= (int64_t)eq ? eq : (uint32_t)room);
-        uint32_t tot_slot;
-        const uint32_t ex_slot = carry_slot + block_excl_scan<kScanThreads>(gt + quota, s_ws, &tot_slot);
-        if (j < a.nchunks) a.chunk_info[(size_t)bh * a.max_chunks + j] = make_uint2(ex_slot, quota);
-        carry_eq += tot_eq;
-        carry_slot += tot_slot;
+    unit_threshold(a, bh, s_ws, &s_last, &s_gt_total);
+    if (tid == 0) a.tickets[(size_t)bh * 2 + 0] = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// Per-query-head retrieval: one pass over a pair's codes scores it for all G
+// query heads of the pair (units pair G + g).  The G bonus tables are packed
+// into one table per (block, centre) in shared memory -- NP words, byte g of
+// word p holding the bonus of head 4p + g -- so one lookup per code yields the
+// bonuses of every head, and summing the 16 words of a key gives every head's
+// S in its own byte (S <= 96: no carry between bytes).  Then each head's S,
+// histogram, suffix counts and threshold go through the same steps as the
+// single-query scan.
+template <int NP>
+__global__ void __launch_bounds__(kScanThreads) k_collision_scan_heads(ScanArgs a)
+{
+    const int pair = blockIdx.y, chunk = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = kScanThreads / 32;
+    const int G = a.kvg;
+    const int u0 = pair * G;                      // the pair's first query unit
+    extern __shared__ __align__(16) uint32_t s_dyn[];
+    uint32_t *ptab = s_dyn;                       // [kB * kNC][NP]
+    uint32_t *s_hist = s_dyn + kB * kNC * NP;     // [NW][G][kHistPad]
+    __shared__ uint32_t s_cum[kHistPad];
+    __shared__ uint32_t s_ws[NW + 1];
+    __shared__ int s_last;
+    __shared__ uint32_t s_gt_total;
+
+    for (int i = tid; i < NW * G * kHistPad; i += kScanThreads) s_hist[i] = 0u;
+    pdl_wait();                                   // bonus tables come from the query preparation
+    for (int e = tid; e < kB * kNC; e += kScanThreads) {
+        uint32_t w[NP];
+#pragma unroll
+        for (int p = 0; p < NP; p++) w[p] = 0u;
+        for (int g = 0; g < G; g++)
+            w[g >> 2] |= (uint32_t)a.bonus_bytes[(size_t)(u0 + g) * kB * kNC + e] << (8 * (g & 3));
+#pragma unroll
+        for (int p = 0; p < NP; p++) ptab[e * NP + p] = w[p];
     }
+    __syncthreads();
+
+    const int64_t lo = (int64_t)chunk * a.chunk;
+    const int64_t hi = min(lo + a.chunk, a.n);
+    const uint32_t ucnt = (uint32_t)(hi - lo);
+    const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes + ((size_t)pair * a.n_cap + lo) * kB);
+    uint8_t *S0 = a.S + (size_t)u0 * a.n_cap + lo;
+    uint32_t *hw = s_hist + warp * G * kHistPad;
+    constexpr int U = 2;                          // keys per lane per iteration
+    const uint32_t step = (uint32_t)NW * 32 * U;
+    for (uint32_t base = (uint32_t)warp * 32 * U + lane; base < ucnt + lane; base += step) {
+        uint4 c[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const uint32_t i = base + u * 32;
+            c[u] = (i < ucnt) ? __ldcs(codes + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const uint32_t i = base + u * 32;
+            uint32_t acc[NP];
+#pragma unroll
+            for (int p = 0; p < NP; p++) acc[p] = 0u;
+            const uint32_t wds[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    const uint32_t e = (uint32_t)(256 * (4 * q + k)) + ((wds[q] >> (8 * k)) & 0xffu);
+                    if (NP == 1) {
+                        acc[0] += ptab[e];
+                    } else {
+                        const uint2 v = reinterpret_cast<const uint2 *>(ptab)[e];
+                        acc[0] += v.x;
+                        acc[NP - 1] += v.y;
+                    }
+                }
+            }
+            if (i < ucnt) {
+                for (int g = 0; g < G; g++) {
+                    const uint32_t sg = (acc[g >> 2] >> (8 * (g & 3))) & 0xffu;
+                    S0[(size_t)g * a.n_cap + i] = (uint8_t)sg;
+                    atomicAdd(&hw[g * kHistPad + sg], 1u);
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    for (int g = 0; g < G; g++) {
+        uint32_t hv = 0;
+        if (tid < kBins)
+            for (int w = 0; w < NW; w++) hv += s_hist[(w * G + g) * kHistPad + tid];
+        chunk_suffix(a, u0 + g, chunk, hv, s_cum, s_ws);
+    }
+    __threadfence();
+    __syncthreads();
+    pdl_trigger();
+    if (tid == 0) s_last = (atomicAdd(&a.tickets[(size_t)u0 * 2 + 0], 1u) == (unsigned)(a.nchunks - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int g = 0; g < G; g++) unit_threshold(a, u0 + g, s_ws, &s_last, &s_gt_total);
+    if (tid == 0) a.tickets[(size_t)u0 * 2 + 0] = 0u;
 }
 
 }  // namespace pk
@@ -238,5 +359,22 @@ namespace pk {
 cudaError_t launch_collision_scan(const ScanArgs &a, int bh, cudaStream_t s)
 {
     return launch_pdl(k_collision_scan, dim3(a.nchunks, bh), dim3(kScanThreads), 0, s, a);
+}
+
+size_t scan_heads_smem(int np, int G) { return ((size_t)kB * kNC * np + (size_t)(kScanThreads / 32) * G * kHistPad) * 4; }
+
+cudaError_t launch_collision_scan_heads(const ScanArgs &a, int pairs, cudaStream_t s)
+{
+    static std::atomic<int> set1[kMaxDevices], set2[kMaxDevices];
+    if (a.kvg <= 4) {
+        const cudaError_t e = dyn_smem_limit(k_collision_scan_heads<1>, (int)scan_heads_smem(1, 4), set1);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(k_collision_scan_heads<1>, dim3(a.nchunks, pairs), dim3(kScanThreads),
+                          scan_heads_smem(1, a.kvg), s, a);
+    }
+    const cudaError_t e = dyn_smem_limit(k_collision_scan_heads<2>, (int)scan_heads_smem(2, kMaxGroup), set2);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_collision_scan_heads<2>, dim3(a.nchunks, pairs), dim3(kScanThreads),
+                      scan_heads_smem(2, a.kvg), s, a);
 }
 }  // namespace pk

@@ -19,6 +19,9 @@ struct TraceRec {
 // query, G per pair for per-query-head search.
 struct Work {
     int32_t units = 0;
+    int32_t scan_units = 0;      // CTAs' worth of work units per chunk of the scan: units, or pairs
+                                 // when one scan pass serves the G query heads of a pair
+    uint8_t *bonus_bytes = nullptr;   // [units][16][256] bonus per centre (per-head search)
     int32_t max_chunks = 1, max_slices = 1;
     float *qt = nullptr, *qnorm = nullptr;
     uint32_t *bonus_packed = nullptr;
@@ -141,7 +144,7 @@ uint64_t splitmix64(uint64_t x)
 // ceil(n / kMaxChunk) chunks.
 void chunking(const pk_index *ix, const Work &w, int64_t n, int32_t *nchunks, int64_t *chunk)
 {
-    int64_t nch = std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / w.units);
+    int64_t nch = std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / w.scan_units);
     nch = std::min<int64_t>(nch, ceil_div(n, kMinChunk));
     nch = std::max<int64_t>(nch, ceil_div(n, kMaxChunk));
     nch = std::max<int64_t>(1, std::min<int64_t>(nch, w.max_chunks));
@@ -200,18 +203,21 @@ void work_free(Work &w)
     cudaFree(w.sstar);
     cudaFree(w.cand);
     cudaFree(w.partial);
+    cudaFree(w.bonus_bytes);
     w = Work{};
 }
 
 template <typename T>
 cudaError_t dalloc(T **p, size_t count);
 
-// Workspace for `units` query units of an index of capacity n_cap; the
-// counters start at zero.  On failure nothing stays allocated.
-cudaError_t work_alloc(pk_index *ix, Work &w, int32_t units, int64_t n_cap, cudaStream_t s)
+// Workspace for `units` query units (kvg per index pair) of an index of
+// capacity n_cap; the counters start at zero.  On failure nothing stays
+// allocated.
+cudaError_t work_alloc(pk_index *ix, Work &w, int32_t units, int32_t kvg, int64_t n_cap, cudaStream_t s)
 {
     w.units = units;
-    w.max_chunks = (int32_t)std::max<int64_t>(std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / units),
+    w.scan_units = units / kvg;
+    w.max_chunks = (int32_t)std::max<int64_t>(std::max<int64_t>(1, (4 * (int64_t)ix->num_sms) / w.scan_units),
                                               ceil_div(n_cap, kMaxChunk) + 1);
     {   // largest slice count any C <= n_cap can need
         const int64_t lo = slice_lo(ix);
@@ -233,6 +239,7 @@ cudaError_t work_alloc(pk_index *ix, Work &w, int32_t units, int64_t n_cap, cuda
     chk(dalloc(&w.sstar, U));
     chk(dalloc(&w.cand, U * NC));
     chk(dalloc(&w.partial, U * MS * (size_t)ix->topk_cap));
+    if (kvg > 1) chk(dalloc(&w.bonus_bytes, U * kB * kNC));
     chk(cudaMemsetAsync(w.head_hist, 0, U * kBins * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(w.tickets, 0, U * 2 * sizeof(uint32_t), s));
     if (e != cudaSuccess) {
@@ -388,6 +395,7 @@ pk_status search_impl(pk_index *ix, Work &w, int32_t kvg, const void *q, int32_t
         pa.dbg_qt = dbg->qt;
         pa.dbg_qnorm = dbg->qnorm;
     }
+    if (kvg > 1) pa.dbg_bonus = w.bonus_bytes;   // the per-head scan reads the bonus bytes
     trace_begin(ix, PK_K_QUERY_PREP, s);
     cudaError_t e = launch_query_prep(pa, s);
     trace_end(ix, s);
@@ -415,7 +423,12 @@ pk_status search_impl(pk_index *ix, Work &w, int32_t kvg, const void *q, int32_t
         sa.dbg_sstar = dbg->sstar;
     }
     trace_begin(ix, PK_K_COLLISION_SCAN, s);
-    e = launch_collision_scan(sa, w.units, s);
+    if (kvg > 1) {   // one pass over each pair's codes for its kvg query heads
+        sa.bonus_bytes = w.bonus_bytes;
+        e = launch_collision_scan_heads(sa, w.units / kvg, s);
+    } else {
+        e = launch_collision_scan(sa, w.units, s);
+    }
     trace_end(ix, s);
     if (e != cudaSuccess) return cuda_status(e);
 
@@ -632,7 +645,7 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(dalloc(&ix->codes, BH * NC * kB));
     chk(dalloc(&ix->rec, BH * NC * kRecBytes));
     chk(dalloc(&ix->occ, BH * kB * kNC));
-    chk(work_alloc(ix, ix->w, ix->bh, n_cap, s));
+    chk(work_alloc(ix, ix->w, ix->bh, 1, n_cap, s));
 
     chk(dalloc(&ix->dev_err, 1));
     chk(dalloc(&ix->dev_err_detail, 1));
@@ -762,7 +775,7 @@ pk_status pk_search_heads(pk_index *ix, const void *q, int32_t topk, int32_t *ou
     if (!ix) return PK_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     if (ix->wh.units == 0) {      // the per-head workspace, made on first use
-        const cudaError_t e = work_alloc(ix, ix->wh, ix->bh * ix->p.group, ix->p.n_cap, s);
+        const cudaError_t e = work_alloc(ix, ix->wh, ix->bh * ix->p.group, ix->p.group, ix->p.n_cap, s);
         if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? PK_ERR_OOM : PK_ERR_CUDA;
     }
     return search_impl(ix, ix->wh, ix->p.group, q, topk, out_idx, out_score, nullptr, s);

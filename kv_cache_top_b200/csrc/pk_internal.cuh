@@ -76,6 +76,7 @@ struct PrepArgs {
 struct ScanArgs {
     const uint8_t *codes;
     const uint32_t *bonus_packed;
+    const uint8_t *bonus_bytes;   // [units][16][256] (one pass for the kvg query heads of a pair)
     int64_t n, n_cap, chunk, C;   // n_cap: row stride of the per-key arrays
     int32_t nchunks;
     int32_t kvg;             // query units per index pair
@@ -288,6 +289,7 @@ cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
 cudaError_t launch_occ_merge(uint32_t *occ, uint32_t *add, int64_t count, cudaStream_t s);
 cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s);
 cudaError_t launch_collision_scan(const ScanArgs &a, int bh, cudaStream_t s);
+cudaError_t launch_collision_scan_heads(const ScanArgs &a, int pairs, cudaStream_t s);
 cudaError_t launch_compact(const CompactArgs &a, int nchunks, int bh, cudaStream_t s);
 cudaError_t launch_rerank_topk(const RerankArgs &a, int bh, cudaStream_t s);
 cudaError_t launch_topk_merge(const MergeArgs &a, int bh, cudaStream_t s);
