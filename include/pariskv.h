@@ -137,7 +137,9 @@ void pk_default_params(pk_params *p);
  *   n      1 <= n <= n_cap (n_cap 0 means n).
  * On success *out owns: codes [BH][n_cap][16] u8, summary records
  * [BH][n_cap][128 B], occupancy [BH][16][256] u32, search workspace, and the
- * K/V store [BH][n_cap][D] (HBM, or cudaHostAlloc'd mapped host memory).
+ * K/V store [BH][n_cap][2][D] (HBM, or cudaHostAlloc'd mapped host memory;
+ * the K and V rows of a key are adjacent, so gathering a selected key's rows
+ * touches one page of a host-resident store instead of two).
  * Errors: PK_ERR_INVALID_ARG, PK_ERR_UNSUPPORTED, PK_ERR_CAPACITY,
  * PK_ERR_OOM (nothing leaks), PK_ERR_CUDA. */
 pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_params *params,

@@ -89,8 +89,8 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
     const int32_t id0 = (tid < kAtRows && rr0 < r_end && rr0 < a.topk) ? a.idx[(size_t)bh * a.topk + rr0] : 0;
     for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][qpad(i % kD)] = ld_as_f32(a.q, qbase + i, a.is_bf16);
     const size_t kp = (size_t)index_pair(bh, a.kvg);     // the index pair holding this unit's rows
-    const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + kp * a.stride * row_bytes;
-    const unsigned char *Vb = reinterpret_cast<const unsigned char *>(a.V) + kp * a.stride * row_bytes;
+    const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + kp * a.stride * a.kv_pitch;
+    const unsigned char *Vb = reinterpret_cast<const unsigned char *>(a.V) + kp * a.stride * a.kv_pitch;
     const unsigned char *dKb = a.dlen ? reinterpret_cast<const unsigned char *>(a.dK) + kp * a.dstride * row_bytes : nullptr;
     const unsigned char *dVb = a.dlen ? reinterpret_cast<const unsigned char *>(a.dV) + kp * a.dstride * row_bytes : nullptr;
     const int d = tid & (kD - 1);
@@ -127,8 +127,8 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
                 const int r = i / vpr, c = i - r * vpr;
                 const int32_t id = s_idx[r];
                 if (id >= 0) {
-                    kr[u] = *reinterpret_cast<const uint4 *>(Kb + (size_t)id * row_bytes + 16 * c);
-                    vr[u] = *reinterpret_cast<const uint4 *>(Vb + (size_t)id * row_bytes + 16 * c);
+                    kr[u] = *reinterpret_cast<const uint4 *>(Kb + (size_t)id * a.kv_pitch + 16 * c);
+                    vr[u] = *reinterpret_cast<const uint4 *>(Vb + (size_t)id * a.kv_pitch + 16 * c);
                 } else if (id <= -2) {
                     const size_t j = (size_t)(-2 - id);
                     kr[u] = *reinterpret_cast<const uint4 *>(dKb + j * row_bytes + 16 * c);

@@ -49,8 +49,10 @@ struct pk_index {
     uint8_t *codes = nullptr;
     uint8_t *rec = nullptr;
     uint32_t *occ = nullptr;
-    // K/V store (device, or mapped pinned host)
-    void *K = nullptr, *V = nullptr;
+    // K/V store (device, or mapped pinned host): one allocation [BH][stride][2][D],
+    // the K and V rows of a key adjacent (one translation covers both when the
+    // attention gathers them); K and V point at the first K and V row
+    void *KV = nullptr, *K = nullptr, *V = nullptr;
     bool kv_host = false;
     // staged appends: n_staged keys encoded at rows n .. n + n_staged - 1,
     // their occupancy counts in occ_stage [BH][16][256] (zero when nothing is
@@ -255,13 +257,8 @@ void free_all(pk_index *ix)
     cudaFree(ix->codes);
     cudaFree(ix->rec);
     cudaFree(ix->occ);
-    if (ix->kv_host) {
-        cudaFreeHost(ix->K);
-        cudaFreeHost(ix->V);
-    } else {
-        cudaFree(ix->K);
-        cudaFree(ix->V);
-    }
+    if (ix->kv_host) cudaFreeHost(ix->KV);
+    else cudaFree(ix->KV);
     work_free(ix->w);
     work_free(ix->wh);
 
@@ -343,15 +340,18 @@ pk_status encode_range(pk_index *ix, const void *Kin, int64_t k_stride, int64_t 
 }
 
 // copy rows 0..n_new-1 of every pair of src ([BH][src_stride][D]) into the
-// store at positions pos0.. of each pair
+// K (store = ix->K) or V (store = ix->V) rows at positions pos0.. of each
+// pair of the interleaved store: one 3-D copy, rows 2 D apart in the store
 pk_status copy_rows(pk_index *ix, void *store, const void *src, int64_t src_stride, int64_t n_new,
                     int64_t pos0, cudaStream_t s)
 {
     const size_t row = (size_t)kD * ix->es;
-    cudaError_t e = cudaMemcpy2DAsync((char *)store + (size_t)pos0 * row, (size_t)ix->stride * row,
-                                      src, (size_t)src_stride * row, (size_t)n_new * row, (size_t)ix->bh,
-                                      cudaMemcpyDefault, s);
-    return cuda_status(e);
+    cudaMemcpy3DParms p = {};
+    p.srcPtr = make_cudaPitchedPtr(const_cast<void *>(src), row, row, (size_t)src_stride);
+    p.dstPtr = make_cudaPitchedPtr((char *)store + (size_t)pos0 * 2 * row, 2 * row, row, (size_t)ix->stride);
+    p.extent = make_cudaExtent(row, (size_t)n_new, (size_t)ix->bh);
+    p.kind = cudaMemcpyDefault;
+    return cuda_status(cudaMemcpy3DAsync(&p, s));
 }
 
 // One search over work `w`: kvg query units per index pair (1: the
@@ -515,6 +515,7 @@ pk_status attend_impl(pk_index *ix, int32_t kvg, const void *q, const int32_t *s
     a.idx = sel_idx;
     a.K = ix->K;
     a.V = ix->V;
+    a.kv_pitch = 2 * (int64_t)kD * ix->es;
     a.out = out;
     a.n = ix->n;
     a.stride = ix->stride;
@@ -649,14 +650,16 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
 
     chk(dalloc(&ix->dev_err, 1));
     chk(dalloc(&ix->dev_err_detail, 1));
-    const size_t kv_bytes = BH * NC * kD * (size_t)es;
+    const size_t kv_bytes = 2 * BH * NC * kD * (size_t)es;
     if (params->kv_location == PK_KV_HOST_PINNED) {
         ix->kv_host = true;
-        chk(cudaHostAlloc(&ix->K, kv_bytes, cudaHostAllocMapped | cudaHostAllocPortable));
-        chk(cudaHostAlloc(&ix->V, kv_bytes, cudaHostAllocMapped | cudaHostAllocPortable));
+        chk(cudaHostAlloc(&ix->KV, kv_bytes, cudaHostAllocMapped | cudaHostAllocPortable));
     } else {
-        chk(cudaMalloc(&ix->K, kv_bytes));
-        chk(cudaMalloc(&ix->V, kv_bytes));
+        chk(cudaMalloc(&ix->KV, kv_bytes));
+    }
+    if (ix->KV) {
+        ix->K = ix->KV;
+        ix->V = (char *)ix->KV + (size_t)kD * es;
     }
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -823,7 +826,7 @@ pk_status pk_get_info(const pk_index *ix, pk_info *info)
     chunking(ix, ix->w, ix->n, &info->nchunks, &info->chunk);
     resolve(ix->n, ix->p.cand_budget, ix->p.collision_ratio, ix->p.topk, &info->cand, &info->coll);
     info->index_bytes = (int64_t)ix->bh * ix->stride * (kB + kRecBytes) + (int64_t)ix->bh * kB * kNC * 4;
-    info->kv_bytes = 2 * (int64_t)ix->bh * ix->stride * kD * ix->es;
+    info->kv_bytes = 2 * (int64_t)ix->bh * ix->stride * kD * ix->es;   // K and V rows
     info->kv_location = ix->p.kv_location;
     info->num_sms = ix->num_sms;
     return PK_OK;

@@ -121,8 +121,9 @@ struct RerankArgs {
 struct AttendArgs {
     const void *q;           // [batch][H*G][D]
     const int32_t *idx;      // [BH][topk]
-    const void *K;           // [BH][stride][D]  (device or mapped host)
-    const void *V;
+    const void *K;           // first K row of the store [BH][stride][2][D] (device or mapped host)
+    const void *V;           // first V row
+    int64_t kv_pitch;        // bytes from one key's rows to the next
     float *out;              // [batch][H*G][D]
     int64_t n, stride;
     int32_t H, G, topk, is_bf16;
