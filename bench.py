@@ -240,12 +240,17 @@ def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
     batch, n, H, G = wl["batch"], wl["n"], wl["H"], wl["G"]
     bh, topk, nq = batch * H, 100, 64
     w = workloads.llama_layer(batch, n, H=H, G=G, seed=seed, device=dev, n_queries=nq)
+    n_app = 4096                                       # keys per pair appended after the timed passes
     p = pk.pk_default_params(batch=batch, n_kv_heads=H, group=G, topk=topk, cand_budget=wl["cand"],
-                             kv_dtype=pk.PK_BF16,
+                             kv_dtype=pk.PK_BF16, n_cap=n + n_app,
                              kv_location=pk.PK_KV_HOST_PINNED if wl["kv_host"] else pk.PK_KV_DEVICE)
     stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    t_b = time.perf_counter()
     h = pk.pk_build_index(w["K"], w["V"], n, p)
     torch.cuda.synchronize()
+    build_s = time.perf_counter() - t_b
+    k_app = torch.randn(batch, H, n_app, 128, device=dev).to(torch.bfloat16)
     C, R = pk.pk_resolve(n, wl["cand"], 0.0, topk)
     info = pk.pk_get_info(h)
     q = w["q"]
@@ -371,8 +376,25 @@ def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
                "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]}
 
+    # index build (host wall clock: allocation, K/V copy-in, encode) and the
+    # encode kernel alone on one append of n_app keys per pair
+    torch.cuda.synchronize()
+    pk.pk_trace_enable(h, True)
+    pk.pk_trace_read(h)
+    pk.pk_append(h, k_app, k_app, n_app)
+    enc = pk.pk_trace_read(h)["encode"]
+    pk.pk_trace_enable(h, False)
+    enc_us = enc[1] * 1000.0 / max(1, enc[0])
+    keys_app = bh * n_app
+    build = {"build_s_wall": build_s, "keys": bh * n,
+             "build_keys_per_s": bh * n / build_s,
+             "append_keys": keys_app, "encode_us": enc_us, "encode_keys_per_s": keys_app / (enc_us * 1e-6),
+             "encode_gbs": keys_app * (128 * 2 + 16 + 128) / (enc_us * 1e-3) / 1e6,
+             "encode_bytes_per_key": "256 B of K read + 144 B of codes and record written"}
+    del k_app
+
     res = dict(ms_total=ms_clean, wall=wall_clean, kern=kern, recall=recall, C=C, R=R, info=info,
-               e2e=e2e, clocks=clocks, ms_traced=ms_traced, graph=graphs is not None)
+               e2e=e2e, clocks=clocks, ms_traced=ms_traced, graph=graphs is not None, build=build)
     del graphs
 
     # dense-attention comparator on the same tensors (HBM workloads only)
@@ -417,17 +439,16 @@ def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
         del hb, db
 
     # CPU baseline: the oracle on a bounded sample of the same workload, on
-    # one core and (HBM workloads) on all host cores
+    # one core and on all host cores
     if want_cpu:
         single = cpu_baseline(wl, seed, w if not wl["kv_host"] else None, dev)
         res["cpu"] = single
-        if not wl["kv_host"]:
-            try:
-                par = cpu_baseline_parallel(wl, seed)
-                par["single_core"] = single
-                res["cpu"] = par
-            except Exception as e:          # the one-core figure stands
-                single["parallel_error"] = str(e)[:200]
+        try:
+            par = cpu_baseline_parallel(wl, seed, queries=64 if wl["n"] <= 200000 else 4 * bh)
+            par["single_core"] = single
+            res["cpu"] = par
+        except Exception as e:          # the one-core figure stands
+            single["parallel_error"] = str(e)[:200]
 
     pk.pk_free(h)
     del w, flush
@@ -444,8 +465,8 @@ def cpu_baseline(wl, seed, w, dev, pairs_wanted=4, queries=32):
     batch, n, H, G = wl["batch"], wl["n"], wl["H"], wl["G"]
     bh = batch * H
     pairs = sorted({(i * bh) // pairs_wanted for i in range(pairs_wanted)})
-    if n > 200000:
-        pairs, queries = pairs[:1], 8
+    if n > 200000:                      # one pair, 4 steps' worth of pair-searches (4 x bh)
+        pairs, queries = pairs[:1], 4 * bh
     tot, cnt = 0.0, 0
     for pidx in pairs:
         b, hh = divmod(pidx, H)
@@ -582,7 +603,7 @@ def main():
                "host_link_frac_of_h2d_copy": ((link_bytes / (att["avg_us"] * 1e-6) / 1e9) / rm["h2d_gbs"])
                if att and rm.get("h2d_gbs") else None,
                "kernels": km, "cand_budget": rm["C"], "collision_budget": rm["R"],
-               "cpu_baseline": rm.get("cpu")}
+               "index_build": rm["build"], "cpu_baseline": rm.get("cpu")}
 
     if world > 1:
         torch.distributed.barrier()
@@ -631,6 +652,7 @@ def main():
         "cpu_baseline": res.get("cpu"),
         "wall_s_timed_region": res["wall"],
         "ms_per_step_traced": res["ms_traced"] / args.steps,
+        "index_build": res["build"],
     }
     if "dense" in res:
         line["dense_attention"] = res["dense"]
@@ -664,7 +686,9 @@ def run_drift(args, wl, peaks):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(T)]
     recalls = []
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     for t in range(T):
+        flush.zero_()                                 # the index (~95 MB) would stay in L2 otherwise
         ev[t][0].record(stream)
         pk.pk_append(h, w["k_new"][t], w["v_new"][t], 1)
         pk.pk_search(h, w["q"][t], 100, idx)
@@ -686,7 +710,7 @@ def run_drift(args, wl, peaks):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wl["name"], "n_prefill": n0, "kv_heads": H, "q_heads": H, "head_dim": 128,
                        "topk": 100, "step": "pk_append (1 key per KV head) + pk_search",
-                       "l2": "not flushed (each step touches the index once)"},
+                       "l2": "flushed between steps (256 MiB write outside the events)"},
             "recall_at_100": [{"step": a, "recall": b} for a, b in recalls],
             "recall_at_100_mean": sum(b for _, b in recalls) / max(1, len(recalls)),
             "gpu_launches": None}

@@ -70,7 +70,8 @@ typedef enum {
     PK_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
     PK_ERR_TIMEOUT = 5,       /* reserved: a bounded device wait gave up        */
     PK_ERR_DEVICE_CHECK = 6,  /* a device-side check recorded a bad value       */
-    PK_ERR_UNSUPPORTED = 7    /* head_dim != 128, sub_dim != 8, topk > 1024     */
+    PK_ERR_UNSUPPORTED = 7    /* head_dim != 128, sub_dim != 8, topk > 1024,
+                                 batch * n_kv_heads * group > 65535             */
 } pk_status;
 
 typedef enum { PK_F32 = 0, PK_BF16 = 1 } pk_dtype;

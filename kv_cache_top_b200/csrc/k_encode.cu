@@ -116,6 +116,34 @@ __global__ void __launch_bounds__(32 * kEncWarps) k_encode_shared(EncodeArgs a)
     }
 }
 
+// K and V rows into the interleaved store: rows 0..n_new-1 of every pair of
+// srcK / srcV ([BH][src_stride][D], row_bytes each, device or mapped host) go
+// to positions pos0.. of the pair in the store, K at dstK, V at dstV, rows
+// `pitch` bytes apart and pairs `pair_rows` rows apart.  Consecutive threads
+// copy consecutive 16-byte pieces, so a row is one coalesced write (posted
+// writes over the host link when the store is pinned host memory).
+// CTA (x, p) copies rows x kStoreRows .. of pair p; a row is per_row =
+// 2^lg 16-byte pieces (16 for bf16, 32 for fp32).
+constexpr int kStoreRows = 64;
+__global__ void __launch_bounds__(256) k_store_rows(StoreArgs a)
+{
+    const int lg = a.row_bytes == 512 ? 5 : 4;
+    const int64_t p = blockIdx.y;
+    const int64_t r0 = (int64_t)blockIdx.x * kStoreRows;
+    const int rows = (int)min((int64_t)kStoreRows, a.n_new - r0);
+    const unsigned char *sK = a.srcK + (size_t)(p * a.src_stride + r0) * a.row_bytes;
+    const unsigned char *sV = a.srcV + (size_t)(p * a.src_stride + r0) * a.row_bytes;
+    unsigned char *dK = a.dstK + (size_t)(p * a.pair_rows + a.pos0 + r0) * a.pitch;
+    unsigned char *dV = a.dstV + (size_t)(p * a.pair_rows + a.pos0 + r0) * a.pitch;
+    for (int e = threadIdx.x; e < (rows << lg); e += 256) {
+        const int r = e >> lg, c = e & ((1 << lg) - 1);
+        const uint4 k = *reinterpret_cast<const uint4 *>(sK + (size_t)r * a.row_bytes + 16 * c);
+        const uint4 v = *reinterpret_cast<const uint4 *>(sV + (size_t)r * a.row_bytes + 16 * c);
+        *reinterpret_cast<uint4 *>(dK + (size_t)r * a.pitch + 16 * c) = k;
+        *reinterpret_cast<uint4 *>(dV + (size_t)r * a.pitch + 16 * c) = v;
+    }
+}
+
 // Publishing staged keys: their counts join the table, and the side table is
 // left at zero for the next staging.
 __global__ void __launch_bounds__(256) k_occ_merge(uint32_t *occ, uint32_t *add, int64_t count)
@@ -139,15 +167,25 @@ cudaError_t launch_occ_merge(uint32_t *occ, uint32_t *add, int64_t count, cudaSt
     return cudaGetLastError();
 }
 
+cudaError_t launch_store_rows(const StoreArgs &a, cudaStream_t s)
+{
+    if (a.n_new <= 0 || a.bh <= 0) return cudaSuccess;
+    if (a.bh > 65535) return cudaErrorInvalidValue;
+    const int64_t gx = (a.n_new + kStoreRows - 1) / kStoreRows;
+    k_store_rows<<<dim3((unsigned)gx, (unsigned)a.bh), 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s)
 {
     const int64_t keys = (int64_t)a.bh * a.n_new;
     if (keys <= 0) return cudaSuccess;
-    // the shared-memory counts pay off from a few thousand keys per pair; a
-    // smaller batch (a decode-time re-indexing) takes one warp per key across
-    // all pairs, so its whole batch encodes in parallel
-    if (a.n_new >= 4 * kEncKeysShared && a.bh <= 65535) {
-        const int64_t gx = (a.n_new + kEncKeysShared - 1) / kEncKeysShared;
+    // the shared-memory counts pay off from a few thousand keys per pair, and
+    // their grid (one CTA per 1024 keys of a pair) must fill the GPU; other
+    // batches (a decode-time re-indexing, few pairs) take one warp per key
+    // across all pairs, so the whole batch encodes in parallel
+    const int64_t gx = (a.n_new + kEncKeysShared - 1) / kEncKeysShared;
+    if (a.n_new >= 4 * kEncKeysShared && a.bh <= 65535 && gx * a.bh >= 512) {
         k_encode_shared<<<dim3((unsigned)gx, (unsigned)a.bh), 32 * kEncWarps, 0, s>>>(a);
     } else {
         const int64_t blocks = (keys + kEncWarps - 1) / kEncWarps;   // one key per warp

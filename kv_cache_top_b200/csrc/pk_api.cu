@@ -306,6 +306,8 @@ pk_status check_params(const pk_params *p)
         return PK_ERR_INVALID_ARG;
     if (p->topk < 1) return PK_ERR_INVALID_ARG;
     if (p->topk > kMaxTopk) return PK_ERR_UNSUPPORTED;
+    // one grid row per query unit (pair x query head for per-head search)
+    if ((int64_t)p->batch * p->n_kv_heads * p->group > 65535) return PK_ERR_UNSUPPORTED;
     if (p->kv_dtype != PK_F32 && p->kv_dtype != PK_BF16) return PK_ERR_INVALID_ARG;
     if (p->kv_location != PK_KV_DEVICE && p->kv_location != PK_KV_HOST_PINNED)
         return PK_ERR_INVALID_ARG;
@@ -339,19 +341,39 @@ pk_status encode_range(pk_index *ix, const void *Kin, int64_t k_stride, int64_t 
     return cuda_status(e);
 }
 
-// copy rows 0..n_new-1 of every pair of src ([BH][src_stride][D]) into the
-// K (store = ix->K) or V (store = ix->V) rows at positions pos0.. of each
-// pair of the interleaved store: one 3-D copy, rows 2 D apart in the store
-pk_status copy_rows(pk_index *ix, void *store, const void *src, int64_t src_stride, int64_t n_new,
+// copy rows 0..n_new-1 of every pair of k_src / v_src ([BH][src_stride][D])
+// into the interleaved store at positions pos0.. of each pair: one kernel of
+// 16-byte pieces when both sources are 16-byte aligned, else two 3-D copies
+pk_status copy_rows(pk_index *ix, const void *k_src, const void *v_src, int64_t src_stride, int64_t n_new,
                     int64_t pos0, cudaStream_t s)
 {
-    const size_t row = (size_t)kD * ix->es;
-    cudaMemcpy3DParms p = {};
-    p.srcPtr = make_cudaPitchedPtr(const_cast<void *>(src), row, row, (size_t)src_stride);
-    p.dstPtr = make_cudaPitchedPtr((char *)store + (size_t)pos0 * 2 * row, 2 * row, row, (size_t)ix->stride);
-    p.extent = make_cudaExtent(row, (size_t)n_new, (size_t)ix->bh);
-    p.kind = cudaMemcpyDefault;
-    return cuda_status(cudaMemcpy3DAsync(&p, s));
+    if (!aligned(k_src, 16) || !aligned(v_src, 16)) {
+        const size_t row = (size_t)kD * ix->es;
+        cudaError_t e = cudaSuccess;
+        for (int kv = 0; kv < 2 && e == cudaSuccess; kv++) {
+            cudaMemcpy3DParms p = {};
+            p.srcPtr = make_cudaPitchedPtr(const_cast<void *>(kv ? v_src : k_src), row, row, (size_t)src_stride);
+            p.dstPtr = make_cudaPitchedPtr((char *)(kv ? ix->V : ix->K) + (size_t)pos0 * 2 * row, 2 * row, row,
+                                           (size_t)ix->stride);
+            p.extent = make_cudaExtent(row, (size_t)n_new, (size_t)ix->bh);
+            p.kind = cudaMemcpyDefault;
+            e = cudaMemcpy3DAsync(&p, s);
+        }
+        return cuda_status(e);
+    }
+    StoreArgs a{};
+    a.srcK = reinterpret_cast<const unsigned char *>(k_src);
+    a.srcV = reinterpret_cast<const unsigned char *>(v_src);
+    a.dstK = reinterpret_cast<unsigned char *>(ix->K);
+    a.dstV = reinterpret_cast<unsigned char *>(ix->V);
+    a.src_stride = src_stride;
+    a.n_new = n_new;
+    a.pos0 = pos0;
+    a.pair_rows = ix->stride;
+    a.row_bytes = kD * ix->es;
+    a.pitch = 2 * (int64_t)kD * ix->es;
+    a.bh = ix->bh;
+    return cuda_status(launch_store_rows(a, s));
 }
 
 // One search over work `w`: kvg query units per index pair (1: the
@@ -670,8 +692,7 @@ pk_status pk_build_index(const void *K, const void *V, int64_t n, const pk_param
     chk(cudaMemsetAsync(ix->occ, 0, BH * kB * kNC * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(ix->dev_err, 0, sizeof(int32_t), s));
     chk(cudaMemsetAsync(ix->dev_err_detail, 0, sizeof(long long), s));
-    if (e == cudaSuccess) st = copy_rows(ix, ix->K, K, n, n, 0, s);
-    if (e == cudaSuccess && st == PK_OK) st = copy_rows(ix, ix->V, V, n, n, 0, s);
+    if (e == cudaSuccess) st = copy_rows(ix, K, V, n, n, 0, s);
     if (e == cudaSuccess && st == PK_OK) st = encode_range(ix, K, n, n, 0, ix->occ, s);
     if (e != cudaSuccess || st != PK_OK) {
         cudaStreamSynchronize(s);
@@ -692,8 +713,7 @@ pk_status pk_append(pk_index *ix, const void *k_new, const void *v_new, int64_t 
     if (!device_accessible(k_new) || !device_accessible(v_new)) return PK_ERR_INVALID_ARG;
     if (!aligned(k_new, ix->es) || !aligned(v_new, ix->es)) return PK_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
-    pk_status st = copy_rows(ix, ix->K, k_new, n_new, n_new, ix->n, s);
-    if (st == PK_OK) st = copy_rows(ix, ix->V, v_new, n_new, n_new, ix->n, s);
+    pk_status st = copy_rows(ix, k_new, v_new, n_new, n_new, ix->n, s);
     if (st == PK_OK) st = encode_range(ix, k_new, n_new, n_new, ix->n, ix->occ, s);
     if (st == PK_OK) ix->n += n_new;
     return st;
@@ -722,8 +742,7 @@ pk_status pk_append_stage(pk_index *ix, const void *k_new, const void *v_new, in
         }
     }
     const int64_t pos0 = ix->n + ix->n_staged;
-    pk_status st = copy_rows(ix, ix->K, k_new, src_stride, n_new, pos0, s);
-    if (st == PK_OK) st = copy_rows(ix, ix->V, v_new, src_stride, n_new, pos0, s);
+    pk_status st = copy_rows(ix, k_new, v_new, src_stride, n_new, pos0, s);
     if (st == PK_OK) st = encode_range(ix, k_new, src_stride, n_new, pos0, ix->occ_stage, s);
     if (st == PK_OK) st = cuda_status(cudaEventRecord(ix->stage_ev, s));
     if (st == PK_OK) ix->n_staged += n_new;

@@ -55,6 +55,13 @@ struct EncodeArgs {
     Levels lv;
 };
 
+struct StoreArgs {
+    const unsigned char *srcK, *srcV;   // [BH][src_stride][row_bytes]
+    unsigned char *dstK, *dstV;         // first K / V row of the store
+    int64_t src_stride, n_new, pos0, pair_rows, pitch;
+    int32_t bh, row_bytes;
+};
+
 struct PrepArgs {
     const void *q;           // [batch][H*G][D]
     int32_t H, G, is_bf16, bh;
@@ -286,6 +293,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *ws, ui
 namespace pk {
 // kernel launchers (one per kernel translation unit)
 cudaError_t launch_encode(const EncodeArgs &a, cudaStream_t s);
+cudaError_t launch_store_rows(const StoreArgs &a, cudaStream_t s);
 // occ[i] += add[i], add[i] = 0 for i < count
 cudaError_t launch_occ_merge(uint32_t *occ, uint32_t *add, int64_t count, cudaStream_t s);
 cudaError_t launch_query_prep(const PrepArgs &a, cudaStream_t s);

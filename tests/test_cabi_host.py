@@ -66,12 +66,16 @@ def test_host_argument_checks_reject_before_any_launch(pk):
     assert pk.lib.pk_build_index(None, None, 10, C.byref(p), None, C.byref(h)) == pk._lib.PK_ERR_UNSUPPORTED
     p = pk.pk_default_params(group=0)
     assert pk.lib.pk_build_index(None, None, 10, C.byref(p), None, C.byref(h)) == pk._lib.PK_ERR_INVALID_ARG
+    p = pk.pk_default_params(batch=4096, n_kv_heads=8, group=4)       # 131072 query units
+    assert pk.lib.pk_build_index(None, None, 10, C.byref(p), None, C.byref(h)) == pk._lib.PK_ERR_UNSUPPORTED
     p = pk.pk_default_params()
     assert pk.lib.pk_build_index(None, None, 10, C.byref(p), None, C.byref(h)) == pk._lib.PK_ERR_INVALID_ARG
     assert pk.lib.pk_build_index(None, None, 10, None, None, C.byref(h)) == pk._lib.PK_ERR_INVALID_ARG
     assert pk.lib.pk_search(None, None, 100, None, None, None) == pk._lib.PK_ERR_INVALID_ARG
     assert pk.lib.pk_attend(None, None, None, 100, None, None) == pk._lib.PK_ERR_INVALID_ARG
     assert pk.lib.pk_append(None, None, None, 1, None) == pk._lib.PK_ERR_INVALID_ARG
+    assert pk.lib.pk_append_stage(None, None, None, 1, 0, None) == pk._lib.PK_ERR_INVALID_ARG
+    assert pk.lib.pk_append_publish(None, None) == pk._lib.PK_ERR_INVALID_ARG
     pk.pk_free(None)
 
 

@@ -470,6 +470,28 @@ def test_append_stage_publish(pk):
         pk.pk_free(h)
 
 
+@pytest.mark.parametrize("kv_location", [0, 1])
+def test_build_from_unaligned_kv(pk, kv_location):
+    """K/V inputs aligned to their element size but not to 16 bytes take the
+    copy path for unaligned sources into the interleaved K/V store; the
+    index and the attention are the same."""
+    w = workloads.llama_layer(1, 3000, H=2, G=2, seed=23, device="cuda")
+    K, V = w["K"], w["V"]
+
+    def shifted(x):                                   # same values at a 2-byte offset
+        flat = torch.empty(x.numel() + 8, dtype=x.dtype, device="cuda")
+        y = flat[1:1 + x.numel()].view(x.shape)
+        y.copy_(x)
+        assert y.data_ptr() % 16 != 0
+        return y
+
+    h = build(pk, shifted(K), shifted(V), 3000, 1, 2, 2, kv_location=kv_location)
+    try:
+        check_pairs(pk, h, K, V, w["q"][0], [0, 1], 1, 2, 2, 3000, 100)
+    finally:
+        pk.pk_free(h)
+
+
 def test_search_rejects_bad_arguments(pk):
     w = workloads.llama_layer(1, 300, H=1, G=1, seed=6, device="cuda")
     h = build(pk, w["K"], w["V"], 300, 1, 1, 1)
