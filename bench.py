@@ -457,7 +457,26 @@ def run_ours(args, wl, rank, world, local_rank, want_cpu, peaks):
             torch.cuda.synchronize()
             best = min(best, a_.elapsed_time(b_))
         res["h2d_gbs"] = (256 << 20) / best / 1e6
-        del hb, db
+        # the same pinned buffer read in place by a kernel over UVA (a torch
+        # reduction over a device view of the host pointer): the contiguous
+        # kernel-read rate of the host link
+        hb.fill_(1)
+
+        class _HostView:
+            __cuda_array_interface__ = {"shape": (64 << 20,), "typestr": "<i4",
+                                        "data": (hb.data_ptr(), False), "version": 3}
+        hv = torch.as_tensor(_HostView(), device=dev)
+        best = 1e9
+        for _ in range(5):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            s_ = hv.sum()
+            b_.record(stream)
+            torch.cuda.synchronize()
+            best = min(best, a_.elapsed_time(b_))
+        assert int(s_) == (64 << 20) * 0x01010101
+        res["uva_read_gbs"] = (256 << 20) / best / 1e6
+        del hv, hb, db
 
     # CPU baseline: the oracle on a bounded sample of the same workload, on
     # one core and on all host cores
@@ -623,6 +642,9 @@ def main():
                "h2d_copy_gbs": rm.get("h2d_gbs"),
                "host_link_frac_of_h2d_copy": ((link_bytes / (att["avg_us"] * 1e-6) / 1e9) / rm["h2d_gbs"])
                if att and rm.get("h2d_gbs") else None,
+               "uva_read_gbs": rm.get("uva_read_gbs"),
+               "host_link_frac_of_uva_read": ((link_bytes / (att["avg_us"] * 1e-6) / 1e9) / rm["uva_read_gbs"])
+               if att and rm.get("uva_read_gbs") else None,
                "kernels": km, "cand_budget": rm["C"], "collision_budget": rm["R"],
                "index_build": rm["build"], "cpu_baseline": rm.get("cpu")}
 
