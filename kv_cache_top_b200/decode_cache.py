@@ -45,6 +45,78 @@ from . import (PK_BF16, PK_F32, PK_KV_DEVICE, PK_KV_HOST_PINNED, pk_append, pk_a
                pk_search)
 
 
+class ReindexPlan:
+    """Which tokens move from the dense tail into the index, and when (pure
+    bookkeeping: no tensors, no GPU).  before_token() is called at the start
+    of a decode step, before the step's token joins the tail, and returns the
+    step's actions, each with the tail length it saw:
+      ("reindex", tail)             in line: pk_append of the oldest `update`
+                                    tail tokens;
+      ("stage", first, count, tail) stage tail tokens first .. first+count-1
+                                    (counted from the tail's start); tail is
+                                    given with the batch's first piece, when
+                                    the surviving tail rows are copied, else
+                                    None;
+      ("publish",)                  the staged batch joins the index.
+    add_token() then records the step's token."""
+
+    def __init__(self, local: int, update: int, async_reindex: bool = False, pieces: int = 4,
+                 publish_lag: int = 1):
+        self.local, self.update = int(local), int(update)
+        self.async_reindex = bool(async_reindex)
+        # A batch is staged and published over pieces + lag steps while as many
+        # tokens arrive; the tail only stays bounded if that is at most `update`.
+        if self.async_reindex and self.update < 2:
+            raise ValueError("asynchronous re-indexing needs update >= 2")
+        self.lag = max(1, min(int(publish_lag), self.update - 1))
+        self.pieces = max(1, min(int(pieces), self.update - self.lag))
+        self.tail = self.local           # dense tail length
+        self.published = 0               # tokens moved from the tail into the index
+        self.reindexed = 0               # batches moved
+        self.staged_for = -1             # steps since the batch's staging began, -1: none
+        self.staged = 0                  # tokens of the batch staged so far
+
+    @property
+    def max_tail(self) -> int:
+        extra = (self.pieces - 1 + self.lag) if self.async_reindex else 0
+        return self.local + self.update + extra
+
+    @property
+    def staging(self) -> bool:
+        return self.async_reindex and self.staged_for >= 0
+
+    def before_token(self):
+        acts = []
+        u = self.update
+        if self.async_reindex:
+            if self.staged_for < 0 and self.tail >= self.local + u:
+                self.staged_for = 0                       # a batch begins
+            elif self.staged_for >= 0:
+                self.staged_for += 1
+            if self.staged_for >= 0 and self.staged_for >= self.pieces - 1 + self.lag:
+                acts.append(("publish",))
+                self.tail -= u
+                self.published += u
+                self.reindexed += 1
+                self.staged_for = -1
+                self.staged = 0
+            elif self.staged_for >= 0 and self.staged_for < self.pieces:
+                c = (u * (self.staged_for + 1)) // self.pieces - self.staged
+                acts.append(("stage", self.staged, c, self.tail if self.staged == 0 else None))
+                self.staged += c
+        elif self.tail == self.local + u:
+            acts.append(("reindex", self.tail))
+            self.tail -= u
+            self.published += u
+            self.reindexed += 1
+        return acts
+
+    def add_token(self):
+        self.tail += 1
+        if self.tail > self.max_tail:
+            raise RuntimeError("dense tail past its capacity")
+
+
 class DecodeCache:
     """K, V: the prefill [batch][H][T0][D] (bf16 or fp32, on the GPU).
     sink, local, update: the layout sizes (pages: sink 4-64, local 256-512,
@@ -68,9 +140,8 @@ class DecodeCache:
                               kv_location=PK_KV_HOST_PINNED if offload else PK_KV_DEVICE, **params)
         self.index = pk_build_index(K[:, :, sink:z].contiguous(), V[:, :, sink:z].contiguous(), z - sink, p)
         self.async_reindex = async_reindex
-        self.publish_lag = max(1, int(publish_lag))
-        self.pieces = max(1, min(int(stage_pieces), update))
-        cap = sink + local + update + ((self.pieces - 1 + self.publish_lag) if async_reindex else 0)
+        self.plan = ReindexPlan(local, update, async_reindex, stage_pieces, publish_lag)
+        cap = sink + self.plan.max_tail
         self.cap = cap
         self.dK = torch.zeros(self.batch, self.H, cap, D, dtype=K.dtype, device=K.device)
         self.dV = torch.zeros_like(self.dK)
@@ -83,12 +154,8 @@ class DecodeCache:
             self.dK2 = self.dK.clone()
             self.dV2 = self.dV.clone()
             self.side = torch.cuda.Stream(device=K.device)
-            self.staged_for = -1                          # steps since staging began, -1: none
-            self.staged = 0                               # tokens of the batch staged so far
-        self.tail = local                                 # dense tail length
         self.T = T0
-        self.zone_end = z
-        self.reindexed = 0
+        self.zone_start_end = z                           # zone end at build
         self.idx = torch.empty(self.batch * self.H, topk, dtype=torch.int32, device=K.device)
         self.out = torch.empty(self.batch, self.H * group, D, dtype=torch.float32, device=K.device)
 
@@ -97,42 +164,51 @@ class DecodeCache:
         """(start, end) positions of the retrieval zone."""
         return self.sink, self.zone_end
 
-    def _reindex(self):
+    @property
+    def zone_end(self):
+        return self.zone_start_end + self.plan.published
+
+    @property
+    def tail(self):
+        """Dense tail length."""
+        return self.plan.tail
+
+    @property
+    def reindexed(self):
+        """Batches moved from the tail into the index."""
+        return self.plan.reindexed
+
+    @property
+    def staged_for(self):
+        return self.plan.staged_for
+
+    def _reindex(self, tail):
         s, u = self.sink, self.update
         pk_append(self.index, self.dK[:, :, s:s + u].contiguous(), self.dV[:, :, s:s + u].contiguous(), u)
-        rest = self.tail - u
-        self.dK[:, :, s:s + rest] = self.dK[:, :, s + u:s + self.tail].clone()
-        self.dV[:, :, s:s + rest] = self.dV[:, :, s + u:s + self.tail].clone()
-        self.tail = rest
-        self.zone_end += u
-        self.reindexed += 1
+        rest = tail - u
+        self.dK[:, :, s:s + rest] = self.dK[:, :, s + u:s + tail].clone()
+        self.dV[:, :, s:s + rest] = self.dV[:, :, s + u:s + tail].clone()
 
-    def _stage_piece(self):
-        """Stage the next piece of the oldest `update` tail tokens on the side
-        stream, in place; with the first piece, copy the tail rows that stay
-        into the second buffer."""
+    def _stage_piece(self, first, count, tail):
+        """Stage tail tokens first .. first+count-1 on the side stream, in
+        place; with the batch's first piece (tail given), copy the tail rows
+        that stay into the second buffer."""
         s, u = self.sink, self.update
         self.side.wait_stream(torch.cuda.current_stream())   # rows written on the decode stream
-        with torch.cuda.stream(self.side):
-            if self.staged == 0:
-                rest = self.tail - u
-                self.dK2[:, :, s:s + rest].copy_(self.dK[:, :, s + u:s + self.tail])
-                self.dV2[:, :, s:s + rest].copy_(self.dV[:, :, s + u:s + self.tail])
-        c = (u * (self.staged_for + 1)) // self.pieces - self.staged
-        r0 = s + self.staged
-        pk_append_stage(self.index, self.dK[:, :, r0:], self.dV[:, :, r0:], c, self.cap, stream=self.side)
-        self.staged += c
+        if tail is not None:
+            with torch.cuda.stream(self.side):
+                rest = tail - u
+                self.dK2[:, :, s:s + rest].copy_(self.dK[:, :, s + u:s + tail])
+                self.dV2[:, :, s:s + rest].copy_(self.dV[:, :, s + u:s + tail])
+        r0 = s + first
+        pk_append_stage(self.index, self.dK[:, :, r0:], self.dV[:, :, r0:], count, self.cap, stream=self.side)
 
     def _publish(self):
-        """Make the staged tokens part of the index and drop them from the tail."""
+        """Make the staged tokens part of the index; the second buffer, which
+        holds the surviving tail, takes over."""
         pk_append_publish(self.index)                     # the decode stream waits for the staging
         self.dK, self.dK2 = self.dK2, self.dK
         self.dV, self.dV2 = self.dV2, self.dV
-        self.tail -= self.update
-        self.zone_end += self.update
-        self.reindexed += 1
-        self.staged_for = -1
-        self.staged = 0
 
     def step(self, q, k_new, v_new):
         """One decode step: add the new token k_new, v_new [batch][H][1][D] to
@@ -141,27 +217,23 @@ class DecodeCache:
         retrieved rows.  Returns the attention output [batch][H*G][D] fp32
         (a buffer reused by the next step).  Everything runs on torch's current
         stream, in order, except the asynchronous staging."""
-        if self.async_reindex:
-            if self.staged_for < 0 and self.tail >= self.local + self.update:
-                self.staged_for = 0                       # a batch begins
-            elif self.staged_for >= 0:
-                self.staged_for += 1
-            if self.staged_for >= 0 and self.staged_for >= self.pieces - 1 + self.publish_lag:
+        for act in self.plan.before_token():
+            if act[0] == "reindex":
+                self._reindex(act[1])
+            elif act[0] == "stage":
+                self._stage_piece(act[1], act[2], act[3])
+            else:
                 self._publish()
-            elif self.staged_for >= 0 and self.staged_for < self.pieces:
-                self._stage_piece()
-        elif self.tail == self.local + self.update:
-            self._reindex()
-        r = self.sink + self.tail
+        r = self.sink + self.plan.tail
         self.dK[:, :, r:r + 1] = k_new
         self.dV[:, :, r:r + 1] = v_new
-        if self.async_reindex and self.staged_for >= 0:   # also into the buffer that takes over
+        if self.plan.staging:                             # also into the buffer that takes over
             self.dK2[:, :, r - self.update:r - self.update + 1] = k_new
             self.dV2[:, :, r - self.update:r - self.update + 1] = v_new
-        self.tail += 1
+        self.plan.add_token()
         self.T += 1
         pk_search(self.index, q, self.topk, self.idx)
-        pk_attend_dense(self.index, q, self.idx, self.topk, self.dK, self.dV, self.sink + self.tail, self.out)
+        pk_attend_dense(self.index, q, self.idx, self.topk, self.dK, self.dV, self.sink + self.plan.tail, self.out)
         return self.out
 
     def close(self):
