@@ -252,6 +252,116 @@ __global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
 }
 
 // ---------------------------------------------------------------------------
+// One warp's versions of chunk_suffix and unit_threshold, so that the G units
+// of a pair run side by side, one warp each.  Lane l holds bins 4 l .. 4 l + 3;
+// the suffix over lanes is a shuffle-down scan.
+
+// inclusive suffix sum over lanes: the sum of t over lanes >= this lane
+__device__ __forceinline__ uint32_t warp_suffix_incl(uint32_t t)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t x = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(kFull, x, o);
+        if (lane + o < 32) x += y;
+    }
+    return x;
+}
+
+// inclusive prefix sum over lanes
+__device__ __forceinline__ uint32_t warp_prefix_incl(uint32_t t)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t x = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+    }
+    return x;
+}
+
+// chunk_suffix for one unit by one warp: hist[w * wstride + s] = #{S = s} of
+// warp w's keys, w < nw.
+__device__ __forceinline__ void warp_chunk_suffix(const ScanArgs &a, int unit, int chunk, const uint32_t *hist,
+                                                  int wstride, int nw)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t h[4], t = 0;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const int s = 4 * lane + k;
+        h[k] = 0u;
+        if (s < kBins)
+            for (int w = 0; w < nw; w++) h[k] += hist[w * wstride + s];
+        t += h[k];
+    }
+    uint32_t c = warp_suffix_incl(t) - t;        // #{S >= 4 lane + 4}
+    uint32_t *out = a.chunk_cum + ((size_t)unit * a.max_chunks + chunk) * kCum;
+#pragma unroll
+    for (int k = 3; k >= 0; k--) {
+        const int s = 4 * lane + k;
+        c += h[k];
+        if (s < kCum) out[s] = c;
+        if (s < kBins && h[k]) atomicAdd(&a.head_hist[(size_t)unit * kBins + s], h[k]);
+    }
+}
+
+// unit_threshold for one unit by one warp
+__device__ __forceinline__ void warp_unit_threshold(const ScanArgs &a, int unit)
+{
+    const int lane = threadIdx.x & 31;
+    uint32_t h[4], t = 0;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const int s = 4 * lane + k;
+        h[k] = (s < kBins) ? __ldcg(&a.head_hist[(size_t)unit * kBins + s]) : 0u;
+        if (a.dbg_hist && s < kBins) a.dbg_hist[(size_t)unit * kBins + s] = h[k];
+        t += h[k];
+    }
+    uint32_t cum[4];
+    {
+        uint32_t c = warp_suffix_incl(t) - t;
+#pragma unroll
+        for (int k = 3; k >= 0; k--) { c += h[k]; cum[k] = c; }
+    }
+    // s* = largest s with #{S >= s} >= C: the number of such s, less one
+    int nsat = 0;
+#pragma unroll
+    for (int k = 0; k < 4; k++) nsat += (4 * lane + k < kCum) && ((int64_t)cum[k] >= a.C);
+    const int sstar = __reduce_add_sync(kFull, (unsigned)nsat) - 1;
+    if (lane == 0) {
+        a.sstar[unit] = sstar;
+        if (a.dbg_sstar) a.dbg_sstar[unit] = sstar;
+    }
+    // gt_total = #{S > s*} = cum[s* + 1], from the lane that holds bin s* + 1
+    const int s1 = sstar + 1, k1 = s1 & 3;
+    const uint32_t mine = k1 == 0 ? cum[0] : k1 == 1 ? cum[1] : k1 == 2 ? cum[2] : cum[3];
+    const uint32_t gt_total = __shfl_sync(kFull, mine, s1 >> 2);
+    const int64_t ties = a.C - (int64_t)gt_total;
+    uint32_t carry_eq = 0, carry_slot = 0;
+    for (int j0 = 0; j0 < a.nchunks; j0 += 32) {
+        const int j = j0 + lane;
+        uint32_t gt = 0, eq = 0;
+        if (j < a.nchunks) {
+            const uint32_t *cj = a.chunk_cum + ((size_t)unit * a.max_chunks + j) * kCum;
+            const uint32_t c0 = __ldcg(cj + sstar), c1 = __ldcg(cj + sstar + 1);
+            gt = c1;
+            eq = c0 - c1;
+        }
+        const uint32_t in_eq = warp_prefix_incl(eq);
+        const int64_t room = ties - (int64_t)(carry_eq + in_eq - eq);
+        const uint32_t quota = room <= 0 ? 0u : (room >= (int64_t)eq ? eq : (uint32_t)room);
+        const uint32_t in_slot = warp_prefix_incl(gt + quota);
+        if (j < a.nchunks)
+            a.chunk_info[(size_t)unit * a.max_chunks + j] = make_uint2(carry_slot + in_slot - (gt + quota), quota);
+        carry_eq += __shfl_sync(kFull, in_eq, 31);
+        carry_slot += __shfl_sync(kFull, in_slot, 31);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Per-query-head retrieval: one pass over a pair's codes scores it for all G
 // query heads of the pair (units pair G + g).  The G bonus tables are packed
 // into one table per (block, centre) in shared memory -- NP words, byte g of
@@ -259,9 +369,10 @@ __global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan(ScanArgs a)
 // bonuses of every head, and summing the 16 words of a key gives every head's
 // S in its own byte (S <= 96: no carry between bytes).  Then each head's S,
 // histogram, suffix counts and threshold go through the same steps as the
-// single-query scan.
+// single-query scan, one warp per head.  The prep writes the packed table
+// ([pairs][16][256][NP] words), so the CTA loads it with 16-byte loads.
 template <int NP>
-__global__ void __launch_bounds__(kScanThreads) k_collision_scan_heads(ScanArgs a)
+__global__ void __launch_bounds__(kScanThreads, 4) k_collision_scan_heads(ScanArgs a)
 {
     const int pair = blockIdx.y, chunk = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -271,21 +382,19 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan_heads(ScanArgs 
     extern __shared__ __align__(16) uint32_t s_dyn[];
     uint32_t *ptab = s_dyn;                       // [kB * kNC][NP]
     uint32_t *s_hist = s_dyn + kB * kNC * NP;     // [NW][G][kHistPad]
-    __shared__ uint32_t s_cum[kHistPad];
-    __shared__ uint32_t s_ws[NW + 1];
     __shared__ int s_last;
-    __shared__ uint32_t s_gt_total;
 
     for (int i = tid; i < NW * G * kHistPad; i += kScanThreads) s_hist[i] = 0u;
     pdl_wait();                                   // bonus tables come from the query preparation
-    for (int e = tid; e < kB * kNC; e += kScanThreads) {
-        uint32_t w[NP];
+    {   // the pair's packed table, written so by the query preparation
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.bonus_bytes + (size_t)pair * kB * kNC * 4 * NP);
+        uint4 *dst = reinterpret_cast<uint4 *>(ptab);
+        constexpr int kVec = kB * kNC * NP / 4;
+        uint4 v[kVec / kScanThreads];
 #pragma unroll
-        for (int p = 0; p < NP; p++) w[p] = 0u;
-        for (int g = 0; g < G; g++)
-            w[g >> 2] |= (uint32_t)a.bonus_bytes[(size_t)(u0 + g) * kB * kNC + e] << (8 * (g & 3));
+        for (int u = 0; u < kVec / kScanThreads; u++) v[u] = __ldcg(src + tid + u * kScanThreads);
 #pragma unroll
-        for (int p = 0; p < NP; p++) ptab[e * NP + p] = w[p];
+        for (int u = 0; u < kVec / kScanThreads; u++) dst[tid + u * kScanThreads] = v[u];
     }
     __syncthreads();
 
@@ -295,15 +404,21 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan_heads(ScanArgs 
     const uint4 *codes = reinterpret_cast<const uint4 *>(a.codes + ((size_t)pair * a.n_cap + lo) * kB);
     uint8_t *S0 = a.S + (size_t)u0 * a.n_cap + lo;
     uint32_t *hw = s_hist + warp * G * kHistPad;
-    constexpr int U = 2;                          // keys per lane per iteration
+    constexpr int U = kScanUnroll;                // keys per lane per iteration
     const uint32_t step = (uint32_t)NW * 32 * U;
-    for (uint32_t base = (uint32_t)warp * 32 * U + lane; base < ucnt + lane; base += step) {
-        uint4 c[U];
+    // the next iteration's codes load while this one is scored
+    auto load = [&](uint32_t b, uint4 (&c)[U]) {
 #pragma unroll
         for (int u = 0; u < U; u++) {
-            const uint32_t i = base + u * 32;
+            const uint32_t i = b + u * 32;
             c[u] = (i < ucnt) ? __ldcs(codes + i) : make_uint4(0, 0, 0, 0);
         }
+    };
+    uint4 c[U], cn[U];
+    uint32_t base = (uint32_t)warp * 32 * U + lane;
+    if (base < ucnt + lane) load(base, c);
+    for (; base < ucnt + lane; base += step) {
+        if (base + step < ucnt + lane) load(base + step, cn);
 #pragma unroll
         for (int u = 0; u < U; u++) {
             const uint32_t i = base + u * 32;
@@ -333,15 +448,12 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan_heads(ScanArgs 
                 }
             }
         }
+#pragma unroll
+        for (int u = 0; u < U; u++) c[u] = cn[u];
     }
     __syncthreads();
 
-    for (int g = 0; g < G; g++) {
-        uint32_t hv = 0;
-        if (tid < kBins)
-            for (int w = 0; w < NW; w++) hv += s_hist[(w * G + g) * kHistPad + tid];
-        chunk_suffix(a, u0 + g, chunk, hv, s_cum, s_ws);
-    }
+    for (int g = warp; g < G; g += NW) warp_chunk_suffix(a, u0 + g, chunk, s_hist + g * kHistPad, G * kHistPad, NW);
     __threadfence();
     __syncthreads();
     pdl_trigger();
@@ -349,7 +461,7 @@ __global__ void __launch_bounds__(kScanThreads) k_collision_scan_heads(ScanArgs 
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int g = 0; g < G; g++) unit_threshold(a, u0 + g, s_ws, &s_last, &s_gt_total);
+    for (int g = warp; g < G; g += NW) warp_unit_threshold(a, u0 + g);
     if (tid == 0) a.tickets[(size_t)u0 * 2 + 0] = 0u;
 }
 

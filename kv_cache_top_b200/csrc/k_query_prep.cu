@@ -53,6 +53,14 @@ __device__ __forceinline__ void load_heads(float (&qv)[4][kMaxGroup], const T *q
         }
 }
 
+// per-query-head search: where unit bh's bonus of centre c of block b goes
+// in its pair's packed table (byte g of the entry, g = bh % kvg)
+__device__ __forceinline__ uint8_t *head_bonus_ptr(const PrepArgs &a, int bh, int b, int c)
+{
+    const int pair = bh / a.kvg, g = bh - pair * a.kvg;
+    return a.bonus_heads + (((size_t)pair * kB + b) * kNC + c) * (4 * a.heads_np) + 4 * (g >> 2) + (g & 3);
+}
+
 __device__ __forceinline__ uint32_t tier_bonus(uint32_t P, unsigned long long R)
 {
     // 6 - floor(6P/R) for P < R, else 0: floor(6P/R) = #{j = 1..5 : 6P >= jR},
@@ -228,6 +236,7 @@ __global__ void __launch_bounds__(kQpThreads) k_query_prep(PrepArgs a)
         const uint8_t bon = (uint8_t)tier_bonus(pre[i], R);
         s_bonus[warp][c] = bon;
         if (db) db[c] = bon;
+        if (a.bonus_heads) *head_bonus_ptr(a, bh, b, (int)c) = bon;
     }
     __syncwarp();
     uint32_t word = 0;
@@ -366,6 +375,10 @@ __global__ void __launch_bounds__(kQwThreads) k_query_prep_wide(PrepArgs a)
         uint8_t *db = a.dbg_bonus + ((size_t)bh * kB + b) * kNC;
         db[c0] = (uint8_t)bon0;
         db[c1] = (uint8_t)bon1;
+    }
+    if (a.bonus_heads) {
+        *head_bonus_ptr(a, bh, b, c0) = (uint8_t)bon0;
+        *head_bonus_ptr(a, bh, b, c1) = (uint8_t)bon1;
     }
     __syncthreads();
     if (t < 32) {                              // first warp of each half

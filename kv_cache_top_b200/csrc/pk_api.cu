@@ -21,7 +21,7 @@ struct Work {
     int32_t units = 0;
     int32_t scan_units = 0;      // CTAs' worth of work units per chunk of the scan: units, or pairs
                                  // when one scan pass serves the G query heads of a pair
-    uint8_t *bonus_bytes = nullptr;   // [units][16][256] bonus per centre (per-head search)
+    uint8_t *bonus_bytes = nullptr;   // [pairs][16][256][np] u32: the kvg heads' bonuses packed per pair (per-head search)
     int32_t max_chunks = 1, max_slices = 1;
     float *qt = nullptr, *qnorm = nullptr;
     uint32_t *bonus_packed = nullptr;
@@ -241,7 +241,11 @@ cudaError_t work_alloc(pk_index *ix, Work &w, int32_t units, int32_t kvg, int64_
     chk(dalloc(&w.sstar, U));
     chk(dalloc(&w.cand, U * NC));
     chk(dalloc(&w.partial, U * MS * (size_t)ix->topk_cap));
-    if (kvg > 1) chk(dalloc(&w.bonus_bytes, U * kB * kNC));
+    if (kvg > 1) {   // the per-pair packed bonus tables of per-head search, unused bytes zero
+        const size_t bytes = (size_t)(U / kvg) * kB * kNC * 4 * ((kvg + 3) / 4);
+        chk(dalloc(&w.bonus_bytes, bytes));
+        chk(cudaMemsetAsync(w.bonus_bytes, 0, bytes, s));
+    }
     chk(cudaMemsetAsync(w.head_hist, 0, U * kBins * sizeof(uint32_t), s));
     chk(cudaMemsetAsync(w.tickets, 0, U * 2 * sizeof(uint32_t), s));
     if (e != cudaSuccess) {
@@ -417,7 +421,10 @@ pk_status search_impl(pk_index *ix, Work &w, int32_t kvg, const void *q, int32_t
         pa.dbg_qt = dbg->qt;
         pa.dbg_qnorm = dbg->qnorm;
     }
-    if (kvg > 1) pa.dbg_bonus = w.bonus_bytes;   // the per-head scan reads the bonus bytes
+    if (kvg > 1) {   // the per-head scan reads the pairs' packed bonus tables
+        pa.bonus_heads = w.bonus_bytes;
+        pa.heads_np = (kvg + 3) / 4;
+    }
     trace_begin(ix, PK_K_QUERY_PREP, s);
     cudaError_t e = launch_query_prep(pa, s);
     trace_end(ix, s);

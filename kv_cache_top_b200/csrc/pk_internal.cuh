@@ -76,6 +76,11 @@ struct PrepArgs {
     uint32_t *head_hist;     // [BH][kBins]   zeroed here
     uint32_t *tickets;       // [BH][2]       zeroed here
     uint8_t *dbg_bonus;      // [BH][16][256] or null
+    // per-query-head search (kvg query units per pair): every unit's bonus
+    // also goes to byte (g & 3) of word (g >> 2) of entry (pair, block,
+    // centre) of a per-pair table [pairs][16][256][heads_np] u32, g = unit % kvg
+    uint8_t *bonus_heads;
+    int32_t heads_np;
     float *dbg_qt;
     float *dbg_qnorm;
 };
@@ -83,7 +88,7 @@ struct PrepArgs {
 struct ScanArgs {
     const uint8_t *codes;
     const uint32_t *bonus_packed;
-    const uint8_t *bonus_bytes;   // [units][16][256] (one pass for the kvg query heads of a pair)
+    const uint8_t *bonus_bytes;   // [pairs][16][256][np] u32 packed bonuses of the kvg query heads of a pair
     int64_t n, n_cap, chunk, C;   // n_cap: row stride of the per-key arrays
     int32_t nchunks;
     int32_t kvg;             // query units per index pair
