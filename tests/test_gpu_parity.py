@@ -366,7 +366,11 @@ def test_decode_cache_sink_local_update(pk, offload, async_reindex):
         cache.close()
 
 
-@pytest.mark.parametrize("batch,H,G,n,kv_location", [(1, 2, 4, 20000, 0), (2, 1, 2, 9000, 1)])
+@pytest.mark.parametrize("batch,H,G,n,kv_location", [
+    (1, 2, 4, 20000, 0), (2, 1, 2, 9000, 1),
+    (1, 1, 6, 40000, 0),     # two packed bonus words per centre, the second half full; 40 key chunks
+    (1, 1, 8, 5000, 1),      # the largest group: both words full
+])
 def test_per_query_head_search(pk, batch, H, G, n, kv_location):
     """pk_search_heads / pk_attend_heads: each query head searches its pair's
     index with its own query (the oracle's search with G = 1 on that head),
