@@ -778,12 +778,14 @@ def run_heads(args, wl):
     idx_a = torch.empty(BH, 100, dtype=torch.int32, device=dev)
     idx_h = torch.empty(U, 100, dtype=torch.int32, device=dev)
     out = torch.empty(B, H * G, 128, dtype=torch.float32, device=dev)
-    rec_a, rec_h = [], []
+    rec_a, rec_h, union_rows = [], [], []
     for qi in range(nq):
         q = w["q"][qi]
         pk.pk_search(h, q, 100, idx_a)
         pk.pk_search_heads(h, q, 100, idx_h)
         ga, gh = idx_a.cpu(), idx_h.cpu()
+        # rows the per-head attention gathers per pair: the union of its G lists
+        union_rows += [len(set(gh[p * G:(p + 1) * G].flatten().tolist())) for p in range(BH)]
         qs = q.float().view(B, H, G, 128)
         for b in range(B):
             for hh in range(H):
@@ -835,7 +837,8 @@ def run_heads(args, wl):
         "aggregated": {"recall_at_100": sum(rec_a) / len(rec_a), "ms_per_step": ms_a,
                        "steps_s": 1000.0 / ms_a, "kernel_us": kern_a},
         "per_head": {"recall_at_100": sum(rec_h) / len(rec_h), "ms_per_step": ms_h, "steps_s": 1000.0 / ms_h,
-                     "kernel_us": kern_h},
+                     "kernel_us": kern_h,
+                     "attend_rows_per_pair": {"union": sum(union_rows) / len(union_rows), "lists": G * 100}},
         "data": "synthetic", "dtype": "f32",
         "config": {"workload": wl["name"], "batch": B, "n": n, "kv_heads": H, "q_heads": H * G, "topk": 100,
                    "queries": nq, "l2": "flushed between steps (outside the events)"}}), flush=True)

@@ -236,7 +236,14 @@ pk_status pk_search_heads(pk_index *index, const void *q, int32_t topk, int32_t 
 
 /* Attention of every query head over its own selected rows (as returned by
  * pk_search_heads): sel_idx [batch][H*G][topk] i32 device; out as for
- * pk_attend.  Errors as pk_attend. */
+ * pk_attend.  With K/V in pinned host memory and G x topk <= 1024, the rows
+ * of a (sequence, KV head) pair cross the host link once: the union of its G
+ * heads' lists, in order of first appearance, each id once; head g then
+ * attends over the rows of its own list.  With K/V in HBM, or longer lists,
+ * each query head's rows are gathered by its own CTAs.  A head's ids are
+ * expected to be distinct (pk_search_heads' are): a repeated id counts once
+ * on the union path and once per appearance on the per-head path.  Errors as
+ * pk_attend. */
 pk_status pk_attend_heads(pk_index *index, const void *q, const int32_t *sel_idx, int32_t topk,
                           float *out, void *stream);
 

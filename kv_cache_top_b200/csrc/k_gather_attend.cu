@@ -23,6 +23,16 @@
 // is arrived at on entry, so the pushes know every CTA of the cluster runs.
 // Ids outside [0, n) are skipped and recorded in the device-check word (no
 // trap).
+//
+// Per-query-head rows (union_heads): each query head of the pair has its own
+// list, and one cluster serves all G heads.  In the prologue every CTA puts
+// the pair's G x topk ids into the same open-addressing table in shared
+// memory (over the not yet used K/V tiles): key = id + 1, with the mask of
+// heads whose list holds it and the smallest entry index e = g topk + r that
+// holds it.  Entry e is a row iff it is that smallest index, so the rows are
+// the union of the lists in order of first appearance: the same on every CTA,
+// each id once, whatever order the inserts ran in.  Each row is fetched once; head g
+// scores it only if its mask holds g (others see -inf, weight 0).
 #include <cooperative_groups.h>
 
 #include "pk_internal.cuh"
@@ -45,8 +55,25 @@ __device__ __forceinline__ void cluster_arrive_relaxed() { asm volatile("barrier
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
-// size of the partials region (dynamic shared memory): [nsplit][G][kD] fp32
-size_t attend_smem(int nsplit, int G) { return (size_t)nsplit * G * kD * sizeof(float); }
+// dynamic shared memory: the partials [nsplit][G][kD] fp32, then (union
+// rows only) the row list [G x topk] of (head mask << 32 | id)
+size_t attend_smem(int nsplit, int G, int union_entries)
+{
+    return (size_t)nsplit * G * kD * sizeof(float) + (size_t)union_entries * sizeof(unsigned long long);
+}
+
+// open-addressing slots for E union entries: a power of two >= 2E
+__host__ __device__ inline int union_slots(int E)
+{
+    int h = 64;
+    while (h < 2 * E) h <<= 1;
+    return h;
+}
+
+__device__ __forceinline__ uint32_t union_hash(uint32_t key)
+{
+    return key * 0x9E3779B1u;     // Fibonacci hashing; the slot index takes the high bits
+}
 
 __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
 {
@@ -55,6 +82,8 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
     unsigned char *sK = s_kv;
     unsigned char *sV = s_kv + kAtRows * kD * 4;
     __shared__ int32_t s_idx[kAtRows];
+    __shared__ uint32_t s_msk[kAtRows];            // heads that score the row (union rows)
+    __shared__ uint32_t s_ws[kAtThreads / 32 + 1];
     __shared__ __align__(16) float s_q[kMaxGroup][kQPad];
     __shared__ float s_p[kMaxGroup][kAtRows];
     __shared__ float s_m[kMaxGroup], s_l[kMaxGroup], s_alpha[kMaxGroup];
@@ -73,20 +102,81 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
     const int es = a.is_bf16 ? 2 : 4;
     const int row_bytes = kD * es;
     const int vpr = row_bytes / 16;
-    // the pair's rows: the topk selected ids, then the dlen dense rows
-    const int nrows = a.topk + a.dlen;
-    const int per = (nrows + nsp - 1) / nsp;
-    const int r_beg = min(nrows, sp * per), r_end = min(nrows, r_beg + per);
-
     const int64_t qbase = ((int64_t)b_seq * a.H * G + (int64_t)h * G) * kD;
     if (tid < G) {
         s_m[tid] = -INFINITY;
         s_l[tid] = 0.0f;
     }
+    unsigned long long *s_rows = reinterpret_cast<unsigned long long *>(s_pacc + (size_t)nsp * G * kD);
     pdl_wait();                                   // the selected ids may come from the search
+    // the pair's rows: the topk selected ids (or the union of the G heads'
+    // lists), then the dlen dense rows
+    int nsel = a.topk;
+    if (a.union_heads) {
+        const int E = G * a.topk, HS = union_slots(E);
+        const int32_t *ids = a.idx + (size_t)bh * E;
+        // keys, head masks, first entries: 12 HS bytes <= the K/V tiles (HS <= 2048)
+        uint32_t *hk = reinterpret_cast<uint32_t *>(s_kv), *hm = hk + HS, *hf = hm + HS;
+        for (int i = tid; i < HS; i += kAtThreads) {
+            hk[i] = hm[i] = 0u;
+            hf[i] = 0xffffffffu;
+        }
+        __syncthreads();
+        const int sh = 32 - (31 - __clz(HS));         // slot = high log2(HS) bits of the hash
+        // insert (e >= 0): claim or find the key's slot, add head e / topk and entry e;
+        // look up (e < 0): the key's slot or -1.  At most HS probes; E < HS keys.
+        auto slot_of = [&](uint32_t key, int e) -> int {
+            uint32_t p = union_hash(key) >> sh;
+            for (int t = 0; t < HS; t++, p = (p + 1) & (HS - 1)) {
+                const uint32_t cur = e >= 0 ? atomicCAS(&hk[p], 0u, key) : hk[p];
+                if (cur == key || (e >= 0 && cur == 0u)) {
+                    if (e >= 0) {
+                        atomicOr(&hm[p], 1u << (e / a.topk));
+                        atomicMin(&hf[p], (uint32_t)e);
+                    }
+                    return (int)p;
+                }
+                if (cur == 0u) return -1;
+            }
+            return -1;
+        };
+        for (int e = tid; e < E; e += kAtThreads) {
+            const int32_t id = ids[e];
+            if (id >= 0 && (int64_t)id < a.n) slot_of((uint32_t)id + 1u, e);
+            else devchk(a.dev_err, a.dev_err_detail, DEVCHK_BAD_INDEX, id);
+        }
+        __syncthreads();
+        // rows in entry order: thread t takes entries [t * per_t, ...) so the scan keeps that order
+        const int per_t = (E + kAtThreads - 1) / kAtThreads;
+        const int e0 = tid * per_t, e1 = min(E, e0 + per_t);
+        uint32_t cnt = 0;
+        for (int e = e0; e < e1; e++) {
+            const int32_t id = ids[e];
+            if (id >= 0 && (int64_t)id < a.n) {
+                const int p = slot_of((uint32_t)id + 1u, -1);
+                cnt += (p >= 0 && hf[p] == (uint32_t)e);
+            }
+        }
+        uint32_t tot;
+        uint32_t pos = block_excl_scan<kAtThreads>(cnt, s_ws, &tot);
+        for (int e = e0; e < e1; e++) {
+            const int32_t id = ids[e];
+            if (id >= 0 && (int64_t)id < a.n) {
+                const int p = slot_of((uint32_t)id + 1u, -1);
+                if (p >= 0 && hf[p] == (uint32_t)e)
+                    s_rows[pos++] = ((unsigned long long)hm[p] << 32) | (uint32_t)id;
+            }
+        }
+        nsel = (int)tot;
+        __syncthreads();                          // rows written; the table's storage goes back to the tiles
+    }
+    const int nrows = nsel + a.dlen;
+    const int per = (nrows + nsp - 1) / nsp;
+    const int r_beg = min(nrows, sp * per), r_end = min(nrows, r_beg + per);
     // the first tile's selected ids and the query heads load together (one round trip)
     const int rr0 = r_beg + tid;
-    const int32_t id0 = (tid < kAtRows && rr0 < r_end && rr0 < a.topk) ? a.idx[(size_t)bh * a.topk + rr0] : 0;
+    const int32_t id0 = (tid < kAtRows && rr0 < r_end && rr0 < nsel && !a.union_heads)
+        ? a.idx[(size_t)bh * a.topk + rr0] : 0;
     for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][qpad(i % kD)] = ld_as_f32(a.q, qbase + i, a.is_bf16);
     const size_t kp = (size_t)index_pair(bh, a.kvg);     // the index pair holding this unit's rows
     const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + kp * a.stride * a.kv_pitch;
@@ -106,13 +196,19 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
         // or -2 - j for dense row j
         if (tid < rows) {
             const int rr = t0 + tid;
-            if (rr < a.topk) {
+            if (rr < nsel && a.union_heads) {     // checked and deduplicated in the prologue
+                const unsigned long long rw = s_rows[rr];
+                s_idx[tid] = (int32_t)(uint32_t)rw;
+                s_msk[tid] = (uint32_t)(rw >> 32);
+            } else if (rr < nsel) {
                 const int32_t id = t0 == r_beg ? id0 : a.idx[(size_t)bh * a.topk + rr];
                 const bool ok = id >= 0 && (int64_t)id < a.n;
                 if (!ok) devchk(a.dev_err, a.dev_err_detail, DEVCHK_BAD_INDEX, id);
                 s_idx[tid] = ok ? id : -1;
+                s_msk[tid] = ~0u;
             } else {
-                s_idx[tid] = -2 - (rr - a.topk);
+                s_idx[tid] = -2 - (rr - nsel);
+                s_msk[tid] = ~0u;
             }
         }
         __syncthreads();
@@ -201,7 +297,8 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
                     sc[g] += __shfl_xor_sync(kFull, sc[g], 1);
                     sc[g] += __shfl_xor_sync(kFull, sc[g], 2);
                     sc[g] += __shfl_xor_sync(kFull, sc[g], 4);
-                    if (j == 0 && r < rows) s_p[g][r] = (s_idx[r] != -1) ? sc[g] * a.scale : -INFINITY;
+                    if (j == 0 && r < rows)
+                        s_p[g][r] = (s_idx[r] != -1 && ((s_msk[r] >> g) & 1u)) ? sc[g] * a.scale : -INFINITY;
                 }
             }
         }
@@ -296,12 +393,12 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
 cudaError_t launch_gather_attend(const AttendArgs &a, int bh, cudaStream_t s)
 {
     static std::atomic<int> smem_set[kMaxDevices];   // the partials region may pass 48 KB in total
-    const cudaError_t e = dyn_smem_limit(k_gather_attend, (int)attend_smem(8, kMaxGroup), smem_set);
+    const cudaError_t e = dyn_smem_limit(k_gather_attend, (int)attend_smem(8, kMaxGroup, kUnionMax), smem_set);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.nsplit, bh, 1);
     cfg.blockDim = dim3(kAtThreads, 1, 1);
-    cfg.dynamicSmemBytes = attend_smem(a.nsplit, a.G);
+    cfg.dynamicSmemBytes = attend_smem(a.nsplit, a.G, a.union_heads ? a.G * a.topk : 0);
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;

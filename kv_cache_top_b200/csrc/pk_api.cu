@@ -522,8 +522,11 @@ pk_status search_impl(pk_index *ix, Work &w, int32_t kvg, const void *q, int32_t
 
 // Attention for kvg query units per index pair (1: each pair's G query heads
 // over the pair's selected rows; G: each query head over its own rows).
+// union_heads (kvg = 1): sel_idx holds each query head's own list, and one
+// cluster per pair gathers the union of the pair's lists once.
 pk_status attend_impl(pk_index *ix, int32_t kvg, const void *q, const int32_t *sel_idx, int32_t topk,
-                      const void *dK, const void *dV, int64_t dstride, int32_t dlen, float *out, cudaStream_t s)
+                      const void *dK, const void *dV, int64_t dstride, int32_t dlen, float *out, cudaStream_t s,
+                      bool union_heads = false)
 {
     if (!ix || !q || !out) return PK_ERR_INVALID_ARG;
     if (topk < 0 || topk > ix->topk_cap || dlen < 0 || topk + (int64_t)dlen < 1) return PK_ERR_INVALID_ARG;
@@ -554,8 +557,9 @@ pk_status attend_impl(pk_index *ix, int32_t kvg, const void *q, const int32_t *s
     a.topk = topk;
     a.is_bf16 = ix->p.kv_dtype == PK_BF16;
     a.scale = ix->scale;
+    a.union_heads = union_heads ? 1 : 0;
     const int32_t units = ix->bh * kvg;
-    a.nsplit = splitting(ix, units, topk + dlen);
+    a.nsplit = splitting(ix, units, (union_heads ? a.G * topk : topk) + dlen);
     a.dev_err = ix->dev_err;
     a.dev_err_detail = ix->dev_err_detail;
     trace_begin(ix, PK_K_GATHER_ATTEND, s);
@@ -815,6 +819,11 @@ pk_status pk_attend_heads(pk_index *ix, const void *q, const int32_t *sel_idx, i
 {
     if (!ix) return PK_ERR_INVALID_ARG;
     if (topk < 1) return PK_ERR_INVALID_ARG;
+    // K/V in host memory: every row of a pair crosses the host link once (the
+    // union of its heads' lists) when the lists fit the kernel's table.  K/V in
+    // HBM, or longer lists: one cluster per query head (more CTAs in flight).
+    if (ix->p.kv_location == PK_KV_HOST_PINNED && (int64_t)ix->p.group * topk <= kUnionMax)
+        return attend_impl(ix, 1, q, sel_idx, topk, nullptr, nullptr, 0, 0, out, (cudaStream_t)stream, true);
     return attend_impl(ix, ix->p.group, q, sel_idx, topk, nullptr, nullptr, 0, 0, out, (cudaStream_t)stream);
 }
 

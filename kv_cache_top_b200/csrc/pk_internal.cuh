@@ -149,7 +149,12 @@ struct AttendArgs {
     const void *dK, *dV;
     int64_t dstride;
     int32_t dlen;
+    // per-query-head rows, gathered once per pair: idx is [BH][G][topk]
+    // (each query head's own list), the CTA's rows are the union of the G
+    // lists, and head g's softmax runs over its own rows only
+    int32_t union_heads;
 };
+constexpr int kUnionMax = 1024;   // G x topk entries a union-gather attention accepts
 
 struct MergeArgs {
     const unsigned long long *partial;

@@ -405,6 +405,54 @@ def test_per_query_head_search(pk, batch, H, G, n, kv_location):
         pk.pk_free(h)
 
 
+@pytest.mark.parametrize("G,topk,kv_location", [
+    (4, 100, 1), (8, 100, 1),      # K/V in host memory: the union gather
+    (4, 100, 0),                   # K/V in HBM: one cluster per query head
+    (8, 200, 1),                   # lists past the union table: one cluster per query head
+])
+def test_attend_heads_union_of_lists(pk, G, topk, kv_location):
+    """pk_attend_heads on hand-made per-head lists: heavy overlap between the
+    heads of a pair, one head's list equal to another's, an id repeated
+    inside one list (union path only) and an out-of-range id.  Each head's
+    output is the oracle's attention over the distinct valid ids of its own
+    list."""
+    batch, H, n = 1, 2, 5000
+    w = workloads.llama_layer(batch, n, H=H, G=G, seed=17, device="cuda")
+    q = w["q"][0]
+    h = build(pk, w["K"], w["V"], n, batch, H, G, topk=topk, kv_location=kv_location)
+    try:
+        rng = np.random.default_rng(5)
+        U = batch * H * G
+        sel = np.empty((U, topk), np.int32)
+        for pair in range(batch * H):
+            pool = rng.choice(n, size=int(1.5 * topk), replace=False).astype(np.int32)
+            for g in range(G):
+                sel[pair * G + g] = rng.choice(pool, size=topk, replace=False)
+            sel[pair * G + 1] = sel[pair * G + 0]           # two heads with the same list
+            if kv_location == 1 and G * topk <= 1024:        # the union path takes a list as a set
+                sel[pair * G + 2, -1] = sel[pair * G + 2, 0]    # an id twice in one list
+        bad = n + 3
+        sel[G + 3, 5] = bad                                  # out of range: skipped and recorded
+        sel_t = torch.from_numpy(sel).cuda()
+        out = torch.full((batch, H * G, 128), float("nan"), dtype=torch.float32, device="cuda")
+        pk.pk_attend_heads(h, q, sel_t, topk, out)
+        torch.cuda.synchronize()
+        st, det = pk.pk_last_device_error(h)
+        assert st == 6 and det == bad, (st, det)
+        o = out.cpu().numpy()
+        for u in range(U):
+            b, j = divmod(u, H * G)
+            hh = j // G
+            K_np = workloads.to_np_f32(w["K"][b, hh, :n])
+            V_np = workloads.to_np_f32(w["V"][b, hh, :n])
+            qh = workloads.to_np_f32(q[b, j:j + 1])
+            ids = np.unique(sel[u][(sel[u] >= 0) & (sel[u] < n)])
+            ref = parity.oracle.attend(qh, K_np, V_np, ids, 1.0 / math.sqrt(128))
+            parity.check_attention(o[b, j:j + 1], ref)
+    finally:
+        pk.pk_free(h)
+
+
 def test_host_pinned_kv_store(pk):
     """K/V kept in pinned host memory and read through UVA by the attention."""
     w = workloads.llama_layer(1, 20000, H=2, G=4, seed=3, device="cuda")
