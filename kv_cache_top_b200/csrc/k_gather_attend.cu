@@ -177,7 +177,29 @@ __global__ void __launch_bounds__(kAtThreads, 3) k_gather_attend(AttendArgs a)
     const int rr0 = r_beg + tid;
     const int32_t id0 = (tid < kAtRows && rr0 < r_end && rr0 < nsel && !a.union_heads)
         ? a.idx[(size_t)bh * a.topk + rr0] : 0;
-    for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][qpad(i % kD)] = ld_as_f32(a.q, qbase + i, a.is_bf16);
+    {   // the query heads: 16-byte loads when the rows start on a 16-byte boundary
+        const uintptr_t at = reinterpret_cast<uintptr_t>(a.q) + (uintptr_t)qbase * (uintptr_t)es;
+        if ((at & 15u) == 0 && a.is_bf16) {
+            for (int v = tid; v < G * kD / 8; v += kAtThreads) {
+                const uint4 x = reinterpret_cast<const uint4 *>(at)[v];
+                const int g = v / (kD / 8), d0 = 8 * (v % (kD / 8));   // 8 elements in one 32-group
+                const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.x));
+                const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.y));
+                const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.z));
+                const float2 f3 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.w));
+                float4 *dst = reinterpret_cast<float4 *>(&s_q[g][qpad(d0)]);
+                dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+                dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+            }
+        } else if ((at & 15u) == 0) {
+            for (int v = tid; v < G * kD / 4; v += kAtThreads) {
+                const int g = v / (kD / 4), d0 = 4 * (v % (kD / 4));
+                *reinterpret_cast<float4 *>(&s_q[g][qpad(d0)]) = reinterpret_cast<const float4 *>(at)[v];
+            }
+        } else {
+            for (int i = tid; i < G * kD; i += kAtThreads) s_q[i / kD][qpad(i % kD)] = ld_as_f32(a.q, qbase + i, a.is_bf16);
+        }
+    }
     const size_t kp = (size_t)index_pair(bh, a.kvg);     // the index pair holding this unit's rows
     const unsigned char *Kb = reinterpret_cast<const unsigned char *>(a.K) + kp * a.stride * a.kv_pitch;
     const unsigned char *Vb = reinterpret_cast<const unsigned char *>(a.V) + kp * a.stride * a.kv_pitch;

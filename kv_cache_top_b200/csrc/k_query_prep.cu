@@ -53,6 +53,51 @@ __device__ __forceinline__ void load_heads(float (&qv)[4][kMaxGroup], const T *q
         }
 }
 
+// The G query heads of a unit (rows of kD at q + base): qv[r][g] = q_g[lane + 32 r].
+// When the rows start on a 16-byte boundary the warp reads them with 16-byte
+// loads into `stage` ([kMaxGroup][kD] fp32, shared) and picks its elements
+// from there: one request per 16 bytes, which matters when q sits in host
+// memory.  Otherwise one element per load.  The values are the same either way.
+__device__ __forceinline__ void load_query(float (&qv)[4][kMaxGroup], const PrepArgs &a, int64_t base, int lane,
+                                           float *stage)
+{
+    const int G = a.G;
+    const uintptr_t at = reinterpret_cast<uintptr_t>(a.q) + (uintptr_t)base * (a.is_bf16 ? 2u : 4u);
+    if ((at & 15u) != 0) {
+        if (a.is_bf16)
+            load_heads(qv, reinterpret_cast<const __nv_bfloat16 *>(a.q) + base, G, lane);
+        else
+            load_heads(qv, reinterpret_cast<const float *>(a.q) + base, G, lane);
+        return;
+    }
+    if (a.is_bf16) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(at);
+        for (int v = lane; v < G * kD / 8; v += 32) {         // element 8 v of the rows
+            const uint4 x = src[v];
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            float4 lo, hi;
+            float2 f;
+            f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[0])); lo.x = f.x; lo.y = f.y;
+            f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[1])); lo.z = f.x; lo.w = f.y;
+            f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[2])); hi.x = f.x; hi.y = f.y;
+            f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[3])); hi.z = f.x; hi.w = f.y;
+            reinterpret_cast<float4 *>(stage)[2 * v] = lo;
+            reinterpret_cast<float4 *>(stage)[2 * v + 1] = hi;
+        }
+    } else {
+        const float4 *src = reinterpret_cast<const float4 *>(at);
+        for (int v = lane; v < G * kD / 4; v += 32) reinterpret_cast<float4 *>(stage)[v] = src[v];
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < 4; r++)
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; g++) {
+            const int gg = g < G ? g : G - 1;          // in bounds; unused when g >= G
+            qv[r][g] = stage[gg * kD + lane + 32 * r];
+        }
+}
+
 // per-query-head search: where unit bh's bonus of centre c of block b goes
 // in its pair's packed table (byte g of the entry, g = bh % kvg)
 __device__ __forceinline__ uint8_t *head_bonus_ptr(const PrepArgs &a, int bh, int b, int c)
@@ -102,6 +147,7 @@ __global__ void __launch_bounds__(kQpThreads) k_query_prep(PrepArgs a)
     __shared__ __align__(16) uint32_t s_occ[kQpWarps][kNC];
     __shared__ float s_x[kD];
     __shared__ uint8_t s_bonus[kQpWarps][kNC];
+    __shared__ __align__(16) float s_qs[kMaxGroup * kD];
 
     if (blockIdx.x == 0) {   // reset the per-call counters of the collision scan and the rerank
         for (int i = tid; i < kBins; i += kQpThreads) a.head_hist[(size_t)bh * kBins + i] = 0u;
@@ -113,10 +159,7 @@ __global__ void __launch_bounds__(kQpThreads) k_query_prep(PrepArgs a)
     if (warp == 0) {
         float qv[4][kMaxGroup];
         const int64_t base = ((int64_t)b_seq * a.H * a.G + (int64_t)h * a.G) * kD;
-        if (a.is_bf16)
-            load_heads(qv, reinterpret_cast<const __nv_bfloat16 *>(a.q) + base, a.G, lane);
-        else
-            load_heads(qv, reinterpret_cast<const float *>(a.q) + base, a.G, lane);
+        load_query(qv, a, base, lane, s_qs);
         float x[4];
 #pragma unroll
         for (int r = 0; r < 4; r++) {
@@ -263,6 +306,7 @@ __global__ void __launch_bounds__(kQwThreads) k_query_prep_wide(PrepArgs a)
     __shared__ float s_x[kD];
     __shared__ uint32_t s_ws[kQwWarps];
     __shared__ uint8_t s_bonus[kQpBlocks][kNC];
+    __shared__ __align__(16) float s_qs[kMaxGroup * kD];
 
     if (blockIdx.x == 0) {   // reset the per-call counters of the collision scan and the rerank
         for (int i = tid; i < kBins; i += kQwThreads) a.head_hist[(size_t)bh * kBins + i] = 0u;
@@ -274,10 +318,7 @@ __global__ void __launch_bounds__(kQwThreads) k_query_prep_wide(PrepArgs a)
     if (warp == 0) {
         float qv[4][kMaxGroup];
         const int64_t base = ((int64_t)b_seq * a.H * a.G + (int64_t)h * a.G) * kD;
-        if (a.is_bf16)
-            load_heads(qv, reinterpret_cast<const __nv_bfloat16 *>(a.q) + base, a.G, lane);
-        else
-            load_heads(qv, reinterpret_cast<const float *>(a.q) + base, a.G, lane);
+        load_query(qv, a, base, lane, s_qs);
         float x[4];
 #pragma unroll
         for (int r = 0; r < 4; r++) {

@@ -454,6 +454,38 @@ def test_attend_heads_union_of_lists(pk, G, topk, kv_location, dtype):
         pk.pk_free(h)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_query_load_paths_agree(pk, dtype):
+    """The query prep and the attention read q with 16-byte loads when its
+    rows start on a 16-byte boundary and one element at a time otherwise
+    (q shifted by one element here): ids, scores and outputs are bit-equal."""
+    batch, H, G, n = 2, 2, 4, 6000
+    w = workloads.llama_layer(batch, n, H=H, G=G, seed=23, device="cuda", dtype=dtype)
+    h = build(pk, w["K"], w["V"], n, batch, H, G)
+    try:
+        q = w["q"][0].contiguous()
+        buf = torch.empty(q.numel() + 8, dtype=dtype, device="cuda")
+        q_odd = buf[1:1 + q.numel()].view_as(q)
+        q_odd.copy_(q)
+        assert q.data_ptr() % 16 == 0 and q_odd.data_ptr() % 16 != 0
+        res = []
+        for qq in (q, q_odd):
+            idx = torch.empty(batch * H, 100, dtype=torch.int32, device="cuda")
+            sc = torch.empty(batch * H, 100, dtype=torch.float32, device="cuda")
+            out = torch.empty(batch, H * G, 128, dtype=torch.float32, device="cuda")
+            pk.pk_search(h, qq, 100, idx, sc)
+            pk.pk_attend(h, qq, idx, 100, out)
+            torch.cuda.synchronize()
+            res.append((idx.cpu(), sc.cpu(), out.cpu()))
+        assert torch.equal(res[0][0], res[1][0])
+        assert torch.equal(res[0][1].view(torch.int32), res[1][1].view(torch.int32))
+        assert torch.equal(res[0][2].view(torch.int32), res[1][2].view(torch.int32))
+        st, det = pk.pk_last_device_error(h)
+        assert st == 0, (st, det)
+    finally:
+        pk.pk_free(h)
+
+
 def test_host_pinned_kv_store(pk):
     """K/V kept in pinned host memory and read through UVA by the attention."""
     w = workloads.llama_layer(1, 20000, H=2, G=4, seed=3, device="cuda")
