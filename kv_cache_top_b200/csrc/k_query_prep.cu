@@ -24,7 +24,10 @@
 // registers -- lane l's word holds the bonus of centre 32 t + l in the 4 bits
 // starting at bit (4 t + r(l)) mod 32, r(l) = (l >> 3) & 3.  With few pairs
 // the SMs have room for more parallelism per block, and k_query_prep_wide
-// (4 warps per block) runs instead; the host chooses.
+// (4 warps per block) runs instead; the host chooses.  For per-query-head
+// search each unit is one query head, and the prep also writes every bonus
+// as byte g of the word (block, centre) of its pair's table, g = the head's
+// index in its group, which the per-head scan copies whole into shared memory.
 #include "pk_internal.cuh"
 
 namespace pk {
