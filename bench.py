@@ -51,6 +51,9 @@ WORKLOADS = {
                   rhos=(0.05, 0.1, 0.2, 0.35, 0.5), queries=8),
     # aggregated vs per-query-head retrieval on the throughput shape
     "heads": dict(name="heads_8x131072", batch=8, n=131072, H=8, G=4, cand=0, kv_host=False, queries=16),
+    # the same with K/V in pinned host memory: the per-head attention gathers
+    # the union of a pair's lists once; timed alone on lists made to overlap
+    "heads_uva": dict(name="heads_uva_8x131072", batch=8, n=131072, H=8, G=4, cand=0, kv_host=True, queries=8),
     # sink / local / update-buffer decoding after an 8 x 131072 prefill
     "longgen": dict(name="longgen_8x131072+1024", batch=8, n=131072, H=8, G=4, cand=0, kv_host=False,
                     steps=1024, sink=64, local=512, update=512),
@@ -606,7 +609,7 @@ def main():
         if world > 1:
             raise SystemExit("the drift mode runs on one GPU")
         return run_drift(args, wl, peak)
-    if args.workload == "heads":
+    if args.workload in ("heads", "heads_uva"):
         if world > 1:
             raise SystemExit("the per-head comparison runs on one GPU")
         return run_heads(args, wl)
@@ -772,7 +775,8 @@ def run_heads(args, wl):
     dev = torch.device("cuda", 0)
     B, n, H, G, nq = wl["batch"], wl["n"], wl["H"], wl["G"], wl["queries"]
     w = workloads.llama_layer(B, n, H=H, G=G, seed=args.seed, device=dev, n_queries=nq)
-    p = pk.pk_default_params(batch=B, n_kv_heads=H, group=G, topk=100, kv_dtype=pk.PK_BF16)
+    p = pk.pk_default_params(batch=B, n_kv_heads=H, group=G, topk=100, kv_dtype=pk.PK_BF16,
+                             kv_location=pk.PK_KV_HOST_PINNED if wl["kv_host"] else pk.PK_KV_DEVICE)
     h = pk.pk_build_index(w["K"], w["V"], n, p)
     BH, U = B * H, B * H * G
     idx_a = torch.empty(BH, 100, dtype=torch.int32, device=dev)
@@ -830,6 +834,29 @@ def run_heads(args, wl):
         return {name: round(ms / nl * 1000.0, 2) for name, (nl, ms) in kern.items() if nl}
 
     kern_a, kern_h = kernels(step_a), kernels(step_h)
+
+    overlap = None
+    if wl["kv_host"]:
+        # pk_attend_heads alone on the heads' own lists, and on lists made to
+        # overlap: heads 1.. of a pair take the first half of head 0's list,
+        # or all of it.  Each distinct row of a pair crosses the host link once.
+        own = []
+        for i in range(nq):
+            pk.pk_search_heads(h, w["q"][i], 100, idx_h)
+            own.append(idx_h.clone())
+
+        def shared(ix, m):
+            v = ix.view(BH, G, 100).clone()
+            v[:, 1:, :m] = v[:, :1, :m]
+            return v.view(U, 100)
+
+        overlap = {}
+        for name, lists in (("own", own), ("half", [shared(x, 50) for x in own]),
+                            ("same", [shared(x, 100) for x in own])):
+            us = 1000.0 * timed(lambda i: pk.pk_attend_heads(h, w["q"][i % nq], lists[i % nq], 100, out))
+            rows = sum(len(set(x[p_ * G:(p_ + 1) * G].flatten().tolist())) for x in lists for p_ in range(BH))
+            overlap[name] = {"attend_us": us, "rows_per_pair": rows / (len(lists) * BH),
+                             "host_bytes_per_call": rows / len(lists) * 2 * 128 * 2}
     pk.pk_free(h)
     print(json.dumps({
         "metric": "Recall@100 against each query head's exact Top-100, and step time: aggregated vs "
@@ -839,9 +866,11 @@ def run_heads(args, wl):
         "per_head": {"recall_at_100": sum(rec_h) / len(rec_h), "ms_per_step": ms_h, "steps_s": 1000.0 / ms_h,
                      "kernel_us": kern_h,
                      "attend_rows_per_pair": {"union": sum(union_rows) / len(union_rows), "lists": G * 100}},
+        "attend_heads_overlap": overlap,
         "data": "synthetic", "dtype": "f32",
         "config": {"workload": wl["name"], "batch": B, "n": n, "kv_heads": H, "q_heads": H * G, "topk": 100,
-                   "queries": nq, "l2": "flushed between steps (outside the events)"}}), flush=True)
+                   "queries": nq, "kv_location": "pinned host (UVA)" if wl["kv_host"] else "hbm",
+                   "l2": "flushed between steps (outside the events)"}}), flush=True)
 
 
 # ------------------------------------------------------ long generation
